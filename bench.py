@@ -1,0 +1,525 @@
+"""Benchmark of the NVFP4 W4A4 linear layer on B200.
+
+One step = one pass of the hot path over one batch: dynamic activation
+global scale (amax), activation quantisation, block-scaled FP4 GEMM with its
+fused epilogue.  Weights are quantised once before timing (offline).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
+
+Prints one JSON line (rank 0).  The default workload is the prefill
+o_proj-shaped projection X[4096,5120] x W[5120,5120].  `--impl reference`
+times the CPU oracle on a bounded row sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "W4A4 GEMM TFLOPS & % dense-FP4 peak; quantize GB/s & % HBM peak (1 B200)"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+FP4_PER_BF16 = 4.0  # nominal dense ratio: 9 PF FP4 / 2.25 PF BF16
+ROTATE = 4          # rotating input sets so consecutive steps miss in L2
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+# --------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        hi = max(sm) if sm else 0
+        loaded = [s for s in sm if s >= 0.5 * hi] or sm
+        return {"sm_mhz": statistics.median(loaded) if loaded else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons, "samples": len(rows)}
+
+
+# --------------------------------------------------------------- distributed
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def dist_init(world):
+    if world <= 1:
+        return None
+    import datetime
+    import torch.distributed as dist
+    dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    return dist
+
+
+def dist_max(dist, value: float, device) -> float:
+    if dist is None:
+        return value
+    import torch
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def dist_barrier(dist):
+    if dist is not None:
+        dist.barrier()
+
+
+# ----------------------------------------------------------------- workloads
+
+def workload_spec(name: str):
+    from bit_quantized_linear_nvfp4_b200 import workloads as wl
+    table = {"oproj": wl.OPROJ, "mlp": wl.MLP, "gdn": wl.GDN, "tiny": wl.TINY,
+             "decode1": wl.DECODE[0], "decode8": wl.DECODE[1], "decode64": wl.DECODE[2]}
+    if name == "quant":
+        return None
+    return table[name]
+
+
+class ProductStep:
+    """Device buffers for ROTATE input sets and CUDA graphs of the two stages."""
+
+    def __init__(self, name: str, device):
+        import torch
+        from bit_quantized_linear_nvfp4_b200 import nvfp4 as nv
+        from bit_quantized_linear_nvfp4_b200 import workloads as wl
+        self.nv, self.torch = nv, torch
+        self.name = name
+        self.device = device
+        self.w = workload_spec(name)
+        if self.w is None:
+            M, K = wl.QUANT_SHAPE
+            x_np = wl.make_quant_input()
+            self.M, self.K, self.N = M, K, 0
+            self.flops = 0.0
+            self.sets = [self._act_set(x_np)]  # 1.14 GB input, larger than L2
+            self.rotate = 1
+            return
+        w = self.w
+        self.M, self.K, self.N = w.M, w.K, w.N
+        self.flops = w.flops()
+        x_np = wl.make_x(w)
+        segs = wl.make_w_segments(w)
+        bounds = np.concatenate([[0], np.cumsum([s.width for s in w.segments])]).astype(np.int64)
+        wdt = torch.float32 if w.dtype == "f32" else torch.bfloat16
+        w_dev = torch.from_numpy(np.concatenate(segs)).to(device).to(wdt)
+        self.W, self.gw = nv.nvfp4_quantize_segments(w_dev, bounds)
+        del w_dev
+        self.a_log = self.dt_bias = None
+        if w.heads:
+            a_log, dt_bias = wl.make_gate_params(w)
+            self.a_log = torch.from_numpy(a_log).to(device)
+            self.dt_bias = torch.from_numpy(dt_bias).to(device)
+        self.bounds = bounds
+        # rotate weights too for the weight-streaming (decode) shapes
+        self.rotate = ROTATE
+        self.wsets = [(self.W, self.gw)]
+        if name.startswith("decode"):
+            for _ in range(ROTATE - 1):
+                Wc = nv.Operand(self.W.codes.clone(), self.W.sf.clone(), self.W.rows, self.W.K)
+                self.wsets.append((Wc, self.gw))
+        self.sets = [self._act_set(x_np) for _ in range(self.rotate)]
+        for i, s in enumerate(self.sets):
+            s["W"], s["gw"] = self.wsets[i % len(self.wsets)]
+            s["segs"] = self._segments(s)
+
+    def _act_set(self, x_np):
+        torch, nv = self.torch, self.nv
+        dt = torch.float32 if (self.w is not None and self.w.dtype == "f32") else torch.bfloat16
+        x = torch.from_numpy(x_np).to(self.device).to(dt)
+        M, K = x.shape
+        s = {
+            "x": x,
+            "codes": torch.empty((M, K // 2), dtype=torch.uint8, device=self.device),
+            "sf": torch.empty(nv.nvfp4_sf_bytes(M, K), dtype=torch.uint8, device=self.device),
+            "g": torch.empty(1, dtype=torch.float32, device=self.device),
+            "ws": torch.empty(nv.nvfp4_quantize_workspace_bytes(1), dtype=torch.uint8, device=self.device),
+        }
+        s["A"] = nv.Operand(s["codes"], s["sf"], M, K)
+        return s
+
+    def _segments(self, s):
+        torch, nv = self.torch, self.nv
+        w = self.w
+        outs, segs = [], []
+        for i, seg in enumerate(w.segments):
+            b0, b1 = int(self.bounds[i]), int(self.bounds[i + 1])
+            if seg.epilogue == "swiglu_up":
+                segs.append(nv.Segment(b0, b1, "swiglu_up"))
+                continue
+            kind = {"identity": "identity_f32" if w.out_dtype == "f32" else "identity_bf16",
+                    "sigmoid": "sigmoid", "gdn_decay": "gdn_decay", "swiglu_gate": "swiglu_gate"}[seg.epilogue]
+            dt = torch.bfloat16 if kind in ("identity_bf16", "swiglu_gate") else torch.float32
+            out = torch.empty((self.M, b1 - b0), dtype=dt, device=self.device)
+            outs.append(out)
+            extra = {}
+            if kind == "gdn_decay":
+                extra = dict(A_log=self.a_log, dt_bias=self.dt_bias)
+            segs.append(nv.Segment(b0, b1, kind, out, **extra))
+        s["outs"] = outs
+        return segs
+
+    # stage launches (all work in libnvfp4)
+    def quantize(self, s):
+        self.nv.nvfp4_quantize(s["x"], codes=s["codes"], sf=s["sf"], g_out=s["g"], workspace=s["ws"])
+
+    def gemm(self, s):
+        self.nv.nvfp4_fused_proj(s["A"], s["g"], s["W"], s["gw"], s["segs"])
+
+    def launches_per_step(self):
+        return 2 if self.w is None else 3  # amax, quantize (+ GEMM)
+
+    def capture(self):
+        torch = self.torch
+        self.gq, self.gg = [], []
+        for s in self.sets:  # warm the launch path once outside capture
+            self.quantize(s)
+            if self.w is not None:
+                self.gemm(s)
+        torch.cuda.synchronize()
+        for s in self.sets:
+            g1 = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g1):
+                self.quantize(s)
+            self.gq.append(g1)
+            if self.w is not None:
+                g2 = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(g2):
+                    self.gemm(s)
+                self.gg.append(g2)
+        torch.cuda.synchronize()
+
+    def alg_bytes_quant(self):
+        # amax pass reads X; the quantiser reads X and writes codes + scales
+        esz = 4 if (self.w is not None and self.w.dtype == "f32") else 2
+        e = self.M * self.K
+        return {"amax": e * esz, "quantize": e * esz + e // 2 + e // 16}
+
+    def alg_bytes_gemm(self):
+        M, N, K = self.M, self.N, self.K
+        out_bytes = 0
+        for seg in self.w.segments:
+            if seg.epilogue in ("identity",):
+                out_bytes += M * seg.width * (4 if self.w.out_dtype == "f32" else 2)
+            elif seg.epilogue in ("sigmoid", "gdn_decay"):
+                out_bytes += M * seg.width * 4
+            elif seg.epilogue == "swiglu_gate":
+                out_bytes += M * seg.width * 2
+        return M * K // 2 + M * K // 16 + N * K // 2 + N * K // 16 + out_bytes
+
+
+def run_product(args):
+    import torch
+    world, rank, local = dist_env()
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    dist = dist_init(world)
+    peaks, peak_src = load_peaks()
+
+    step = ProductStep(args.workload, device)
+    step.capture()
+    stream = torch.cuda.current_stream()
+    K, Wm = args.steps, args.warmup
+    R = len(step.sets)
+
+    def one(i, evs=None):
+        r = i % R
+        if evs is not None:
+            evs[0].record(stream)
+        step.gq[r].replay()
+        if evs is not None:
+            evs[1].record(stream)
+        if step.w is not None:
+            step.gg[r].replay()
+        if evs is not None:
+            evs[2].record(stream)
+
+    for i in range(Wm):
+        one(i)
+    torch.cuda.synchronize()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    dist_barrier(dist)
+    torch.cuda.synchronize()
+    t0.record(stream)
+    for i in range(K):
+        one(i, evs[i])
+    t1.record(stream)
+    torch.cuda.synchronize()
+    dist_barrier(dist)
+    clk = clocks.stop()
+    total_ms = t0.elapsed_time(t1)
+    total_ms = dist_max(dist, total_ms, device)
+    ms_step = total_ms / K
+    q_ms = sum(e[0].elapsed_time(e[1]) for e in evs) / K
+    g_ms = sum(e[1].elapsed_time(e[2]) for e in evs) / K if step.w is not None else 0.0
+    nv = step.nv
+    nv.nvfp4_check()
+
+    # end to end through host buffers: pinned X in, result out, every step
+    e2e = measure_e2e(step, K, Wm, stream)
+
+    qb = step.alg_bytes_quant()
+    hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    kernels = {"quantize_stage_ms": q_ms,
+               "quantize_stage_gbs": (qb["amax"] + qb["quantize"]) / (q_ms * 1e-3) / 1e9,
+               "quantize_stage_frac_hbm": (qb["amax"] + qb["quantize"]) / (q_ms * 1e-3) / 1e9 / hbm}
+    if step.w is not None:
+        fp4_peak = float(peaks["bf16_tflops_sustained"]) * FP4_PER_BF16
+        ach = step.flops / (g_ms * 1e-3) / 1e12
+        roof = {"bound": "tensor", "achieved": ach, "peak": fp4_peak, "unit": "TFLOP/s",
+                "frac": ach / fp4_peak, "traffic": None,
+                "peak_source": f"{peak_src} sustained bf16 x {FP4_PER_BF16:g} (nominal dense FP4/BF16)",
+                "kernel": "nvfp4 gemm (tcgen05 mxf4nvf4)", "ms_per_launch": g_ms,
+                "frac_of_nominal_9pf": ach / 9000.0}
+        kernels["gemm_ms"] = g_ms
+        kernels["gemm_alg_bytes"] = step.alg_bytes_gemm()
+        kernels["gemm_gbs"] = step.alg_bytes_gemm() / (g_ms * 1e-3) / 1e9
+        value = step.flops * world / (ms_step * 1e-3) / 1e12
+        unit = "TFLOP/s"
+    else:
+        bytes_step = qb["amax"] + qb["quantize"]
+        ach = bytes_step / (q_ms * 1e-3) / 1e9
+        roof = {"bound": "hbm", "achieved": ach, "peak": hbm, "unit": "GB/s", "frac": ach / hbm,
+                "traffic": None, "peak_source": f"{peak_src} copy bandwidth",
+                "kernel": "nvfp4 amax + quantize", "ms_per_launch": q_ms}
+        value = bytes_step * world / (ms_step * 1e-3) / 1e9
+        unit = "GB/s"
+
+    line = {
+        "metric": METRIC, "value": value, "unit": unit, "n_gpus": world, "steps": K, "warmup": Wm,
+        "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "nvfp4", "data": "synthetic (seeded N(0,1) activations with outlier channels, N(0,0.02) weights)",
+        "config": {"workload": step.name if step.w is None else step.w.name, "M": step.M, "N": step.N, "K": step.K,
+                   "parallelism": "replicas" if world > 1 else "single",
+                   "l2": f"{R} rotating input sets, {'weights rotated too, ' if args.workload.startswith('decode') else ''}"
+                         "working set above the 126 MB L2" if R > 1 else "input larger than L2"},
+        "roofline": roof, "kernels": kernels, "clocks": clk, "e2e": e2e,
+        "gpu_launches": step.launches_per_step() * K,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(args.workload, target_s=args.cpu_seconds)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    for g in step.gq + step.gg:
+        del g
+    if dist is not None:
+        dist.destroy_process_group()
+
+
+def measure_e2e(step, K, Wm, stream):
+    import torch
+    s = step.sets[0]
+    x_host = s["x"].cpu().pin_memory()
+    outs = s.get("outs") or [s["codes"]]
+    out_host = [o.cpu().pin_memory() for o in outs]
+    h2d = x_host.numel() * x_host.element_size()
+    d2h = sum(o.numel() * o.element_size() for o in out_host)
+
+    def one():
+        s["x"].copy_(x_host, non_blocking=True)
+        step.gq[0].replay()
+        if step.w is not None:
+            step.gg[0].replay()
+        for dst, src in zip(out_host, outs):
+            dst.copy_(src, non_blocking=True)
+
+    for _ in range(Wm):
+        one()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(K):
+        one()
+    b.record(stream)
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b) / K
+    if step.w is not None:
+        val, unit = step.flops / (ms * 1e-3) / 1e12, "TFLOP/s"
+    else:
+        qb = step.alg_bytes_quant()
+        val, unit = (qb["amax"] + qb["quantize"]) / (ms * 1e-3) / 1e9, "GB/s"
+    return {"value": val, "unit": unit, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+            "ms_per_step": ms}
+
+
+# ------------------------------------------------------------- CPU oracle
+
+def _oracle_sample_step(name, rows, x_np, wq, g_a, extra):
+    """One oracle pass over `rows` rows of the workload: quantise the rows,
+    FP64 GEMM against the pre-quantised weights, epilogues."""
+    from oracle import nvfp4_oracle as o
+    aq = o.quantize(x_np[:rows], g_a)
+    if wq is None:
+        return
+    w, segs_q, scales, epis, gate = extra
+    o.fused_projection(aq, segs_q, scales, epis, gate)
+
+
+def _prepare_oracle(name):
+    from bit_quantized_linear_nvfp4_b200 import workloads as wl
+    from oracle import nvfp4_oracle as o
+    w = workload_spec(name)
+    if w is None:
+        x = wl.make_quant_input(rows=2048)
+        return None, x, None, o.global_scale(x), None
+    x = wl.make_x(w, rows=min(w.M, 4096))
+    g_a = o.global_scale(x)
+    segs = wl.make_w_segments(w)
+    wq = [o.quantize(s) for s in segs]
+    gate = wl.make_gate_params(w) if w.heads else None
+    extra = (w, [(c, s) for c, s, _ in wq], [g for _, _, g in wq], [s.epilogue for s in w.segments], gate)
+    return w, x, wq, g_a, extra
+
+
+def _blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def cpu_baseline(name, target_s=12.0, steps=None):
+    """Time the oracle as it stands on a bounded row sample; throughput in the
+    bench's unit scaled by the rows processed."""
+    w, x, wq, g_a, extra = _prepare_oracle(name)
+    K = x.shape[1]
+    rows = 8
+    t = time.perf_counter()
+    _oracle_sample_step(name, rows, x, wq, g_a, extra)
+    dt = max(time.perf_counter() - t, 1e-3)
+    rows = int(min(x.shape[0], max(8, rows * (target_s / 2) / dt)))
+    t = time.perf_counter()
+    n = 0
+    while True:
+        _oracle_sample_step(name, rows, x, wq, g_a, extra)
+        n += 1
+        el = time.perf_counter() - t
+        if el >= target_s * 0.5 or n >= 4:
+            break
+    per = el / n
+    if w is not None:
+        val = 2.0 * rows * w.N * K / per / 1e12
+        unit = "TFLOP/s"
+    else:
+        val = rows * K * (2 + 2 + 0.5 + 0.0625) / per / 1e9
+        unit = "GB/s"
+    return {"value": val, "unit": unit, "cores": _blas_threads(), "kind": "oracle",
+            "sample": f"{rows} rows of the workload per pass ({n} passes, {el:.1f} s): quantise rows + FP64 GEMM + epilogue"
+                      if w is not None else f"{rows} rows x {K} per pass ({n} passes): amax + quantise",
+            "host_cpus": os.cpu_count()}
+
+
+def run_reference(args):
+    world, rank, _ = dist_env()
+    if rank != 0:
+        return
+    w, x, wq, g_a, extra = _prepare_oracle(args.workload)
+    K = x.shape[1]
+    rows = 16
+    for _ in range(args.warmup):
+        _oracle_sample_step(args.workload, rows, x, wq, g_a, extra)
+    t = time.perf_counter()
+    for _ in range(args.steps):
+        _oracle_sample_step(args.workload, rows, x, wq, g_a, extra)
+    el = time.perf_counter() - t
+    per = el / args.steps
+    if w is not None:
+        val, unit = 2.0 * rows * w.N * K / per / 1e12, "TFLOP/s"
+        cfg = {"workload": w.name, "M": w.M, "N": w.N, "K": w.K}
+    else:
+        val, unit = rows * K * 4.5625 / per / 1e9, "GB/s"
+        cfg = {"workload": "quant", "M": x.shape[0], "K": K}
+    sample = f"{rows} rows of the workload per step (quantise + FP64 GEMM + epilogue)"
+    line = {"impl": "reference", "metric": METRIC, "value": val, "unit": unit, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": per * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64 (oracle)", "data": "synthetic",
+            "config": cfg,
+            "cpu_baseline": {"value": val, "unit": unit, "cores": _blas_threads(), "kind": "oracle", "sample": sample},
+            "e2e": {"value": val, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="oproj",
+                    choices=["oproj", "mlp", "gdn", "tiny", "decode1", "decode8", "decode64", "quant"])
+    ap.add_argument("--impl", default="product", choices=["product", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_product(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,240 @@
+// extern "C" entry points of libnvfp4 (declared in include/nvfp4.h): host-side
+// argument checks, then the launches.  No entry point allocates device memory,
+// synchronises (except nvfp4_check) or aborts.
+#include <cstdint>
+#include <cstring>
+
+#include <cuda_runtime.h>
+
+#include "internal.h"
+#include "ptx.cuh"
+
+namespace {
+
+thread_local int t_last_cuda_error = 0;
+
+int cuda_fail(cudaError_t e) {
+  t_last_cuda_error = static_cast<int>(e);
+  return NVFP4_ERR_CUDA;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int check_device() {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e);
+  int major = 0, minor = 0;
+  cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+  cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
+  if (major != 10 || minor != 0) return NVFP4_ERR_DEVICE;
+  return NVFP4_OK;
+}
+
+int check_quant_args(const void* x, int dtype, int64_t M, int64_t K, int64_t ld, float* g_out,
+                     uint8_t* codes, uint8_t* sf) {
+  if (dtype != NVFP4_DTYPE_BF16 && dtype != NVFP4_DTYPE_F32) return NVFP4_ERR_INVALID_ARG;
+  if (M < 0 || K <= 0 || g_out == nullptr) return NVFP4_ERR_INVALID_ARG;
+  if (K % 16 != 0) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+  if (M > (int64_t(1) << 31) || K > (int64_t(1) << 30)) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+  if (M == 0) return NVFP4_OK;
+  if (x == nullptr || codes == nullptr || sf == nullptr) return NVFP4_ERR_INVALID_ARG;
+  if (ld < K) return NVFP4_ERR_INVALID_ARG;
+  const int esz = dtype == NVFP4_DTYPE_BF16 ? 2 : 4;
+  if (!aligned16(x) || (ld * esz) % 16 != 0) return NVFP4_ERR_MISALIGNED;
+  if (!aligned16(codes) || !aligned16(sf) || (K / 2) % 4 != 0) return NVFP4_ERR_MISALIGNED;
+  if ((reinterpret_cast<uintptr_t>(g_out) & 3u) != 0) return NVFP4_ERR_MISALIGNED;
+  return NVFP4_OK;
+}
+
+int quantize_impl(const void* x, int dtype, int64_t M, int64_t K, int64_t ld,
+                  const nvfp4::RowSegments& segs, const float* g_in, float* g_out, uint8_t* codes,
+                  uint8_t* sf, void* ws, size_t ws_bytes, void* stream) {
+  int st = check_quant_args(x, dtype, M, K, ld, g_out, codes, sf);
+  if (st != NVFP4_OK) return st;
+  if (g_in == nullptr && (ws == nullptr || ws_bytes < nvfp4_quantize_workspace_bytes(segs.n) ||
+                          !aligned16(ws)))
+    return NVFP4_ERR_WORKSPACE;
+  st = check_device();
+  if (st != NVFP4_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  unsigned int* bits = static_cast<unsigned int*>(ws);
+  if (g_in == nullptr) {
+    cudaError_t e = nvfp4::launch_amax(x, dtype, K, ld, segs, bits, s);
+    if (e != cudaSuccess) return cuda_fail(e);
+  }
+  cudaError_t e = nvfp4::launch_quantize(x, dtype, M, K, ld, segs, g_in, bits, g_out, codes, sf, s);
+  if (e != cudaSuccess) return cuda_fail(e);
+  return NVFP4_OK;
+}
+
+int check_operand(const nvfp4_operand* o) {
+  if (o == nullptr || o->codes == nullptr || o->sf == nullptr) return NVFP4_ERR_INVALID_ARG;
+  if (o->rows <= 0 || o->K <= 0) return NVFP4_ERR_INVALID_ARG;
+  if (o->K % 32 != 0) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+  if (o->rows > (int64_t(1) << 31) || o->K > (int64_t(1) << 30)) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+  if (!aligned16(o->codes) || !aligned16(o->sf)) return NVFP4_ERR_MISALIGNED;
+  return NVFP4_OK;
+}
+
+bool epi_is_bf16(int kind) { return kind == NVFP4_EPI_IDENTITY_BF16 || kind == NVFP4_EPI_SWIGLU_GATE; }
+
+}  // namespace
+
+extern "C" {
+
+const char* nvfp4_status_string(int status) {
+  switch (status) {
+    case NVFP4_OK: return "ok";
+    case NVFP4_ERR_INVALID_ARG: return "invalid argument";
+    case NVFP4_ERR_UNSUPPORTED_SHAPE: return "unsupported shape";
+    case NVFP4_ERR_MISALIGNED: return "misaligned pointer or leading dimension";
+    case NVFP4_ERR_CUDA: return "CUDA error";
+    case NVFP4_ERR_DEVICE_TIMEOUT: return "device-side wait timed out";
+    case NVFP4_ERR_WORKSPACE: return "workspace missing or too small";
+    case NVFP4_ERR_DEVICE: return "device is not compute capability 10.0";
+    default: return "unknown status";
+  }
+}
+
+int nvfp4_last_cuda_error(void) { return t_last_cuda_error; }
+
+size_t nvfp4_sf_bytes(int64_t rows, int64_t K) {
+  if (rows <= 0 || K <= 0) return 0;
+  return nvfp4::sf_bytes(rows, K);
+}
+
+size_t nvfp4_quantize_workspace_bytes(int nseg) {
+  if (nseg < 1) nseg = 1;
+  return 16 * static_cast<size_t>((nseg * 4 + 15) / 16);
+}
+
+int nvfp4_quantize(const void* x, int x_dtype, int64_t M, int64_t K, int64_t ld_x,
+                   const float* g_in, float* g_out, uint8_t* codes, uint8_t* sf, void* workspace,
+                   size_t workspace_bytes, void* stream) {
+  nvfp4::RowSegments segs{};
+  segs.n = 1;
+  segs.begin[0] = 0;
+  segs.begin[1] = M;
+  return quantize_impl(x, x_dtype, M, K, ld_x, segs, g_in, g_out, codes, sf, workspace,
+                       workspace_bytes, stream);
+}
+
+int nvfp4_quantize_segments(const void* w, int w_dtype, int64_t N, int64_t K, int64_t ld_w,
+                            const int64_t* row_bounds, int nseg, const float* g_in, float* g_out,
+                            uint8_t* codes, uint8_t* sf, void* workspace, size_t workspace_bytes,
+                            void* stream) {
+  if (row_bounds == nullptr || nseg < 1 || nseg > NVFP4_MAX_SEGMENTS) return NVFP4_ERR_INVALID_ARG;
+  if (row_bounds[0] != 0 || row_bounds[nseg] != N) return NVFP4_ERR_INVALID_ARG;
+  nvfp4::RowSegments segs{};
+  segs.n = nseg;
+  for (int i = 0; i <= nseg; ++i) {
+    if (i > 0 && row_bounds[i] <= row_bounds[i - 1]) return NVFP4_ERR_INVALID_ARG;
+    segs.begin[i] = row_bounds[i];
+  }
+  return quantize_impl(w, w_dtype, N, K, ld_w, segs, g_in, g_out, codes, sf, workspace,
+                       workspace_bytes, stream);
+}
+
+size_t nvfp4_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K) {
+  return nvfp4::gemm_workspace_bytes(M, N, K);
+}
+
+int nvfp4_fused_proj(const nvfp4_operand* A, const float* g_a, const nvfp4_operand* W,
+                     const float* seg_global_scale, const nvfp4_segment* segs, int nseg,
+                     void* workspace, size_t workspace_bytes, void* stream) {
+  int st = check_operand(A);
+  if (st != NVFP4_OK) return st;
+  st = check_operand(W);
+  if (st != NVFP4_OK) return st;
+  if (A->K != W->K) return NVFP4_ERR_INVALID_ARG;
+  if (g_a == nullptr || seg_global_scale == nullptr || segs == nullptr) return NVFP4_ERR_INVALID_ARG;
+  if (nseg < 1 || nseg > NVFP4_MAX_SEGMENTS) return NVFP4_ERR_INVALID_ARG;
+
+  nvfp4::GemmProblem p{};
+  p.a_codes = A->codes;
+  p.a_sf = A->sf;
+  p.w_codes = W->codes;
+  p.w_sf = W->sf;
+  p.M = A->rows;
+  p.N = W->rows;
+  p.K = A->K;
+  p.g_a = g_a;
+  p.seg_scale = seg_global_scale;
+  p.nseg = nseg;
+  int n_swiglu = 0;
+  for (int i = 0; i < nseg; ++i) {
+    const nvfp4_segment& s = segs[i];
+    const int64_t expect_begin = i == 0 ? 0 : segs[i - 1].n_end;
+    if (s.n_begin != expect_begin || s.n_end <= s.n_begin) return NVFP4_ERR_INVALID_ARG;
+    if (s.epilogue < NVFP4_EPI_IDENTITY_BF16 || s.epilogue > NVFP4_EPI_SWIGLU_UP || s.reserved != 0)
+      return NVFP4_ERR_INVALID_ARG;
+    const int64_t width = s.n_end - s.n_begin;
+    if (s.epilogue == NVFP4_EPI_SWIGLU_GATE || s.epilogue == NVFP4_EPI_SWIGLU_UP) ++n_swiglu;
+    if (s.epilogue != NVFP4_EPI_SWIGLU_UP) {
+      if (s.out == nullptr) return NVFP4_ERR_INVALID_ARG;
+      if (!aligned16(s.out)) return NVFP4_ERR_MISALIGNED;
+      const int64_t vec = epi_is_bf16(s.epilogue) ? 8 : 4;
+      if (s.ld_out < width || s.ld_out % vec != 0) return NVFP4_ERR_MISALIGNED;
+    }
+    if (s.epilogue == NVFP4_EPI_GDN_DECAY_F32) {
+      if (s.A_log == nullptr || s.dt_bias == nullptr) return NVFP4_ERR_INVALID_ARG;
+    }
+    nvfp4::EpiSegment& e = p.seg[i];
+    e.n_begin = s.n_begin;
+    e.n_end = s.n_end;
+    e.kind = s.epilogue;
+    e.scale_index = i;
+    e.out = s.out;
+    e.ld_out = s.ld_out;
+    e.a_log = s.A_log;
+    e.dt_bias = s.dt_bias;
+  }
+  if (segs[nseg - 1].n_end != W->rows) return NVFP4_ERR_INVALID_ARG;
+  if (n_swiglu != 0) {
+    if (nseg != 2 || segs[0].epilogue != NVFP4_EPI_SWIGLU_GATE ||
+        segs[1].epilogue != NVFP4_EPI_SWIGLU_UP)
+      return NVFP4_ERR_INVALID_ARG;
+    if (segs[0].n_end * 2 != W->rows) return NVFP4_ERR_INVALID_ARG;
+    if (segs[0].n_end % 128 != 0) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    p.swiglu = true;
+  }
+  if (workspace_bytes < nvfp4::gemm_workspace_bytes(p.M, p.N, p.K) ||
+      (nvfp4::gemm_workspace_bytes(p.M, p.N, p.K) > 0 && workspace == nullptr))
+    return NVFP4_ERR_WORKSPACE;
+  st = check_device();
+  if (st != NVFP4_OK) return st;
+  cudaError_t e = nvfp4::launch_gemm(p, workspace, workspace_bytes, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e);
+  return NVFP4_OK;
+}
+
+int nvfp4_gemm(const nvfp4_operand* A, const float* g_a, const nvfp4_operand* W, const float* g_w,
+               void* out, int out_dtype, int64_t ld_out, void* workspace, size_t workspace_bytes,
+               void* stream) {
+  if (W == nullptr) return NVFP4_ERR_INVALID_ARG;
+  if (out_dtype != NVFP4_DTYPE_BF16 && out_dtype != NVFP4_DTYPE_F32) return NVFP4_ERR_INVALID_ARG;
+  nvfp4_segment seg{};
+  seg.n_begin = 0;
+  seg.n_end = W->rows;
+  seg.epilogue = out_dtype == NVFP4_DTYPE_BF16 ? NVFP4_EPI_IDENTITY_BF16 : NVFP4_EPI_IDENTITY_F32;
+  seg.out = out;
+  seg.ld_out = ld_out;
+  return nvfp4_fused_proj(A, g_a, W, g_w, &seg, 1, workspace, workspace_bytes, stream);
+}
+
+int nvfp4_check(void* stream) {
+  cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e);
+  unsigned int flag = 0, zero = 0;
+  e = cudaMemcpyFromSymbol(&flag, nvfp4::g_device_error, sizeof(flag));
+  if (e != cudaSuccess) return cuda_fail(e);
+  if (flag != 0) {
+    e = cudaMemcpyToSymbol(nvfp4::g_device_error, &zero, sizeof(zero));
+    if (e != cudaSuccess) return cuda_fail(e);
+    return NVFP4_ERR_DEVICE_TIMEOUT;
+  }
+  return NVFP4_OK;
+}
+
+}  // extern "C"

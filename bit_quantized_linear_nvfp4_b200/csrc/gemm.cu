@@ -1,0 +1,472 @@
+// Block-scaled NVFP4 x NVFP4 GEMM with fused per-segment epilogues, sm_100a.
+//
+// Computes acc[m, n] = sum_k e2m1(a[m,k]) Sa[m,k/16] * e2m1(w[n,k]) Sw[n,k/16]
+// in FP32 on the 5th-generation tensor cores ("Why Gated DeltaNet Survives
+// 4-Bit Quantization", ai.info summary, "Methodology in Plain English": W4A4,
+// E2M1 values with one E4M3 scale per 16 elements), then, per output column n
+// of segment s, y = acc * g_a * g_w[s] ("Main Findings", fused-GEMM scaling
+// bullet: each fused module keeps its own global scale) followed by the
+// segment's epilogue (identity, sigmoid write strength, log-space decay
+// -exp(A_log) * softplus(y + dt_bias), or SwiGLU; "Main Findings",
+// gate-parameterisation bullets).
+//
+// Kernel shape: persistent, one CTA per SM, 320 threads.
+//   warp 0      TMA producer: codes (128-byte swizzle) and scale atoms -> smem
+//   warp 1      allocates TMEM; one lane issues tcgen05.cp (scales -> TMEM)
+//               and tcgen05.mma ... kind::mxf4nvf4.block_scale into TMEM
+//   warps 2..9  epilogue: tcgen05.ld TMEM -> registers, release TMEM, then
+//               scale, nonlinearity, store
+// Tile 128 x 256 (M x N), 256 K-elements (128 bytes per row) per stage,
+// 4 stages.  Each stage is 4 MMAs of K = 64.
+#include <cfloat>
+#include <cstdint>
+#include <cstdio>
+#include <mutex>
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "internal.h"
+#include "ptx.cuh"
+
+namespace nvfp4 {
+namespace gk {
+
+constexpr int BM = 128;
+constexpr int BN = 256;
+constexpr int BK = 256;
+constexpr int kStages = 4;
+constexpr int kABytes = BM * BK / 2;     // 16 KB
+constexpr int kBBytes = BN * BK / 2;     // 32 KB
+constexpr int kSFABytes = BM * BK / 16;  // 2 KB
+constexpr int kSFBBytes = BN * BK / 16;  // 4 KB
+constexpr int kStageBytes = kABytes + kBBytes + kSFABytes + kSFBBytes;
+constexpr int kNumEpiWarps = 8;
+constexpr int kThreads = 64 + kNumEpiWarps * 32;
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kColAcc = 0, kColSFA = 256, kColSFB = 272;
+constexpr int kSmemBytes = kStages * kStageBytes + 1024 /*align*/ + 256 /*barriers*/;
+static_assert(kStageBytes % 1024 == 0, "stage buffers keep 1024-byte alignment");
+
+struct KernelArgs {
+  int64_t M, N, K;
+  int num_m_blocks, num_n_blocks, num_k_stages, group_m;
+  int swiglu;
+  int64_t up_row0;  // SwiGLU: first W row of the up half
+  int64_t n_out;    // SwiGLU: output width (= N / 2)
+  const float* g_a;
+  const float* seg_scale;
+  int nseg;
+  EpiSegment seg[kMaxSeg];
+};
+
+struct SharedTail {
+  uint64_t full[kStages];
+  uint64_t empty[kStages];
+  uint64_t tmem_full;
+  uint64_t tmem_empty;
+  uint64_t drain;
+  uint32_t tmem_base;
+  int abort_flag;
+};
+
+__device__ __forceinline__ void tile_coords(const KernelArgs& a, int t, int& m_blk, int& n_blk) {
+  const int per_group = a.group_m * a.num_n_blocks;
+  const int grp = t / per_group;
+  const int first_m = grp * a.group_m;
+  int gm = a.num_m_blocks - first_m;
+  if (gm > a.group_m) gm = a.group_m;
+  const int r = t - grp * per_group;
+  m_blk = first_m + r % gm;
+  n_blk = r / gm;
+}
+
+__device__ __forceinline__ float sigmoid_f(float y) { return 1.0f / (1.0f + expf(-y)); }
+__device__ __forceinline__ float softplus_f(float t) {
+  return t > 0.0f ? t + log1pf(expf(-t)) : log1pf(expf(t));
+}
+
+__device__ __forceinline__ int seg_of(const KernelArgs& a, int64_t n) {
+  int s = 0;
+#pragma unroll
+  for (int i = 1; i < kMaxSeg; ++i)
+    if (i < a.nseg && n >= a.seg[i].n_begin) s = i;
+  return s;
+}
+
+__device__ __forceinline__ float apply_epi(const EpiSegment& sg, float y, int64_t j) {
+  switch (sg.kind) {
+    case NVFP4_EPI_SIGMOID_F32:
+      return sigmoid_f(y);
+    case NVFP4_EPI_GDN_DECAY_F32:
+      return -expf(__ldg(sg.a_log + j)) * softplus_f(y + __ldg(sg.dt_bias + j));
+    default:
+      return y;
+  }
+}
+
+__device__ __forceinline__ bool epi_is_bf16(int kind) {
+  return kind == NVFP4_EPI_IDENTITY_BF16 || kind == NVFP4_EPI_SWIGLU_GATE;
+}
+
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+  const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t*>(&v);
+}
+
+// Store 32 consecutive results of one row: columns n0 .. n0+31 (absolute W row index).
+__device__ __forceinline__ void store_chunk(const KernelArgs& a, int64_t row, int64_t n0,
+                                           const uint32_t (&r)[32]) {
+  if (n0 >= a.N) return;
+  const int s = seg_of(a, n0);
+  const EpiSegment& sg = a.seg[s];
+  const int64_t n_last = n0 + 31;
+  const bool bf16 = epi_is_bf16(sg.kind);
+  const int vec = bf16 ? 8 : 4;
+  const bool uniform = n_last < sg.n_end && ((n0 - sg.n_begin) % vec) == 0;
+  if (uniform) {
+    const float scale = __ldg(a.g_a) * __ldg(a.seg_scale + s);
+    const int64_t j0 = n0 - sg.n_begin;
+    if (bf16) {
+      __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(sg.out) + row * sg.ld_out + j0;
+#pragma unroll
+      for (int v = 0; v < 4; ++v) {
+        uint4 w;
+        w.x = pack_bf16(__uint_as_float(r[8 * v + 0]) * scale, __uint_as_float(r[8 * v + 1]) * scale);
+        w.y = pack_bf16(__uint_as_float(r[8 * v + 2]) * scale, __uint_as_float(r[8 * v + 3]) * scale);
+        w.z = pack_bf16(__uint_as_float(r[8 * v + 4]) * scale, __uint_as_float(r[8 * v + 5]) * scale);
+        w.w = pack_bf16(__uint_as_float(r[8 * v + 6]) * scale, __uint_as_float(r[8 * v + 7]) * scale);
+        *reinterpret_cast<uint4*>(dst + 8 * v) = w;
+      }
+    } else {
+      float* dst = static_cast<float*>(sg.out) + row * sg.ld_out + j0;
+#pragma unroll
+      for (int v = 0; v < 8; ++v) {
+        float4 w;
+        w.x = apply_epi(sg, __uint_as_float(r[4 * v + 0]) * scale, j0 + 4 * v + 0);
+        w.y = apply_epi(sg, __uint_as_float(r[4 * v + 1]) * scale, j0 + 4 * v + 1);
+        w.z = apply_epi(sg, __uint_as_float(r[4 * v + 2]) * scale, j0 + 4 * v + 2);
+        w.w = apply_epi(sg, __uint_as_float(r[4 * v + 3]) * scale, j0 + 4 * v + 3);
+        *reinterpret_cast<float4*>(dst + 4 * v) = w;
+      }
+    }
+    return;
+  }
+  // general path: column by column (segment boundaries, N tail, odd alignment)
+  const float ga = __ldg(a.g_a);
+#pragma unroll
+  for (int j = 0; j < 32; ++j) {
+    const int64_t n = n0 + j;
+    if (n >= a.N) continue;
+    const int sj = seg_of(a, n);
+    const EpiSegment& q = a.seg[sj];
+    const float y = __uint_as_float(r[j]) * (ga * __ldg(a.seg_scale + sj));
+    const int64_t jj = n - q.n_begin;
+    if (epi_is_bf16(q.kind))
+      static_cast<__nv_bfloat16*>(q.out)[row * q.ld_out + jj] = __float2bfloat16_rn(y);
+    else
+      static_cast<float*>(q.out)[row * q.ld_out + jj] = apply_epi(q, y, jj);
+  }
+}
+
+// SwiGLU: output columns o0 .. o0+31 from gate values rg and up values ru.
+__device__ __forceinline__ void store_swiglu(const KernelArgs& a, int64_t row, int64_t o0,
+                                             const uint32_t (&rg)[32], const uint32_t (&ru)[32]) {
+  if (o0 >= a.n_out) return;
+  const EpiSegment& sg = a.seg[0];
+  const float ga = __ldg(a.g_a);
+  const float sgate = ga * __ldg(a.seg_scale + 0);
+  const float sup = ga * __ldg(a.seg_scale + 1);
+  float v[32];
+#pragma unroll
+  for (int j = 0; j < 32; ++j) {
+    const float gv = __uint_as_float(rg[j]) * sgate;
+    const float uv = __uint_as_float(ru[j]) * sup;
+    v[j] = gv / (1.0f + expf(-gv)) * uv;
+  }
+  __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(sg.out) + row * sg.ld_out + o0;
+  if (o0 + 31 < a.n_out && (o0 % 8) == 0) {
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      uint4 w;
+      w.x = pack_bf16(v[8 * q + 0], v[8 * q + 1]);
+      w.y = pack_bf16(v[8 * q + 2], v[8 * q + 3]);
+      w.z = pack_bf16(v[8 * q + 4], v[8 * q + 5]);
+      w.w = pack_bf16(v[8 * q + 6], v[8 * q + 7]);
+      *reinterpret_cast<uint4*>(dst + 8 * q) = w;
+    }
+  } else {
+#pragma unroll
+    for (int j = 0; j < 32; ++j)
+      if (o0 + j < a.n_out) dst[j] = __float2bfloat16_rn(v[j]);
+  }
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
+                const __grid_constant__ CUtensorMap tm_sfa, const __grid_constant__ CUtensorMap tm_sfb,
+                const __grid_constant__ KernelArgs args) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  SharedTail* tail = reinterpret_cast<SharedTail*>(smem + kStages * kStageBytes);
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int num_tiles = args.num_m_blocks * args.num_n_blocks;
+  volatile int* abort_flag = &tail->abort_flag;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&tail->full[s], 1);
+      mbar_init(&tail->empty[s], 1);
+    }
+    mbar_init(&tail->tmem_full, 1);
+    mbar_init(&tail->tmem_empty, kNumEpiWarps);
+    mbar_init(&tail->drain, 1);
+    tail->abort_flag = 0;
+    fence_mbarrier_init();
+    prefetch_tmap(&tm_a);
+    prefetch_tmap(&tm_b);
+    prefetch_tmap(&tm_sfa);
+    prefetch_tmap(&tm_sfb);
+  }
+  if (warp == 1) {
+    tmem_alloc(&tail->tmem_base, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tail->tmem_base;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (elect_one()) {
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t issued_phase[kStages];
+      bool issued[kStages];
+      for (int s = 0; s < kStages; ++s) issued[s] = false;
+      bool ok = true;
+      for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
+        int m_blk, n_blk;
+        tile_coords(args, t, m_blk, n_blk);
+        const int64_t b_row0 = args.swiglu ? static_cast<int64_t>(n_blk) * 128 : static_cast<int64_t>(n_blk) * BN;
+        const int64_t b_row1 = args.swiglu ? args.up_row0 + static_cast<int64_t>(n_blk) * 128 : b_row0 + 128;
+        for (int ks = 0; ks < args.num_k_stages; ++ks) {
+          if (!mbar_wait_bounded(&tail->empty[stage], phase ^ 1u, abort_flag)) { ok = false; break; }
+          uint8_t* st = smem + stage * kStageBytes;
+          mbar_arrive_expect_tx(&tail->full[stage], kStageBytes);
+          const int32_t kx = ks * (BK / 2);
+          tma_load_2d(st, &tm_a, &tail->full[stage], kx, m_blk * BM);
+          tma_load_2d(st + kABytes, &tm_b, &tail->full[stage], kx, static_cast<int32_t>(b_row0));
+          tma_load_2d(st + kABytes + kBBytes / 2, &tm_b, &tail->full[stage], kx, static_cast<int32_t>(b_row1));
+          uint8_t* sfa = st + kABytes + kBBytes;
+          uint8_t* sfb = sfa + kSFABytes;
+          tma_load_3d(sfa, &tm_sfa, &tail->full[stage], 0, ks * 4, m_blk);
+          tma_load_3d(sfb, &tm_sfb, &tail->full[stage], 0, ks * 4, static_cast<int32_t>(b_row0 / 128));
+          tma_load_3d(sfb + kSFBBytes / 2, &tm_sfb, &tail->full[stage], 0, ks * 4, static_cast<int32_t>(b_row1 / 128));
+          issued[stage] = true;
+          issued_phase[stage] = phase;
+          if (++stage == kStages) { stage = 0; phase ^= 1u; }
+        }
+      }
+      if (*abort_flag) {
+        // let copies already in flight land before the CTA leaves
+        for (int s = 0; s < kStages; ++s)
+          if (issued[s]) mbar_wait_bounded(&tail->full[s], issued_phase[s], nullptr, 200000000ull);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (elect_one()) {
+      // instruction descriptor: E2M1 x E2M1, UE4M3 scales, K-major A and B, M=128, N=256
+      const uint32_t idesc = (1u << 7) | (1u << 10) | (static_cast<uint32_t>(BN >> 3) << 17) |
+                             (static_cast<uint32_t>(BM >> 4) << 24);
+      const uint32_t base = smem_u32(smem);
+      int stage = 0;
+      uint32_t phase = 0;
+      int local = 0;
+      bool ok = true;
+      bool any_issued = false;
+      for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x, ++local) {
+        if (local > 0) {
+          if (!mbar_wait_bounded(&tail->tmem_empty, (local - 1) & 1, abort_flag)) { ok = false; break; }
+        }
+        tc_fence_after();
+        for (int ks = 0; ks < args.num_k_stages; ++ks) {
+          if (!mbar_wait_bounded(&tail->full[stage], phase, abort_flag)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t sa = base + stage * kStageBytes;
+          const uint32_t sb = sa + kABytes;
+          const uint32_t ssfa = sb + kBBytes;
+          const uint32_t ssfb = ssfa + kSFABytes;
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            tmem_cp_32x128b_warpx4(tmem + kColSFA + 4 * j, make_smem_desc(ssfa + 512 * j, 0, 128, kLayoutSwizzleNone));
+            tmem_cp_32x128b_warpx4(tmem + kColSFB + 8 * j, make_smem_desc(ssfb + 512 * j, 0, 128, kLayoutSwizzleNone));
+            tmem_cp_32x128b_warpx4(tmem + kColSFB + 8 * j + 4,
+                                   make_smem_desc(ssfb + kSFBBytes / 2 + 512 * j, 0, 128, kLayoutSwizzleNone));
+          }
+          const uint64_t adesc = make_smem_desc(sa, 16, 1024, kLayoutSwizzle128B);
+          const uint64_t bdesc = make_smem_desc(sb, 16, 1024, kLayoutSwizzle128B);
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            // advance the start address by j * 32 bytes (64 FP4 elements) inside the swizzle atom
+            mma_mxf4nvf4(tmem + kColAcc, adesc + 2 * j, bdesc + 2 * j, idesc, tmem + kColSFA + 4 * j,
+                         tmem + kColSFB + 8 * j, (ks | j) != 0 ? 1u : 0u);
+          }
+          any_issued = true;
+          tc_commit(&tail->empty[stage]);
+          if (++stage == kStages) { stage = 0; phase ^= 1u; }
+        }
+        if (!ok) break;
+        tc_commit(&tail->tmem_full);
+      }
+      if (*abort_flag && any_issued) {
+        tc_commit(&tail->drain);
+        mbar_wait_bounded(&tail->drain, 0, nullptr, 200000000ull);
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int q = warp & 3;            // TMEM lane quadrant this warp may read
+    const int h = (warp - 2) >> 2;     // which half of the tile's columns
+    int local = 0;
+    for (int t = blockIdx.x; t < num_tiles; t += gridDim.x, ++local) {
+      int m_blk, n_blk;
+      tile_coords(args, t, m_blk, n_blk);
+      if (!mbar_wait_bounded(&tail->tmem_full, local & 1, abort_flag)) break;
+      tc_fence_after();
+      const uint32_t lane_addr = tmem + (static_cast<uint32_t>(q * 32) << 16);
+      uint32_t r0[32], r1[32], r2[32], r3[32];
+      if (!args.swiglu) {
+        tmem_ld_32x32b_x32(lane_addr + kColAcc + h * 128 + 0, r0);
+        tmem_ld_32x32b_x32(lane_addr + kColAcc + h * 128 + 32, r1);
+        tmem_ld_32x32b_x32(lane_addr + kColAcc + h * 128 + 64, r2);
+        tmem_ld_32x32b_x32(lane_addr + kColAcc + h * 128 + 96, r3);
+      } else {
+        tmem_ld_32x32b_x32(lane_addr + kColAcc + h * 64 + 0, r0);
+        tmem_ld_32x32b_x32(lane_addr + kColAcc + h * 64 + 32, r1);
+        tmem_ld_32x32b_x32(lane_addr + kColAcc + 128 + h * 64 + 0, r2);
+        tmem_ld_32x32b_x32(lane_addr + kColAcc + 128 + h * 64 + 32, r3);
+      }
+      tmem_ld_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tail->tmem_empty);
+
+      const int64_t row = static_cast<int64_t>(m_blk) * BM + q * 32 + lane;
+      if (row < args.M) {
+        if (!args.swiglu) {
+          const int64_t n0 = static_cast<int64_t>(n_blk) * BN + h * 128;
+          store_chunk(args, row, n0 + 0, r0);
+          store_chunk(args, row, n0 + 32, r1);
+          store_chunk(args, row, n0 + 64, r2);
+          store_chunk(args, row, n0 + 96, r3);
+        } else {
+          const int64_t o0 = static_cast<int64_t>(n_blk) * 128 + h * 64;
+          store_swiglu(args, row, o0, r0, r2);
+          store_swiglu(args, row, o0 + 32, r1, r3);
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+// ------------------------------------------------------------------ host side
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// Codes [rows, K/2] bytes: box 128 bytes x 128 rows, 128-byte swizzle.
+bool make_codes_map(CUtensorMap* m, const uint8_t* codes, int64_t rows, int64_t K) {
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(K / 2), static_cast<cuuint64_t>(rows)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(K / 2)};
+  const cuuint32_t box[2] = {128, 128};
+  const cuuint32_t estr[2] = {1, 1};
+  return encode_fn()(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(codes), dims, strides,
+                     box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Scale atoms: [row blocks][K atoms][512 bytes] viewed as u32 {128, KA, RB}; box = 4 atoms.
+bool make_sf_map(CUtensorMap* m, const uint8_t* sf, int64_t rows, int64_t K) {
+  const int64_t KA = ceil_div(K, 64), RB = ceil_div(rows, 128);
+  const cuuint64_t dims[3] = {128, static_cast<cuuint64_t>(KA), static_cast<cuuint64_t>(RB)};
+  const cuuint64_t strides[2] = {512, static_cast<cuuint64_t>(KA * 512)};
+  const cuuint32_t box[3] = {128, 4, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return encode_fn()(m, CU_TENSOR_MAP_DATA_TYPE_UINT32, 3, const_cast<uint8_t*>(sf), dims, strides,
+                     box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace gk
+
+size_t gemm_workspace_bytes(int64_t, int64_t, int64_t) { return 0; }
+
+cudaError_t launch_gemm(const GemmProblem& p, void*, size_t, cudaStream_t stream) {
+  using namespace gk;
+  if (encode_fn() == nullptr) return cudaErrorNotSupported;
+  CUtensorMap tm_a, tm_b, tm_sfa, tm_sfb;
+  if (!make_codes_map(&tm_a, p.a_codes, p.M, p.K) || !make_codes_map(&tm_b, p.w_codes, p.N, p.K) ||
+      !make_sf_map(&tm_sfa, p.a_sf, p.M, p.K) || !make_sf_map(&tm_sfb, p.w_sf, p.N, p.K))
+    return cudaErrorInvalidValue;
+
+  KernelArgs a{};
+  a.M = p.M;
+  a.N = p.N;
+  a.K = p.K;
+  a.swiglu = p.swiglu ? 1 : 0;
+  a.n_out = p.swiglu ? p.N / 2 : p.N;
+  a.up_row0 = p.swiglu ? p.N / 2 : 0;
+  a.num_m_blocks = static_cast<int>(ceil_div(p.M, BM));
+  a.num_n_blocks = static_cast<int>(p.swiglu ? ceil_div(p.N / 2, 128) : ceil_div(p.N, BN));
+  a.num_k_stages = static_cast<int>(ceil_div(p.K, BK));
+  a.group_m = 16;
+  a.g_a = p.g_a;
+  a.seg_scale = p.seg_scale;
+  a.nseg = p.nseg;
+  for (int i = 0; i < p.nseg; ++i) a.seg[i] = p.seg[i];
+
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  const int tiles = a.num_m_blocks * a.num_n_blocks;
+  if (tiles == 0) return cudaSuccess;
+  const int grid = tiles < sms ? tiles : sms;
+  gemm_kernel<<<grid, kThreads, kSmemBytes, stream>>>(tm_a, tm_b, tm_sfa, tm_sfb, a);
+  return cudaGetLastError();
+}
+
+}  // namespace nvfp4

@@ -1,0 +1,64 @@
+// Internal host-side interfaces between the C ABI layer and the kernels.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "../../include/nvfp4.h"
+
+namespace nvfp4 {
+
+constexpr int kMaxSeg = NVFP4_MAX_SEGMENTS;
+
+// Row ranges that share one global scale (modules stacked along rows).
+struct RowSegments {
+  int n;
+  int64_t begin[kMaxSeg + 1];  // begin[n] == total rows
+};
+
+inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+inline size_t sf_bytes(int64_t rows, int64_t K) {
+  return static_cast<size_t>(ceil_div(rows, 128) * 128) * static_cast<size_t>(ceil_div(K, 64) * 4);
+}
+
+// amax over each row range into ws_bits[s] (float bits, pre-zeroed).
+cudaError_t launch_amax(const void* x, int dtype, int64_t K, int64_t ld, const RowSegments& segs,
+                        unsigned int* ws_bits, cudaStream_t stream);
+
+// Quantise rows [0, M) (scale layout padded to 128 rows).  Scale of segment s:
+// g_in[s] if g_in, else (float bits ws_bits[s]) / 2688.  Writes g_out[s].
+cudaError_t launch_quantize(const void* x, int dtype, int64_t M, int64_t K, int64_t ld,
+                            const RowSegments& segs, const float* g_in,
+                            const unsigned int* ws_bits, float* g_out, uint8_t* codes,
+                            uint8_t* sf, cudaStream_t stream);
+
+// GEMM epilogue description handed to the kernels.
+struct EpiSegment {
+  int64_t n_begin, n_end;
+  int32_t kind;
+  int32_t scale_index;
+  void* out;
+  int64_t ld_out;
+  const float* a_log;
+  const float* dt_bias;
+};
+
+struct GemmProblem {
+  const uint8_t* a_codes;
+  const uint8_t* a_sf;
+  const uint8_t* w_codes;
+  const uint8_t* w_sf;
+  int64_t M, N, K;
+  const float* g_a;
+  const float* seg_scale;  // device [nseg]
+  int nseg;
+  EpiSegment seg[kMaxSeg];
+  bool swiglu;             // two segments: gate [0, N/2), up [N/2, N)
+};
+
+size_t gemm_workspace_bytes(int64_t M, int64_t N, int64_t K);
+cudaError_t launch_gemm(const GemmProblem& p, void* workspace, size_t workspace_bytes,
+                        cudaStream_t stream);
+
+}  // namespace nvfp4

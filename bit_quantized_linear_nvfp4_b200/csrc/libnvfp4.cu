@@ -1,0 +1,5 @@
+// Single translation unit of libnvfp4: the kernels share the device error
+// word, so they are compiled together without relocatable device code.
+#include "quantize.cu"
+#include "gemm.cu"
+#include "api.cu"

@@ -1,0 +1,260 @@
+"""ctypes binding of libnvfp4 (include/nvfp4.h).
+
+Argument marshalling only: tensors are allocated with PyTorch (device memory
+and streams are PyTorch's), every step of the computation runs in the CUDA
+library.  There is no fallback: if the library cannot be loaded, or a call
+returns a non-zero status, an exception is raised.
+"""
+from __future__ import annotations
+
+import ctypes
+import dataclasses
+import os
+from typing import Optional, Sequence
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libnvfp4.so")
+
+DTYPE_BF16 = 0
+DTYPE_F32 = 1
+MAX_SEGMENTS = 8
+
+EPI_IDENTITY_BF16 = 0
+EPI_IDENTITY_F32 = 1
+EPI_SIGMOID_F32 = 2
+EPI_GDN_DECAY_F32 = 3
+EPI_SWIGLU_GATE = 4
+EPI_SWIGLU_UP = 5
+
+EPILOGUES = {
+    "identity": EPI_IDENTITY_BF16,
+    "identity_bf16": EPI_IDENTITY_BF16,
+    "identity_f32": EPI_IDENTITY_F32,
+    "sigmoid": EPI_SIGMOID_F32,
+    "gdn_decay": EPI_GDN_DECAY_F32,
+    "swiglu_gate": EPI_SWIGLU_GATE,
+    "swiglu_up": EPI_SWIGLU_UP,
+}
+
+# Names the header declares; tests check the shared library exports each one.
+EXPORTED = (
+    "nvfp4_status_string", "nvfp4_last_cuda_error", "nvfp4_sf_bytes",
+    "nvfp4_quantize_workspace_bytes", "nvfp4_quantize", "nvfp4_quantize_segments",
+    "nvfp4_gemm_workspace_bytes", "nvfp4_gemm", "nvfp4_fused_proj", "nvfp4_check",
+)
+
+
+class Nvfp4Error(RuntimeError):
+    def __init__(self, status: int, where: str):
+        msg = _lib().nvfp4_status_string(status).decode()
+        if status == 4:
+            msg += f" (cudaError {_lib().nvfp4_last_cuda_error()})"
+        super().__init__(f"{where}: {msg} [status {status}]")
+        self.status = status
+
+
+class _Operand(ctypes.Structure):
+    _fields_ = [("codes", ctypes.c_void_p), ("sf", ctypes.c_void_p),
+                ("rows", ctypes.c_int64), ("K", ctypes.c_int64)]
+
+
+class _Segment(ctypes.Structure):
+    _fields_ = [("n_begin", ctypes.c_int64), ("n_end", ctypes.c_int64),
+                ("epilogue", ctypes.c_int32), ("reserved", ctypes.c_int32),
+                ("out", ctypes.c_void_p), ("ld_out", ctypes.c_int64),
+                ("A_log", ctypes.c_void_p), ("dt_bias", ctypes.c_void_p)]
+
+
+_LIB = None
+
+
+def _lib():
+    global _LIB
+    if _LIB is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"libnvfp4.so is not built ({LIB_PATH}); run bit_quantized_linear_nvfp4_b200/build.py")
+        lib = ctypes.CDLL(LIB_PATH)
+        c = ctypes
+        lib.nvfp4_status_string.restype = c.c_char_p
+        lib.nvfp4_status_string.argtypes = [c.c_int]
+        lib.nvfp4_last_cuda_error.restype = c.c_int
+        lib.nvfp4_sf_bytes.restype = c.c_size_t
+        lib.nvfp4_sf_bytes.argtypes = [c.c_int64, c.c_int64]
+        lib.nvfp4_quantize_workspace_bytes.restype = c.c_size_t
+        lib.nvfp4_quantize_workspace_bytes.argtypes = [c.c_int]
+        lib.nvfp4_quantize.restype = c.c_int
+        lib.nvfp4_quantize.argtypes = [c.c_void_p, c.c_int, c.c_int64, c.c_int64, c.c_int64,
+                                       c.c_void_p, c.c_void_p, c.c_void_p, c.c_void_p,
+                                       c.c_void_p, c.c_size_t, c.c_void_p]
+        lib.nvfp4_quantize_segments.restype = c.c_int
+        lib.nvfp4_quantize_segments.argtypes = [c.c_void_p, c.c_int, c.c_int64, c.c_int64, c.c_int64,
+                                                c.POINTER(c.c_int64), c.c_int, c.c_void_p, c.c_void_p,
+                                                c.c_void_p, c.c_void_p, c.c_void_p, c.c_size_t,
+                                                c.c_void_p]
+        lib.nvfp4_gemm_workspace_bytes.restype = c.c_size_t
+        lib.nvfp4_gemm_workspace_bytes.argtypes = [c.c_int64, c.c_int64, c.c_int64]
+        lib.nvfp4_gemm.restype = c.c_int
+        lib.nvfp4_gemm.argtypes = [c.POINTER(_Operand), c.c_void_p, c.POINTER(_Operand), c.c_void_p,
+                                   c.c_void_p, c.c_int, c.c_int64, c.c_void_p, c.c_size_t, c.c_void_p]
+        lib.nvfp4_fused_proj.restype = c.c_int
+        lib.nvfp4_fused_proj.argtypes = [c.POINTER(_Operand), c.c_void_p, c.POINTER(_Operand),
+                                         c.c_void_p, c.POINTER(_Segment), c.c_int, c.c_void_p,
+                                         c.c_size_t, c.c_void_p]
+        lib.nvfp4_check.restype = c.c_int
+        lib.nvfp4_check.argtypes = [c.c_void_p]
+        _LIB = lib
+    return _LIB
+
+
+def library():
+    """The loaded ctypes library (raises ImportError if it is not built)."""
+    return _lib()
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _call(name: str, *args):
+    st = getattr(_lib(), name)(*args)
+    if st != 0:
+        raise Nvfp4Error(st, name)
+
+
+def nvfp4_sf_bytes(rows: int, K: int) -> int:
+    return int(_lib().nvfp4_sf_bytes(rows, K))
+
+
+def nvfp4_quantize_workspace_bytes(nseg: int = 1) -> int:
+    return int(_lib().nvfp4_quantize_workspace_bytes(nseg))
+
+
+def nvfp4_gemm_workspace_bytes(M: int, N: int, K: int) -> int:
+    return int(_lib().nvfp4_gemm_workspace_bytes(M, N, K))
+
+
+@dataclasses.dataclass
+class Operand:
+    """A quantised operand: packed E2M1 codes [rows, K/2] and E4M3 scales in the
+    tcgen05 block-scale layout, both CUDA uint8 tensors."""
+    codes: torch.Tensor
+    sf: torch.Tensor
+    rows: int
+    K: int
+
+    def _c(self) -> _Operand:
+        return _Operand(self.codes.data_ptr(), self.sf.data_ptr(), self.rows, self.K)
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return DTYPE_BF16
+    if t.dtype == torch.float32:
+        return DTYPE_F32
+    raise TypeError(f"quantiser input must be bfloat16 or float32, not {t.dtype}")
+
+
+def _check_2d(x: torch.Tensor):
+    if not x.is_cuda or x.dim() != 2 or x.stride(1) != 1:
+        raise ValueError("expected a CUDA 2-D tensor with unit column stride")
+
+
+def nvfp4_quantize(x: torch.Tensor, g_in: Optional[torch.Tensor] = None, *, codes=None, sf=None,
+                   g_out=None, workspace=None, stream=None):
+    """Quantise activations x[M, K] (BF16/F32) -> (Operand, g_out[1])."""
+    _check_2d(x)
+    M, K = x.shape
+    dev = x.device
+    codes = torch.empty((M, K // 2), dtype=torch.uint8, device=dev) if codes is None else codes
+    sf = torch.empty(nvfp4_sf_bytes(max(M, 1), K), dtype=torch.uint8, device=dev) if sf is None else sf
+    g_out = torch.empty(1, dtype=torch.float32, device=dev) if g_out is None else g_out
+    if g_in is None and workspace is None:
+        workspace = torch.empty(nvfp4_quantize_workspace_bytes(1), dtype=torch.uint8, device=dev)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _call("nvfp4_quantize", _ptr(x), _dtype_code(x), M, K, x.stride(0), _ptr(g_in), _ptr(g_out),
+          _ptr(codes), _ptr(sf), _ptr(workspace), ws_bytes, _stream(stream))
+    return Operand(codes, sf, M, K), g_out
+
+
+def nvfp4_quantize_segments(w: torch.Tensor, row_bounds: Sequence[int], g_in=None, *, codes=None,
+                            sf=None, g_out=None, workspace=None, stream=None):
+    """Quantise stacked modules w[N, K], one global scale per row range -> (Operand, g_out[nseg])."""
+    _check_2d(w)
+    N, K = w.shape
+    nseg = len(row_bounds) - 1
+    dev = w.device
+    codes = torch.empty((N, K // 2), dtype=torch.uint8, device=dev) if codes is None else codes
+    sf = torch.empty(nvfp4_sf_bytes(N, K), dtype=torch.uint8, device=dev) if sf is None else sf
+    g_out = torch.empty(nseg, dtype=torch.float32, device=dev) if g_out is None else g_out
+    if g_in is None and workspace is None:
+        workspace = torch.empty(nvfp4_quantize_workspace_bytes(nseg), dtype=torch.uint8, device=dev)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    bounds = (ctypes.c_int64 * (nseg + 1))(*[int(b) for b in row_bounds])
+    _call("nvfp4_quantize_segments", _ptr(w), _dtype_code(w), N, K, w.stride(0), bounds, nseg,
+          _ptr(g_in), _ptr(g_out), _ptr(codes), _ptr(sf), _ptr(workspace), ws_bytes, _stream(stream))
+    return Operand(codes, sf, N, K), g_out
+
+
+def nvfp4_gemm(A: Operand, g_a: torch.Tensor, W: Operand, g_w: torch.Tensor, out=None,
+               out_dtype=torch.bfloat16, workspace=None, stream=None):
+    """out[M, N] = (A . W^T) * g_a * g_w, BF16 or F32."""
+    if out is None:
+        out = torch.empty((A.rows, W.rows), dtype=out_dtype, device=A.codes.device)
+    code = DTYPE_BF16 if out.dtype == torch.bfloat16 else DTYPE_F32
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    if workspace is None and nvfp4_gemm_workspace_bytes(A.rows, W.rows, A.K) > 0:
+        workspace = torch.empty(nvfp4_gemm_workspace_bytes(A.rows, W.rows, A.K), dtype=torch.uint8,
+                                device=A.codes.device)
+        ws_bytes = workspace.numel()
+    a, w = A._c(), W._c()
+    _call("nvfp4_gemm", ctypes.byref(a), _ptr(g_a), ctypes.byref(w), _ptr(g_w), _ptr(out), code,
+          out.stride(0), _ptr(workspace), ws_bytes, _stream(stream))
+    return out
+
+
+@dataclasses.dataclass
+class Segment:
+    """One module of a fused projection: W rows [n_begin, n_end)."""
+    n_begin: int
+    n_end: int
+    epilogue: str
+    out: Optional[torch.Tensor] = None
+    A_log: Optional[torch.Tensor] = None
+    dt_bias: Optional[torch.Tensor] = None
+
+
+def nvfp4_fused_proj(A: Operand, g_a: torch.Tensor, W: Operand, seg_global_scale: torch.Tensor,
+                     segments: Sequence[Segment], workspace=None, stream=None):
+    """One GEMM over the segments, each with its own global scale and epilogue;
+    results go to each segment's `out` tensor."""
+    n = len(segments)
+    arr = (_Segment * n)()
+    for i, s in enumerate(segments):
+        arr[i].n_begin = s.n_begin
+        arr[i].n_end = s.n_end
+        arr[i].epilogue = EPILOGUES[s.epilogue] if isinstance(s.epilogue, str) else int(s.epilogue)
+        arr[i].reserved = 0
+        arr[i].out = None if s.out is None else s.out.data_ptr()
+        arr[i].ld_out = 0 if s.out is None else s.out.stride(0)
+        arr[i].A_log = None if s.A_log is None else s.A_log.data_ptr()
+        arr[i].dt_bias = None if s.dt_bias is None else s.dt_bias.data_ptr()
+    need = nvfp4_gemm_workspace_bytes(A.rows, W.rows, A.K)
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=A.codes.device)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    a, w = A._c(), W._c()
+    _call("nvfp4_fused_proj", ctypes.byref(a), _ptr(g_a), ctypes.byref(w), _ptr(seg_global_scale),
+          arr, n, _ptr(workspace), ws_bytes, _stream(stream))
+
+
+def nvfp4_check(stream=None):
+    """Synchronise the stream and raise if a device-side wait timed out."""
+    _call("nvfp4_check", _stream(stream))

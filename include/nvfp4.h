@@ -1,0 +1,193 @@
+/*
+ * nvfp4.h — C ABI of libnvfp4: the NVFP4 W4A4 linear layer on B200 (sm_100a).
+ *
+ * What it computes.  "Why Gated DeltaNet Survives 4-Bit Quantization: NVFP4
+ * W4A4 for the Recurrent Half of a Hybrid 27B LLM" (ai.info summary),
+ * "Methodology in Plain English": weights and activations are stored as 4-bit
+ * E2M1 values with one E4M3 scale per block of 16 consecutive elements along
+ * K; "Main Findings", fused-GEMM scaling bullet: each linear module keeps one
+ * FP32 global scale, and a GEMM that fuses several modules must apply each
+ * module's own global scale (the repair of the global-scale mismatch);
+ * "Main Findings", gate-parameterisation bullets: the GDN write strength is
+ * sigmoid(b) and the decay is log-space, -exp(A_log) * softplus(a + dt_bias).
+ *
+ * Conventions for every entry point
+ *   - All pointers named "device" are device memory owned by the caller; the
+ *     library allocates no device memory and keeps no pointer after a call.
+ *   - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default
+ *     stream) and is asynchronous: no entry point synchronises, except
+ *     nvfp4_check.  Arguments are validated on the host before any launch; a
+ *     non-zero status means nothing was enqueued (NVFP4_ERR_CUDA: a launch or
+ *     driver call failed, see nvfp4_last_cuda_error).  Nothing aborts.
+ *   - Global scales are dequantisation multipliers: x ~= e2m1 * S * g with
+ *     g = amax / (6 * 448) when the library computes it.
+ *   - Codes: row-major [rows, K/2] bytes, element 2j of a row in the low
+ *     nibble, 2j+1 in the high nibble.
+ *   - Scale bytes (E4M3) use the tcgen05 block-scale layout: rows padded to
+ *     a multiple of 128, K/16 padded to a multiple of 4; 512-byte atoms hold
+ *     128 rows x 4 scales, scale (r, j) at byte
+ *       ((r/128) * KA + j/4) * 512 + (r%32)*16 + ((r/32)%4)*4 + j%4,
+ *     KA = ceil(K/64).  Padding bytes are zero (nvfp4_quantize writes them).
+ *   - Devices: compute capability 10.0 (B200) only.
+ */
+#ifndef NVFP4_H
+#define NVFP4_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum nvfp4_status {
+  NVFP4_OK = 0,
+  NVFP4_ERR_INVALID_ARG = 1,       /* null pointer, bad count or enum value */
+  NVFP4_ERR_UNSUPPORTED_SHAPE = 2, /* a size outside what the kernels take */
+  NVFP4_ERR_MISALIGNED = 3,        /* pointer or leading dimension alignment */
+  NVFP4_ERR_CUDA = 4,              /* a CUDA runtime/driver call failed */
+  NVFP4_ERR_DEVICE_TIMEOUT = 5,    /* a bounded device-side wait gave up */
+  NVFP4_ERR_WORKSPACE = 6,         /* workspace missing or too small */
+  NVFP4_ERR_DEVICE = 7             /* current device is not sm_100 */
+} nvfp4_status;
+
+/* Input element types for the quantiser. */
+enum { NVFP4_DTYPE_BF16 = 0, NVFP4_DTYPE_F32 = 1 };
+
+/* Largest number of segments (modules) in one fused projection or one
+ * segmented weight quantisation. */
+#define NVFP4_MAX_SEGMENTS 8
+
+/* A quantised operand in device memory (the struct itself is host memory). */
+typedef struct nvfp4_operand {
+  const uint8_t* codes; /* device, [rows, K/2], 16-byte aligned */
+  const uint8_t* sf;    /* device, nvfp4_sf_bytes(rows, K) bytes, 16-byte aligned */
+  int64_t rows;         /* M for activations, N for weights */
+  int64_t K;            /* reduction length, a multiple of 32 for the GEMMs */
+} nvfp4_operand;
+
+/* Per-segment epilogues of nvfp4_fused_proj.  y = acc * g_a * g_w[segment]. */
+typedef enum nvfp4_epilogue {
+  NVFP4_EPI_IDENTITY_BF16 = 0, /* out = bf16(y)                                   */
+  NVFP4_EPI_IDENTITY_F32 = 1,  /* out = y                                         */
+  NVFP4_EPI_SIGMOID_F32 = 2,   /* out = 1 / (1 + exp(-y))   (GDN write strength)  */
+  NVFP4_EPI_GDN_DECAY_F32 = 3, /* out = -exp(A_log[h]) * softplus(y + dt_bias[h]),
+                                  h = column - n_begin     (GDN log-space decay)  */
+  NVFP4_EPI_SWIGLU_GATE = 4,   /* out = bf16(silu(y) * y_up), paired with the
+                                  NVFP4_EPI_SWIGLU_UP segment of equal width      */
+  NVFP4_EPI_SWIGLU_UP = 5      /* consumed by the gate segment; writes nothing   */
+} nvfp4_epilogue;
+
+/* One segment (module) of a fused projection: W rows [n_begin, n_end). */
+typedef struct nvfp4_segment {
+  int64_t n_begin, n_end;
+  int32_t epilogue;      /* nvfp4_epilogue */
+  int32_t reserved;      /* must be 0 */
+  void* out;             /* device; element (m, j) at out[m * ld_out + j], j = n - n_begin;
+                            16-byte aligned; NULL only for NVFP4_EPI_SWIGLU_UP */
+  int64_t ld_out;        /* elements; multiple of 8 (BF16) or 4 (F32) */
+  const float* A_log;    /* device [n_end - n_begin], GDN decay only, else NULL */
+  const float* dt_bias;  /* device [n_end - n_begin], GDN decay only, else NULL */
+} nvfp4_segment;
+
+/* Human-readable name of a status code (static storage). */
+const char* nvfp4_status_string(int status);
+
+/* The CUDA error (cudaError_t value) behind the last NVFP4_ERR_CUDA on this thread. */
+int nvfp4_last_cuda_error(void);
+
+/* Bytes of the scale-factor buffer for a [rows, K] operand (padded layout above). */
+size_t nvfp4_sf_bytes(int64_t rows, int64_t K);
+
+/* Workspace bytes nvfp4_quantize / nvfp4_quantize_segments need (dynamic
+ * scales only; 0 when every global scale is given). */
+size_t nvfp4_quantize_workspace_bytes(int nseg);
+
+/*
+ * nvfp4_quantize — on-the-fly NVFP4 quantisation of an activation tensor
+ * (the "A4" half of W4A4, "Main Findings", activation-statistics bullet:
+ * per-token activation quantisation; format per "Methodology in Plain
+ * English").
+ *   x       device, [M, K] row-major with row stride ld_x elements; BF16 or F32
+ *           (x_dtype); 16-byte aligned base, ld_x * elem_size % 16 == 0.
+ *           Values must be finite.
+ *   K       multiple of 16.  M >= 0 (M == 0 writes only g_out).
+ *   g_in    device float, a calibrated (static) global scale, or NULL to use
+ *           g = amax|x| / 2688 computed on the device (two passes over x).
+ *   g_out   device float, receives the global scale used (may equal g_in).
+ *   codes   device, [M, K/2] bytes, 16-byte aligned.
+ *   sf      device, nvfp4_sf_bytes(M, K) bytes, 16-byte aligned; padding zeroed.
+ *   workspace / workspace_bytes: device scratch of at least
+ *           nvfp4_quantize_workspace_bytes(1) bytes when g_in == NULL.
+ * Per block of 16 (FP32): s = (amax_b / 6) / g; sf = E4M3_rn_satfinite(s);
+ * S = decode(sf); inv = 1 / (S * g) (0 if S * g == 0, at most FLT_MAX);
+ * code = E2M1_rn_satfinite(x * inv).  g <= 0 gives all-zero codes and scales.
+ */
+int nvfp4_quantize(const void* x, int x_dtype, int64_t M, int64_t K, int64_t ld_x,
+                   const float* g_in, float* g_out, uint8_t* codes, uint8_t* sf,
+                   void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * nvfp4_quantize_segments — the same quantiser over a weight matrix made of
+ * nseg modules stacked along rows, each with its own FP32 global scale ("one
+ * FP32 global scale per linear module", "Main Findings", fused-GEMM bullet).
+ *   row_bounds  host, nseg + 1 increasing row indices, row_bounds[0] == 0,
+ *               row_bounds[nseg] == N.
+ *   g_in        device float [nseg] or NULL (per-module amax / 2688).
+ *   g_out       device float [nseg].
+ *   Other arguments as nvfp4_quantize with M -> N; workspace of
+ *   nvfp4_quantize_workspace_bytes(nseg) bytes when g_in == NULL.
+ */
+int nvfp4_quantize_segments(const void* w, int w_dtype, int64_t N, int64_t K, int64_t ld_w,
+                            const int64_t* row_bounds, int nseg, const float* g_in, float* g_out,
+                            uint8_t* codes, uint8_t* sf, void* workspace, size_t workspace_bytes,
+                            void* stream);
+
+/* Workspace bytes nvfp4_gemm / nvfp4_fused_proj need for an [M, N, K]
+ * problem (non-zero for the small-M weight-streaming path only). */
+size_t nvfp4_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K);
+
+/*
+ * nvfp4_gemm — block-scaled FP4 x FP4 GEMM, out = (A . W^T) * g_a * g_w with
+ * FP32 accumulation: acc[m, n] = sum_k e2m1(a) Sa * e2m1(w) Sw
+ * ("Methodology in Plain English": W4A4 with 16-element E4M3 block scales).
+ *   A        host struct, device buffers: activations [M, K].
+ *   W        host struct, device buffers: weights [N, K] (same K).
+ *   g_a,g_w  device floats.
+ *   out      device, [M, N] row-major, stride ld_out elements; out_dtype is
+ *            NVFP4_DTYPE_BF16 or NVFP4_DTYPE_F32.
+ * Equivalent to nvfp4_fused_proj with one identity segment.
+ */
+int nvfp4_gemm(const nvfp4_operand* A, const float* g_a, const nvfp4_operand* W,
+               const float* g_w, void* out, int out_dtype, int64_t ld_out,
+               void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * nvfp4_fused_proj — one GEMM over nseg weight segments (modules) that keep
+ * their own global scales, with a per-segment epilogue: the fused GDN input
+ * projection (q, k, v, z identity to BF16; b -> sigmoid; a -> log-space decay)
+ * and the fused MLP gate/up projection (SwiGLU).  Column n of segment s is
+ * scaled by g_a * seg_global_scale[s] before its epilogue ("Main Findings",
+ * fused-GEMM scaling bullet).  Passing the same value for every segment
+ * reproduces the mismatch the pages describe.
+ *   seg_global_scale  device float [nseg].
+ *   segs              host array [nseg]; segments must tile [0, W->rows) in
+ *                     increasing order; a SwiGLU call has exactly two segments,
+ *                     gate then up, of equal width.
+ */
+int nvfp4_fused_proj(const nvfp4_operand* A, const float* g_a, const nvfp4_operand* W,
+                     const float* seg_global_scale, const nvfp4_segment* segs, int nseg,
+                     void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * nvfp4_check — synchronise `stream`, then report (and clear) the library's
+ * device error word: NVFP4_ERR_DEVICE_TIMEOUT if a bounded wait inside a
+ * kernel gave up since the last check, NVFP4_ERR_CUDA on a CUDA error.
+ */
+int nvfp4_check(void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* NVFP4_H */

@@ -1,0 +1,124 @@
+"""The C-ABI library loads on a machine without a GPU, exports every entry
+point include/nvfp4.h declares, and rejects bad arguments on the host before
+any CUDA call (CPU only: pointers below are never dereferenced)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from bit_quantized_linear_nvfp4_b200 import build as nvbuild
+from bit_quantized_linear_nvfp4_b200 import nvfp4 as nv
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    nvbuild.build(verbose=False)
+    return nv.library()
+
+
+def _declared():
+    text = open(os.path.join(ROOT, "include", "nvfp4.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(nvfp4_[a-z_0-9]+)\s*\(", text)))
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = _declared()
+    assert len(names) >= 10
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(names) == set(nv.EXPORTED)
+
+
+def test_status_strings(lib):
+    for s in range(8):
+        assert nv.library().nvfp4_status_string(s)
+    assert b"unknown" in nv.library().nvfp4_status_string(99)
+
+
+def test_sf_bytes_padding(lib):
+    assert nv.nvfp4_sf_bytes(1, 16) == 128 * 4
+    assert nv.nvfp4_sf_bytes(128, 64) == 512
+    assert nv.nvfp4_sf_bytes(129, 64) == 1024
+    assert nv.nvfp4_sf_bytes(4096, 5120) == 4096 * 320
+    assert nv.nvfp4_sf_bytes(12352, 5120) == 97 * 128 * 320
+    assert nv.nvfp4_sf_bytes(0, 16) == 0
+    assert nv.nvfp4_quantize_workspace_bytes(1) >= 4
+    assert nv.nvfp4_quantize_workspace_bytes(8) >= 32
+
+
+FAKE = 0x10000  # aligned, never dereferenced: validation fails first
+STREAM = None
+
+
+def _q(lib, x=FAKE, dtype=0, M=4, K=32, ld=32, g_in=FAKE, g_out=FAKE, codes=FAKE, sf=FAKE, ws=None, wsb=0):
+    v = ctypes.c_void_p
+    return lib.nvfp4_quantize(v(x) if x else None, dtype, M, K, ld, v(g_in) if g_in else None,
+                              v(g_out) if g_out else None, v(codes) if codes else None,
+                              v(sf) if sf else None, v(ws) if ws else None, wsb, None)
+
+
+def test_quantize_rejects_bad_arguments(lib):
+    assert _q(lib, K=24) == 2          # K % 16
+    assert _q(lib, dtype=7) == 1       # dtype
+    assert _q(lib, x=0) == 1           # null input
+    assert _q(lib, g_out=0) == 1       # null g_out
+    assert _q(lib, M=-1) == 1
+    assert _q(lib, ld=16) == 1         # ld < K
+    assert _q(lib, x=FAKE + 2) == 3    # misaligned input
+    assert _q(lib, ld=36) == 3         # row stride not a multiple of 16 bytes
+    assert _q(lib, codes=FAKE + 8) == 3
+    assert _q(lib, g_in=0) == 6        # dynamic scale without workspace
+    assert _q(lib, g_in=0, ws=FAKE, wsb=2) == 6
+
+
+def _op(codes=FAKE, sf=FAKE, rows=128, K=256):
+    return nv._Operand(codes, sf, rows, K)
+
+
+def _fp(lib, A=None, W=None, segs=None, nseg=None, g_a=FAKE, sc=FAKE):
+    A = A or _op()
+    W = W or _op(rows=256)
+    if segs is None:
+        segs = [nv._Segment(0, 256, 0, 0, FAKE, 256, None, None)]
+    arr = (nv._Segment * len(segs))(*segs)
+    v = ctypes.c_void_p
+    return lib.nvfp4_fused_proj(ctypes.byref(A), v(g_a) if g_a else None, ctypes.byref(W),
+                                v(sc) if sc else None, arr, len(segs) if nseg is None else nseg,
+                                None, 0, None)
+
+
+def test_fused_proj_rejects_bad_arguments(lib):
+    S = nv._Segment
+    assert _fp(lib, A=_op(K=48)) == 2                         # K % 32
+    assert _fp(lib, A=_op(K=512)) == 1                        # K mismatch
+    assert _fp(lib, A=_op(codes=FAKE + 4)) == 3
+    assert _fp(lib, g_a=0) == 1
+    assert _fp(lib, nseg=0) == 1
+    assert _fp(lib, nseg=9) == 1
+    # segments must tile [0, N)
+    assert _fp(lib, segs=[S(0, 100, 0, 0, FAKE, 256, None, None)]) == 1
+    assert _fp(lib, segs=[S(0, 100, 0, 0, FAKE, 256, None, None), S(120, 256, 0, 0, FAKE, 256, None, None)]) == 1
+    assert _fp(lib, segs=[S(0, 256, 9, 0, FAKE, 256, None, None)]) == 1     # epilogue kind
+    assert _fp(lib, segs=[S(0, 256, 0, 0, None, 256, None, None)]) == 1     # null out
+    assert _fp(lib, segs=[S(0, 256, 0, 0, FAKE + 2, 256, None, None)]) == 3  # misaligned out
+    assert _fp(lib, segs=[S(0, 256, 0, 0, FAKE, 260, None, None)]) == 3     # ld not multiple of 8
+    assert _fp(lib, segs=[S(0, 256, 3, 0, FAKE, 256, None, None)]) == 1     # decay without params
+    # SwiGLU needs gate then up of equal width, 128-row aligned
+    assert _fp(lib, segs=[S(0, 128, 4, 0, FAKE, 128, None, None), S(128, 256, 0, 0, FAKE, 128, None, None)]) == 1
+    assert _fp(lib, W=_op(rows=200), segs=[S(0, 100, 4, 0, FAKE, 104, None, None), S(100, 200, 5, 0, None, 0, None, None)]) == 2
+
+
+def test_segmented_quantize_rejects_bad_bounds(lib):
+    v = ctypes.c_void_p
+    def call(bounds, N=256):
+        b = (ctypes.c_int64 * len(bounds))(*bounds)
+        return lib.nvfp4_quantize_segments(v(FAKE), 0, N, 64, 64, b, len(bounds) - 1, v(FAKE), v(FAKE),
+                                           v(FAKE), v(FAKE), None, 0, None)
+    assert call([0, 100, 90, 256]) == 1
+    assert call([1, 256]) == 1
+    assert call([0, 200]) == 1
+    assert call([0] + list(range(10, 256, 30)) + [256]) == 1   # more than 8 segments

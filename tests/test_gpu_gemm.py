@@ -1,0 +1,203 @@
+"""GPU parity of nvfp4_gemm / nvfp4_fused_proj with the oracle (FP64 GEMM on
+the dequantised operands, FP64 epilogues)."""
+import numpy as np
+import pytest
+import torch
+
+from bit_quantized_linear_nvfp4_b200 import nvfp4 as nv
+from bit_quantized_linear_nvfp4_b200 import workloads as wl
+from oracle import nvfp4_oracle as o
+from tests.gpu_helpers import (TOL_ACC, assert_quant_equal, check_bf16, check_fp32, f32_ulp,
+                               to_np)
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda:0"
+
+
+def _dev(x, dtype="bf16"):
+    t = torch.from_numpy(np.ascontiguousarray(x)).to(DEV)
+    return t.to(torch.bfloat16) if dtype == "bf16" else t
+
+
+def _rand(M, K, seed, scale=1.0, outliers=0, dtype="bf16"):
+    rng = np.random.default_rng(seed)
+    x = (scale * rng.standard_normal((M, K))).astype(np.float32)
+    if outliers:
+        x[:, rng.choice(K, size=outliers, replace=False)] *= 50
+    return wl.round_to_bf16(x) if dtype == "bf16" else x
+
+
+def test_tiny_workload_fp32():
+    """X[64,512] x W[256,512] FP32 in, FP32 out, every element."""
+    w = wl.TINY
+    x, wt = wl.make_x(w), wl.make_w_segment(w, 0)
+    A, ga = nv.nvfp4_quantize(_dev(x, "f32"))
+    W, gw = nv.nvfp4_quantize(_dev(wt, "f32"))
+    out = nv.nvfp4_gemm(A, ga, W, gw, out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    assert_quant_equal(A, ga, x)
+    assert_quant_equal(W, gw, wt)
+    y, mag, _, _ = o.linear(x, wt)
+    check_fp32(to_np(out), y, mag, "tiny")
+
+
+@pytest.mark.parametrize("M,N,K", [(1, 256, 256), (100, 64, 512), (129, 200, 256), (300, 520, 1024),
+                                   (64, 384, 288), (257, 256, 5120)])
+@pytest.mark.parametrize("out_dtype", [torch.float32, torch.bfloat16])
+def test_ragged_gemm(M, N, K, out_dtype):
+    x = _rand(M, K, M + N + K, outliers=2)
+    wt = _rand(N, K, 7 * N + K, scale=0.02)
+    A, ga = nv.nvfp4_quantize(_dev(x))
+    W, gw = nv.nvfp4_quantize(_dev(wt))
+    out = nv.nvfp4_gemm(A, ga, W, gw, out_dtype=out_dtype)
+    torch.cuda.synchronize()
+    y, mag, _, _ = o.linear(x, wt)
+    if out_dtype == torch.float32:
+        check_fp32(to_np(out), y, mag, f"{M}x{N}x{K}")
+    else:
+        check_bf16(to_np(out), y, TOL_ACC * mag, f"{M}x{N}x{K}")
+
+
+def test_output_leading_dimension():
+    M, N, K = 70, 256, 256
+    x, wt = _rand(M, K, 1), _rand(N, K, 2, 0.02)
+    A, ga = nv.nvfp4_quantize(_dev(x))
+    W, gw = nv.nvfp4_quantize(_dev(wt))
+    big = torch.full((M, N + 64), -7.0, dtype=torch.bfloat16, device=DEV)
+    nv.nvfp4_gemm(A, ga, W, gw, out=big[:, 32:32 + N])
+    torch.cuda.synchronize()
+    y, mag, _, _ = o.linear(x, wt)
+    check_bf16(to_np(big[:, 32:32 + N]), y, TOL_ACC * mag)
+    assert torch.all(big[:, :32] == -7) and torch.all(big[:, 32 + N:] == -7)
+
+
+def _gdn_case(M, seed=3, b_a_scale=1.0):
+    """GDN in-projection segments with their own global scales (reduced M)."""
+    w = wl.GDN
+    rng = np.random.default_rng(seed)
+    K = w.K
+    x = _rand(M, K, seed, outliers=26)
+    segs = [wl.make_w_segment(w, s) for s in range(len(w.segments))]
+    if b_a_scale != 1.0:
+        segs[4] = wl.round_to_bf16(segs[4] * np.float32(b_a_scale))
+        segs[5] = wl.round_to_bf16(segs[5] * np.float32(b_a_scale))
+    a_log, dt_bias = wl.make_gate_params(w)
+    return w, x, segs, a_log, dt_bias
+
+
+def _run_fused(w, x, segs, a_log, dt_bias, common=False):
+    bounds = np.concatenate([[0], np.cumsum([s.width for s in w.segments])])
+    wcat = np.concatenate(segs)
+    A, ga = nv.nvfp4_quantize(_dev(x))
+    W, gw = nv.nvfp4_quantize_segments(_dev(wcat), bounds)
+    scales = gw
+    if common:
+        scales = torch.full_like(gw, float(gw.min().item()))
+    M = x.shape[0]
+    outs = []
+    nsegs = []
+    for s, seg in enumerate(w.segments):
+        kind = {"identity": "identity_bf16", "sigmoid": "sigmoid", "gdn_decay": "gdn_decay"}[seg.epilogue]
+        dt = torch.bfloat16 if kind == "identity_bf16" else torch.float32
+        out = torch.empty((M, seg.width), dtype=dt, device=DEV)
+        outs.append(out)
+        extra = {}
+        if kind == "gdn_decay":
+            extra = dict(A_log=torch.from_numpy(a_log).to(DEV), dt_bias=torch.from_numpy(dt_bias).to(DEV))
+        nsegs.append(nv.Segment(int(bounds[s]), int(bounds[s + 1]), kind, out, **extra))
+    nv.nvfp4_fused_proj(A, ga, W, scales, nsegs)
+    torch.cuda.synchronize()
+    return outs, gw.cpu().numpy(), float(ga.item())
+
+
+def _oracle_fused(x, segs, g_scales, a_log, dt_bias, w):
+    aq = o.quantize(x)
+    wq = [o.quantize(s) for s in segs]
+    epis = [s.epilogue for s in w.segments]
+    outs, pre = o.fused_projection(aq, [(c, s) for c, s, _ in wq], g_scales, epis, (a_log, dt_bias))
+    return outs, pre, [g for _, _, g in wq]
+
+
+def _check_gdn(outs, o_outs, pre, a_log, dt_bias, w):
+    for s, seg in enumerate(w.segments):
+        gpu = to_np(outs[s])
+        y, mag = pre[s]
+        tol = TOL_ACC * mag
+        if seg.epilogue == "identity":
+            check_bf16(gpu, o_outs[s], tol, seg.name)
+        elif seg.epilogue == "sigmoid":
+            bound = tol / 4 + 4 * f32_ulp(o_outs[s])
+            assert np.all(np.abs(gpu - o_outs[s]) <= bound), seg.name
+        else:
+            t = y + dt_bias[None, :]
+            deriv = np.exp(a_log)[None, :] * o.sigmoid(t)
+            bound = deriv * (tol + f32_ulp(t)) + 8 * f32_ulp(o_outs[s])
+            assert np.all(np.abs(gpu - o_outs[s]) <= bound), seg.name
+
+
+def test_gdn_fused_projection_reduced_rows():
+    w, x, segs, a_log, dt_bias = _gdn_case(300)
+    outs, g_gpu, _ = _run_fused(w, x, segs, a_log, dt_bias)
+    wq_g = [o.quantize(s)[2] for s in segs]
+    np.testing.assert_array_equal(g_gpu, np.array(wq_g, np.float32))
+    o_outs, pre, _ = _oracle_fused(x, segs, wq_g, a_log, dt_bias, w)
+    _check_gdn(outs, o_outs, pre, a_log, dt_bias, w)
+
+
+def test_gdn_common_scale_mismatch():
+    """One common global scale (the fused serving bug): segment s comes out
+    multiplied by g_c / g_s; with the per-segment table it does not."""
+    w, x, segs, a_log, dt_bias = _gdn_case(130, seed=11, b_a_scale=2.75)
+    good, g_gpu, _ = _run_fused(w, x, segs, a_log, dt_bias)
+    bad, _, _ = _run_fused(w, x, segs, a_log, dt_bias, common=True)
+    g_c = float(np.min(g_gpu))
+    # identity segments: exact ratio up to BF16 rounding of both sides
+    for s in range(4):
+        ratio = g_c / float(g_gpu[s])
+        gd, bd = to_np(good[s]), to_np(bad[s])
+        assert np.allclose(bd, gd * ratio, rtol=2 ** -7, atol=1e-6), s
+    # oracle with the common scale predicts the corrupted gates
+    o_bad, pre_bad, _ = _oracle_fused(x, segs, [g_c] * 6, a_log, dt_bias, w)
+    _check_gdn(bad, o_bad, pre_bad, a_log, dt_bias, w)
+    assert g_gpu[4] > g_c * 2  # the b/a modules were the mismatched ones
+
+
+def test_swiglu_reduced():
+    M, K, H = 200, 512, 384
+    x = _rand(M, K, 21, outliers=3)
+    gate = _rand(H, K, 22, 0.02)
+    up = _rand(H, K, 23, 0.05)
+    A, ga = nv.nvfp4_quantize(_dev(x))
+    W, gw = nv.nvfp4_quantize_segments(_dev(np.concatenate([gate, up])), [0, H, 2 * H])
+    out = torch.empty((M, H), dtype=torch.bfloat16, device=DEV)
+    nv.nvfp4_fused_proj(A, ga, W, gw, [nv.Segment(0, H, "swiglu_gate", out), nv.Segment(H, 2 * H, "swiglu_up")])
+    torch.cuda.synchronize()
+    aq = o.quantize(x)
+    gq, uq = o.quantize(gate), o.quantize(up)
+    outs, pre = o.fused_projection(aq, [gq[:2], uq[:2]], [gq[2], uq[2]], ["swiglu_gate", "swiglu_up"])
+    yg, mg = pre[0]
+    yu, mu = pre[1]
+    sg = o.sigmoid(yg)
+    dsilu = sg * (1 + yg * (1 - sg))
+    tol = np.abs(dsilu * yu) * TOL_ACC * mg + np.abs(yg * sg) * TOL_ACC * mu + 8 * f32_ulp(outs[0])
+    check_bf16(to_np(out), outs[0], tol, "swiglu")
+
+
+@pytest.mark.slow
+def test_oproj_full_size_sampled_rows():
+    """Prefill o_proj 4096x5120x5120 at full size; 256 sampled rows x all columns."""
+    w = wl.OPROJ
+    x = wl.make_x(w)
+    wt = wl.make_w_segment(w, 0)
+    A, ga = nv.nvfp4_quantize(_dev(x))
+    W, gw = nv.nvfp4_quantize(_dev(wt))
+    out = nv.nvfp4_gemm(A, ga, W, gw)
+    torch.cuda.synchronize()
+    rows = wl.sample_rows(w.M, 256)
+    g_a = o.global_scale(x)
+    assert np.float32(ga.item()) == g_a
+    aq = o.quantize(x[rows], g_a)
+    wq = o.quantize(wt)
+    acc, mag = o.gemm(aq[0], aq[1], wq[0], wq[1])
+    s = float(g_a) * float(wq[2])
+    check_bf16(to_np(out[torch.from_numpy(rows).to(DEV)]), acc * s, TOL_ACC * mag * s, "oproj")
