@@ -30,6 +30,10 @@ METRIC = "W4A4 GEMM TFLOPS & % dense-FP4 peak; quantize GB/s & % HBM peak (1 B20
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 FP4_PER_BF16 = 4.0  # nominal dense ratio: 9 PF FP4 / 2.25 PF BF16
 ROTATE = 4          # rotating input sets so consecutive steps miss in L2
+# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) per launch of the
+# dominant kernel, from one ncu capture of the kernel as it is now; None once
+# the kernel changes until it is captured again.
+TRAFFIC_BYTES = {"oproj": 26737408 + 813568}
 
 
 def load_peaks():
@@ -328,7 +332,7 @@ def run_product(args):
         fp4_peak = float(peaks["bf16_tflops_sustained"]) * FP4_PER_BF16
         ach = step.flops / (g_ms * 1e-3) / 1e12
         roof = {"bound": "tensor", "achieved": ach, "peak": fp4_peak, "unit": "TFLOP/s",
-                "frac": ach / fp4_peak, "traffic": None,
+                "frac": ach / fp4_peak, "traffic": TRAFFIC_BYTES.get(args.workload),
                 "peak_source": f"{peak_src} sustained bf16 x {FP4_PER_BF16:g} (nominal dense FP4/BF16)",
                 "kernel": "nvfp4 gemm (tcgen05 mxf4nvf4)", "ms_per_launch": g_ms,
                 "frac_of_nominal_9pf": ach / 9000.0}
@@ -505,8 +509,8 @@ def run_reference(args):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=50)
-    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--workload", default="oproj",
                     choices=["oproj", "mlp", "gdn", "tiny", "decode1", "decode8", "decode64", "quant"])
     ap.add_argument("--impl", default="product", choices=["product", "reference"])
