@@ -3,3 +3,4 @@
 #include "quantize.cu"
 #include "gemm.cu"
 #include "api.cu"
+#include "noalloc.cu"

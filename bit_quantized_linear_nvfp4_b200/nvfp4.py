@@ -43,6 +43,7 @@ EXPORTED = (
     "nvfp4_status_string", "nvfp4_last_cuda_error", "nvfp4_sf_bytes",
     "nvfp4_quantize_workspace_bytes", "nvfp4_quantize", "nvfp4_quantize_segments",
     "nvfp4_gemm_workspace_bytes", "nvfp4_gemm", "nvfp4_fused_proj", "nvfp4_check",
+    "nvfp4_quantize_noalloc",
 )
 
 
@@ -102,6 +103,9 @@ def _lib():
         lib.nvfp4_fused_proj.argtypes = [c.POINTER(_Operand), c.c_void_p, c.POINTER(_Operand),
                                          c.c_void_p, c.POINTER(_Segment), c.c_int, c.c_void_p,
                                          c.c_size_t, c.c_void_p]
+        lib.nvfp4_quantize_noalloc.restype = c.c_int
+        lib.nvfp4_quantize_noalloc.argtypes = [c.c_void_p, c.c_int, c.c_int64, c.c_int64, c.c_int64,
+                                               c.c_void_p, c.c_void_p, c.c_void_p, c.c_void_p]
         lib.nvfp4_check.restype = c.c_int
         lib.nvfp4_check.argtypes = [c.c_void_p]
         _LIB = lib

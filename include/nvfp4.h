@@ -143,6 +143,32 @@ int nvfp4_quantize_segments(const void* w, int w_dtype, int64_t N, int64_t K, in
                             uint8_t* codes, uint8_t* sf, void* workspace, size_t workspace_bytes,
                             void* stream);
 
+/*
+ * nvfp4_quantize_noalloc — nvfp4_quantize with the device-computed global
+ * scale (g = amax|x| / 2688), for callers that cannot allocate device memory.
+ * The paper has no counterpart: it is an interface for this library's users.
+ * Some callers have no device allocator at hand at the point where they
+ * quantise activations: a plugin enqueued by an inference runtime that owns
+ * all memory, code running under a fixed memory plan, or a C caller that only
+ * holds the tensors it was given.  The dynamic scale needs a few bytes of
+ * device scratch between its two passes; this entry point keeps that scratch
+ * in a static array inside the library (NVFP4_NOALLOC_SCRATCH_BYTES bytes,
+ * held on every GPU that loads the library until the process exits), so the
+ * caller passes only inputs and outputs and nothing is allocated.
+ *   Arguments as nvfp4_quantize with g_in = NULL and no workspace.
+ *   One call uses nvfp4_quantize_workspace_bytes(1) bytes of the scratch; a
+ *   call needing more than NVFP4_NOALLOC_SCRATCH_BYTES is rejected with
+ *   NVFP4_ERR_UNSUPPORTED_SHAPE.
+ *   The first call on a device looks up the scratch address on that device;
+ *   make that first call before any stream capture on the device.
+ *   Every call shares the one scratch array (each call clears it before use):
+ *   calls whose work overlaps on the GPU, on different streams, race and must
+ *   be serialised by the caller.
+ */
+#define NVFP4_NOALLOC_SCRATCH_BYTES 256
+int nvfp4_quantize_noalloc(const void* x, int x_dtype, int64_t M, int64_t K, int64_t ld_x,
+                           float* g_out, uint8_t* codes, uint8_t* sf, void* stream);
+
 /* Workspace bytes nvfp4_gemm / nvfp4_fused_proj need for an [M, N, K]
  * problem (non-zero for the small-M weight-streaming path only). */
 size_t nvfp4_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K);
