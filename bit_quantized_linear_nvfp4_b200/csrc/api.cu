@@ -37,6 +37,9 @@ int check_quant_args(const void* x, int dtype, int64_t M, int64_t K, int64_t ld,
   if (M < 0 || K <= 0 || g_out == nullptr) return NVFP4_ERR_INVALID_ARG;
   if (K % 16 != 0) return NVFP4_ERR_UNSUPPORTED_SHAPE;
   if (M > (int64_t(1) << 31) || K > (int64_t(1) << 30)) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+  // the kernels index (row, 512-element chunk) work items with 32-bit integers
+  if (nvfp4::ceil_div(M, 128) * 128 * nvfp4::ceil_div(K, 512) >= (int64_t(1) << 30))
+    return NVFP4_ERR_UNSUPPORTED_SHAPE;
   if (M == 0) return NVFP4_OK;
   if (x == nullptr || codes == nullptr || sf == nullptr) return NVFP4_ERR_INVALID_ARG;
   if (ld < K) return NVFP4_ERR_INVALID_ARG;
@@ -59,10 +62,6 @@ int quantize_impl(const void* x, int dtype, int64_t M, int64_t K, int64_t ld,
   if (st != NVFP4_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   unsigned int* bits = static_cast<unsigned int*>(ws);
-  if (g_in == nullptr) {
-    cudaError_t e = nvfp4::launch_amax(x, dtype, K, ld, segs, bits, s);
-    if (e != cudaSuccess) return cuda_fail(e);
-  }
   cudaError_t e = nvfp4::launch_quantize(x, dtype, M, K, ld, segs, g_in, bits, g_out, codes, sf, s);
   if (e != cudaSuccess) return cuda_fail(e);
   return NVFP4_OK;
@@ -106,7 +105,7 @@ size_t nvfp4_sf_bytes(int64_t rows, int64_t K) {
 
 size_t nvfp4_quantize_workspace_bytes(int nseg) {
   if (nseg < 1) nseg = 1;
-  return 16 * static_cast<size_t>((nseg * 4 + 15) / 16);
+  return 16 * ((nvfp4::quantize_scratch_words(nseg) * sizeof(unsigned int) + 15) / 16);
 }
 
 int nvfp4_quantize(const void* x, int x_dtype, int64_t M, int64_t K, int64_t ld_x,

@@ -382,6 +382,467 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
+// ------------------------------------------------------------------ CTA-pair kernel
+//
+// Same computation on a 256 x 256 tile shared by the two CTAs of a cluster
+// pair: each CTA loads 128 rows of A and 128 of the 256 B rows, the even CTA
+// issues tcgen05.mma.cta_group::2 with M = 256, and each CTA's TMEM holds its
+// own 128 x 256 accumulator.
+//
+// The operand feed is bound by the number of TMA copies in flight per SM more
+// than by bytes, so copies are kept few and large: the codes of a K-stage are
+// two 16 KB boxes, and the scale atoms of four K-stages arrive together in a
+// separate two-slot ring (one 8 KB box for A, one 16 KB box for the 256 B
+// rows; every CTA keeps the scales of all 256 B rows, as the pair MMA reads
+// them from each CTA's own TMEM).
+constexpr int kStages2 = 5;
+constexpr int kBHalfBytes = kBBytes / 2;                  // 16 KB
+constexpr int kCodeStage2 = kABytes + kBHalfBytes;       // 32 KB
+constexpr int kSFGroup = 4;                              // K-stages per scale group
+constexpr int kSFSlots = 2;
+constexpr int kSFASlotBytes = kSFGroup * kSFABytes;      // 8 KB
+constexpr int kSFBSlotBytes = kSFGroup * kSFBBytes;      // 16 KB
+constexpr int kSFSlotBytes = kSFASlotBytes + kSFBSlotBytes;
+constexpr int kSmemBytes2 = kStages2 * kCodeStage2 + kSFSlots * kSFSlotBytes + 1024 + 256;
+static_assert(kCodeStage2 % 1024 == 0 && kSFSlotBytes % 1024 == 0, "buffers keep 1024-byte alignment");
+
+struct SharedTail2 {
+  uint64_t full[kStages2];
+  uint64_t empty[kStages2];
+  uint64_t sf_full[kSFSlots];
+  uint64_t sf_empty[kSFSlots];
+  uint64_t tmem_full;
+  uint64_t tmem_empty;
+  uint64_t drain;
+  uint32_t tmem_base;
+  int abort_flag;
+};
+
+__global__ void __launch_bounds__(kThreads, 1)
+    gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
+                     const __grid_constant__ CUtensorMap tm_sfa, const __grid_constant__ CUtensorMap tm_sfb1,
+                     const __grid_constant__ CUtensorMap tm_sfb2, const __grid_constant__ KernelArgs args) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  uint8_t* sf_smem = smem + kStages2 * kCodeStage2;
+  SharedTail2* tail = reinterpret_cast<SharedTail2*>(sf_smem + kSFSlots * kSFSlotBytes);
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_rank() & 1u;  // position in the pair
+  const bool leader = rank == 0;
+  const int pair = blockIdx.x >> 1;
+  const int num_pairs = gridDim.x >> 1;
+  const int num_tiles = args.num_m_blocks * args.num_n_blocks;  // m blocks of 256 rows
+  const int KS = args.num_k_stages;
+  volatile int* abort_flag = &tail->abort_flag;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages2; ++s) {
+      mbar_init(&tail->full[s], 1);
+      mbar_init(&tail->empty[s], 1);
+    }
+    for (int s = 0; s < kSFSlots; ++s) {
+      mbar_init(&tail->sf_full[s], 1);
+      mbar_init(&tail->sf_empty[s], 1);
+    }
+    mbar_init(&tail->tmem_full, 1);
+    mbar_init(&tail->tmem_empty, 2 * kNumEpiWarps);
+    mbar_init(&tail->drain, 1);
+    tail->abort_flag = 0;
+    fence_mbarrier_init();
+    prefetch_tmap(&tm_a);
+    prefetch_tmap(&tm_b);
+    prefetch_tmap(&tm_sfa);
+    prefetch_tmap(&tm_sfb1);
+    prefetch_tmap(&tm_sfb2);
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(&tail->tmem_base, kTmemCols);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  cluster_sync_all();  // both CTAs' barriers exist before any cross-CTA signal
+  tc_fence_after();
+  const uint32_t tmem = tail->tmem_base;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer (both CTAs)
+    if (elect_one()) {
+      int stage = 0, sslot = 0;
+      uint32_t phase = 0, sphase = 0;
+      bool issued[kStages2], sissued[kSFSlots];
+      uint32_t issued_phase[kStages2], sissued_phase[kSFSlots];
+      for (int s = 0; s < kStages2; ++s) issued[s] = false;
+      for (int s = 0; s < kSFSlots; ++s) sissued[s] = false;
+      bool ok = true;
+      for (int t = pair; t < num_tiles && ok; t += num_pairs) {
+        int m_blk, n_blk;
+        tile_coords(args, t, m_blk, n_blk);
+        const int32_t a_row = m_blk * 256 + static_cast<int32_t>(rank) * 128;
+        const int64_t b_row0 = args.swiglu ? static_cast<int64_t>(n_blk) * 128 : static_cast<int64_t>(n_blk) * BN;
+        const int64_t b_row1 = args.swiglu ? args.up_row0 + static_cast<int64_t>(n_blk) * 128 : b_row0 + 128;
+        const int64_t b_mine = rank ? b_row1 : b_row0;
+        for (int ks = 0; ks < KS; ++ks) {
+          if (ks % kSFGroup == 0) {
+            // scale atoms of K-stages ks .. ks+3 for this CTA's A rows and all 256 B rows
+            if (!mbar_wait_bounded(&tail->sf_empty[sslot], sphase ^ 1u, abort_flag)) { ok = false; break; }
+            const uint32_t sbar = map_to_rank(smem_u32(&tail->sf_full[sslot]), 0);
+            if (leader) mbar_arrive_expect_tx(&tail->sf_full[sslot], 2 * kSFSlotBytes);
+            uint8_t* slot = sf_smem + sslot * kSFSlotBytes;
+            tma_load_3d_pair(slot, &tm_sfa, sbar, 0, ks * 4, a_row / 128);
+            if (args.swiglu) {
+              tma_load_3d_pair(slot + kSFASlotBytes, &tm_sfb1, sbar, 0, ks * 4, static_cast<int32_t>(b_row0 / 128));
+              tma_load_3d_pair(slot + kSFASlotBytes + kSFBSlotBytes / 2, &tm_sfb1, sbar, 0, ks * 4,
+                               static_cast<int32_t>(b_row1 / 128));
+            } else {
+              tma_load_3d_pair(slot + kSFASlotBytes, &tm_sfb2, sbar, 0, ks * 4, static_cast<int32_t>(b_row0 / 128));
+            }
+            sissued[sslot] = true;
+            sissued_phase[sslot] = sphase;
+            if (++sslot == kSFSlots) { sslot = 0; sphase ^= 1u; }
+          }
+          if (!mbar_wait_bounded(&tail->empty[stage], phase ^ 1u, abort_flag)) { ok = false; break; }
+          uint8_t* st = smem + stage * kCodeStage2;
+          const uint32_t bar = map_to_rank(smem_u32(&tail->full[stage]), 0);  // even CTA of the pair
+          if (leader) mbar_arrive_expect_tx(&tail->full[stage], 2 * kCodeStage2);
+          const int32_t kx = ks * (BK / 2);
+          tma_load_2d_pair(st, &tm_a, bar, kx, a_row);
+          tma_load_2d_pair(st + kABytes, &tm_b, bar, kx, static_cast<int32_t>(b_mine));
+          issued[stage] = true;
+          issued_phase[stage] = phase;
+          if (++stage == kStages2) { stage = 0; phase ^= 1u; }
+        }
+      }
+      if (*abort_flag && leader) {
+        for (int s = 0; s < kStages2; ++s)
+          if (issued[s]) mbar_wait_bounded(&tail->full[s], issued_phase[s], nullptr, 200000000ull);
+        for (int s = 0; s < kSFSlots; ++s)
+          if (sissued[s]) mbar_wait_bounded(&tail->sf_full[s], sissued_phase[s], nullptr, 200000000ull);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer (even CTA)
+    if (leader && elect_one()) {
+      // E2M1 x E2M1, UE4M3 scales, K-major A and B, M = 256 (pair), N = 256
+      const uint32_t idesc = (1u << 7) | (1u << 10) | (static_cast<uint32_t>(BN >> 3) << 17) |
+                             (static_cast<uint32_t>(256 >> 4) << 24);
+      const uint32_t base = smem_u32(smem);
+      const uint32_t sbase = smem_u32(sf_smem);
+      int stage = 0, sslot = 0;
+      uint32_t phase = 0, sphase = 0;
+      int local = 0;
+      bool ok = true;
+      bool any_issued = false;
+      for (int t = pair; t < num_tiles && ok; t += num_pairs, ++local) {
+        if (local > 0) {
+          if (!mbar_wait_bounded(&tail->tmem_empty, (local - 1) & 1, abort_flag)) { ok = false; break; }
+        }
+        tc_fence_after();
+        for (int ks = 0; ks < KS; ++ks) {
+          const int j = ks % kSFGroup;
+          if (j == 0) {
+            if (!mbar_wait_bounded(&tail->sf_full[sslot], sphase, abort_flag)) { ok = false; break; }
+          }
+          if (!mbar_wait_bounded(&tail->full[stage], phase, abort_flag)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t sa = base + stage * kCodeStage2;
+          const uint32_t sb = sa + kABytes;
+          const uint32_t ssfa = sbase + sslot * kSFSlotBytes + j * kSFABytes;
+          const uint32_t ssfb0 = sbase + sslot * kSFSlotBytes + kSFASlotBytes + j * kSFABytes;
+          const uint32_t ssfb1 = ssfb0 + kSFBSlotBytes / 2;
+#pragma unroll
+          for (int kb = 0; kb < 4; ++kb) {
+            tmem_cp_32x128b_warpx4_pair(tmem + kColSFA + 4 * kb, make_smem_desc(ssfa + 512 * kb, 0, 128, kLayoutSwizzleNone));
+            tmem_cp_32x128b_warpx4_pair(tmem + kColSFB + 8 * kb, make_smem_desc(ssfb0 + 512 * kb, 0, 128, kLayoutSwizzleNone));
+            tmem_cp_32x128b_warpx4_pair(tmem + kColSFB + 8 * kb + 4, make_smem_desc(ssfb1 + 512 * kb, 0, 128, kLayoutSwizzleNone));
+          }
+          const uint64_t adesc = make_smem_desc(sa, 16, 1024, kLayoutSwizzle128B);
+          const uint64_t bdesc = make_smem_desc(sb, 16, 1024, kLayoutSwizzle128B);
+#pragma unroll
+          for (int kb = 0; kb < 4; ++kb)
+            mma_mxf4nvf4_pair(tmem + kColAcc, adesc + 2 * kb, bdesc + 2 * kb, idesc, tmem + kColSFA + 4 * kb,
+                              tmem + kColSFB + 8 * kb, (ks | kb) != 0 ? 1u : 0u);
+          any_issued = true;
+          tc_commit_pair_mc(&tail->empty[stage], 0x3);
+          if (++stage == kStages2) { stage = 0; phase ^= 1u; }
+          if (j == kSFGroup - 1 || ks == KS - 1) {
+            tc_commit_pair_mc(&tail->sf_empty[sslot], 0x3);
+            if (++sslot == kSFSlots) { sslot = 0; sphase ^= 1u; }
+          }
+        }
+        if (!ok) break;
+        tc_commit_pair_mc(&tail->tmem_full, 0x3);
+      }
+      if (*abort_flag && any_issued) {
+        tc_commit_pair_mc(&tail->drain, 0x1);
+        mbar_wait_bounded(&tail->drain, 0, nullptr, 200000000ull);
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue (both CTAs)
+    const int q = warp & 3;
+    const int h = (warp - 2) >> 2;
+    const uint32_t empty_leader = map_to_rank(smem_u32(&tail->tmem_empty), 0);
+    int local = 0;
+    for (int t = pair; t < num_tiles; t += num_pairs, ++local) {
+      int m_blk, n_blk;
+      tile_coords(args, t, m_blk, n_blk);
+      if (!mbar_wait_bounded(&tail->tmem_full, local & 1, abort_flag)) break;
+      tc_fence_after();
+      const uint32_t lane_addr = tmem + (static_cast<uint32_t>(q * 32) << 16);
+      uint32_t r0[32], r1[32], r2[32], r3[32];
+      if (!args.swiglu) {
+        tmem_ld_32x32b_x32(lane_addr + kColAcc + h * 128 + 0, r0);
+        tmem_ld_32x32b_x32(lane_addr + kColAcc + h * 128 + 32, r1);
+        tmem_ld_32x32b_x32(lane_addr + kColAcc + h * 128 + 64, r2);
+        tmem_ld_32x32b_x32(lane_addr + kColAcc + h * 128 + 96, r3);
+      } else {
+        tmem_ld_32x32b_x32(lane_addr + kColAcc + h * 64 + 0, r0);
+        tmem_ld_32x32b_x32(lane_addr + kColAcc + h * 64 + 32, r1);
+        tmem_ld_32x32b_x32(lane_addr + kColAcc + 128 + h * 64 + 0, r2);
+        tmem_ld_32x32b_x32(lane_addr + kColAcc + 128 + h * 64 + 32, r3);
+      }
+      tmem_ld_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_remote(empty_leader);
+
+      const int64_t row = static_cast<int64_t>(m_blk) * 256 + rank * 128 + q * 32 + lane;
+      if (row < args.M) {
+        if (!args.swiglu) {
+          const int64_t n0 = static_cast<int64_t>(n_blk) * BN + h * 128;
+          store_chunk(args, row, n0 + 0, r0);
+          store_chunk(args, row, n0 + 32, r1);
+          store_chunk(args, row, n0 + 64, r2);
+          store_chunk(args, row, n0 + 96, r3);
+        } else {
+          const int64_t o0 = static_cast<int64_t>(n_blk) * 128 + h * 64;
+          store_swiglu(args, row, o0, r0, r2);
+          store_swiglu(args, row, o0 + 32, r1, r3);
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  cluster_sync_all();  // no pair-wide tcgen05 work remains in either CTA
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem, kTmemCols);
+  }
+}
+
+// ------------------------------------------------------------------ CTA-pair kernel, N = 192
+//
+// The 256 x 256 pair kernel holds a single accumulator per CTA (256 of the 512
+// TMEM columns, plus 48 for scales), so each tile ends with the MMA pipe
+// draining and the epilogue reading TMEM while the tensor cores wait.  With an
+// N = 192 tile two accumulators fit (2 x 192 + 16 SFA + 32 SFB columns), and
+// the next tile's MMAs run while the epilogue drains the previous one.  Each
+// CTA loads 128 A rows and 96 B rows; the B scale atoms are those of the two
+// 128-row blocks the 192 rows touch (a tile starts at 0 or 64 within its first
+// block), and the MMA's SFB address is shifted by (n0 mod 128) / 32 = 0 or 2
+// columns so that row n0 meets its scales (scale addresses stay 2-column
+// aligned).  Used for every fused projection except SwiGLU.
+constexpr int BN3 = 192;
+constexpr int kStages3 = 6;
+constexpr int kBRows3 = BN3 / 2;                           // 96 rows per CTA
+constexpr int kBBytes3 = kBRows3 * BK / 2;                 // 12 KB
+constexpr int kSFBBlocks3 = 2;
+constexpr int kSFBBytes3 = kSFBBlocks3 * 4 * 512;          // 2 row blocks x 4 atoms
+constexpr int kStageBytes3 = kABytes + kBBytes3 + kSFABytes + kSFBBytes3;  // 34 KB
+constexpr int kSmemBytes3 = kStages3 * kStageBytes3 + 1024 + 256;
+__device__ __forceinline__ uint32_t col_acc3(int buf) { return buf ? 192u : 0u; }
+constexpr uint32_t kColSFA3 = 384, kColSFB3 = 400;
+static_assert(kStageBytes3 % 1024 == 0, "stage buffers keep 1024-byte alignment");
+
+struct SharedTail3 {
+  uint64_t full[kStages3];
+  uint64_t empty[kStages3];
+  uint64_t tmem_full[2];
+  uint64_t tmem_empty[2];
+  uint64_t drain;
+  uint32_t tmem_base;
+  int abort_flag;
+};
+
+__global__ void __launch_bounds__(kThreads, 1)
+    gemm_pair_db_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
+                        const __grid_constant__ CUtensorMap tm_sfa, const __grid_constant__ CUtensorMap tm_sfb,
+                        const __grid_constant__ KernelArgs args) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  SharedTail3* tail = reinterpret_cast<SharedTail3*>(smem + kStages3 * kStageBytes3);
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_rank() & 1u;
+  const bool leader = rank == 0;
+  const int pair = blockIdx.x >> 1;
+  const int num_pairs = gridDim.x >> 1;
+  const int num_tiles = args.num_m_blocks * args.num_n_blocks;
+  volatile int* abort_flag = &tail->abort_flag;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages3; ++s) {
+      mbar_init(&tail->full[s], 1);
+      mbar_init(&tail->empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&tail->tmem_full[b], 1);
+      mbar_init(&tail->tmem_empty[b], 2 * kNumEpiWarps);
+    }
+    mbar_init(&tail->drain, 1);
+    tail->abort_flag = 0;
+    fence_mbarrier_init();
+    prefetch_tmap(&tm_a);
+    prefetch_tmap(&tm_b);
+    prefetch_tmap(&tm_sfa);
+    prefetch_tmap(&tm_sfb);
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(&tail->tmem_base, kTmemCols);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  cluster_sync_all();
+  tc_fence_after();
+  const uint32_t tmem = tail->tmem_base;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer (both CTAs)
+    if (elect_one()) {
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t issued_phase[kStages3];
+      bool issued[kStages3];
+      for (int s = 0; s < kStages3; ++s) issued[s] = false;
+      bool ok = true;
+      for (int t = pair; t < num_tiles && ok; t += num_pairs) {
+        int m_blk, n_blk;
+        tile_coords(args, t, m_blk, n_blk);
+        const int32_t a_row = m_blk * 256 + static_cast<int32_t>(rank) * 128;
+        const int32_t n0 = n_blk * BN3;
+        const int32_t b_row = n0 + static_cast<int32_t>(rank) * kBRows3;
+        for (int ks = 0; ks < args.num_k_stages; ++ks) {
+          if (!mbar_wait_bounded(&tail->empty[stage], phase ^ 1u, abort_flag)) { ok = false; break; }
+          uint8_t* st = smem + stage * kStageBytes3;
+          const uint32_t bar = map_to_rank(smem_u32(&tail->full[stage]), 0);
+          if (leader) mbar_arrive_expect_tx(&tail->full[stage], 2 * kStageBytes3);
+          const int32_t kx = ks * (BK / 2);
+          tma_load_2d_pair(st, &tm_a, bar, kx, a_row);
+          tma_load_2d_pair(st + kABytes, &tm_b, bar, kx, b_row);
+          uint8_t* sfa = st + kABytes + kBBytes3;
+          tma_load_3d_pair(sfa, &tm_sfa, bar, 0, ks * 4, a_row / 128);
+          tma_load_3d_pair(sfa + kSFABytes, &tm_sfb, bar, 0, ks * 4, n0 / 128);
+          issued[stage] = true;
+          issued_phase[stage] = phase;
+          if (++stage == kStages3) { stage = 0; phase ^= 1u; }
+        }
+      }
+      if (*abort_flag && leader) {
+        for (int s = 0; s < kStages3; ++s)
+          if (issued[s]) mbar_wait_bounded(&tail->full[s], issued_phase[s], nullptr, 200000000ull);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer (even CTA)
+    if (leader && elect_one()) {
+      // E2M1 x E2M1, UE4M3 scales, K-major A and B, M = 256 (pair), N = 192
+      const uint32_t idesc = (1u << 7) | (1u << 10) | (static_cast<uint32_t>(BN3 >> 3) << 17) |
+                             (static_cast<uint32_t>(256 >> 4) << 24);
+      const uint32_t base = smem_u32(smem);
+      int stage = 0;
+      uint32_t phase = 0;
+      int local = 0;
+      bool ok = true;
+      bool any_issued = false;
+      for (int t = pair; t < num_tiles && ok; t += num_pairs, ++local) {
+        int m_blk, n_blk;
+        tile_coords(args, t, m_blk, n_blk);
+        const uint32_t shift = static_cast<uint32_t>((n_blk * BN3) % 128) / 32;
+        const int buf = local & 1;
+        if (local >= 2) {
+          if (!mbar_wait_bounded(&tail->tmem_empty[buf], ((local >> 1) - 1) & 1, abort_flag)) { ok = false; break; }
+        }
+        tc_fence_after();
+        for (int ks = 0; ks < args.num_k_stages; ++ks) {
+          if (!mbar_wait_bounded(&tail->full[stage], phase, abort_flag)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t sa = base + stage * kStageBytes3;
+          const uint32_t sb = sa + kABytes;
+          const uint32_t ssfa = sb + kBBytes3;
+          const uint32_t ssfb = ssfa + kSFABytes;
+#pragma unroll
+          for (int kb = 0; kb < 4; ++kb) {
+            tmem_cp_32x128b_warpx4_pair(tmem + kColSFA3 + 4 * kb, make_smem_desc(ssfa + 512 * kb, 0, 128, kLayoutSwizzleNone));
+#pragma unroll
+            for (int z = 0; z < kSFBBlocks3; ++z)
+              tmem_cp_32x128b_warpx4_pair(tmem + kColSFB3 + 4 * kSFBBlocks3 * kb + 4 * z,
+                                          make_smem_desc(ssfb + 2048 * z + 512 * kb, 0, 128, kLayoutSwizzleNone));
+          }
+          const uint64_t adesc = make_smem_desc(sa, 16, 1024, kLayoutSwizzle128B);
+          const uint64_t bdesc = make_smem_desc(sb, 16, 1024, kLayoutSwizzle128B);
+#pragma unroll
+          for (int kb = 0; kb < 4; ++kb)
+            mma_mxf4nvf4_pair(tmem + col_acc3(buf), adesc + 2 * kb, bdesc + 2 * kb, idesc, tmem + kColSFA3 + 4 * kb,
+                              tmem + kColSFB3 + 4 * kSFBBlocks3 * kb + shift, (ks | kb) != 0 ? 1u : 0u);
+          any_issued = true;
+          tc_commit_pair_mc(&tail->empty[stage], 0x3);
+          if (++stage == kStages3) { stage = 0; phase ^= 1u; }
+        }
+        if (!ok) break;
+        tc_commit_pair_mc(&tail->tmem_full[buf], 0x3);
+      }
+      if (*abort_flag && any_issued) {
+        tc_commit_pair_mc(&tail->drain, 0x1);
+        mbar_wait_bounded(&tail->drain, 0, nullptr, 200000000ull);
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue (both CTAs)
+    const int q = warp & 3;
+    const int h = (warp - 2) >> 2;  // columns [0, 96) or [96, 192)
+    uint32_t empty_leader[2];
+    empty_leader[0] = map_to_rank(smem_u32(&tail->tmem_empty[0]), 0);
+    empty_leader[1] = map_to_rank(smem_u32(&tail->tmem_empty[1]), 0);
+    int local = 0;
+    for (int t = pair; t < num_tiles; t += num_pairs, ++local) {
+      int m_blk, n_blk;
+      tile_coords(args, t, m_blk, n_blk);
+      const int buf = local & 1;
+      if (!mbar_wait_bounded(&tail->tmem_full[buf], (local >> 1) & 1, abort_flag)) break;
+      tc_fence_after();
+      const uint32_t col = tmem + (static_cast<uint32_t>(q * 32) << 16) + col_acc3(buf) + h * 96;
+      uint32_t r0[32], r1[32], r2[32];
+      tmem_ld_32x32b_x32(col + 0, r0);
+      tmem_ld_32x32b_x32(col + 32, r1);
+      tmem_ld_32x32b_x32(col + 64, r2);
+      tmem_ld_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_remote(empty_leader[buf]);
+
+      const int64_t row = static_cast<int64_t>(m_blk) * 256 + rank * 128 + q * 32 + lane;
+      if (row < args.M) {
+        const int64_t n0 = static_cast<int64_t>(n_blk) * BN3 + h * 96;
+        store_chunk(args, row, n0 + 0, r0);
+        store_chunk(args, row, n0 + 32, r1);
+        store_chunk(args, row, n0 + 64, r2);
+      }
+    }
+  }
+
+  tc_fence_before();
+  cluster_sync_all();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem, kTmemCols);
+  }
+}
+
+
 // ------------------------------------------------------------------ host side
 
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
@@ -402,23 +863,24 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// Codes [rows, K/2] bytes: box 128 bytes x 128 rows, 128-byte swizzle.
-bool make_codes_map(CUtensorMap* m, const uint8_t* codes, int64_t rows, int64_t K) {
+// Codes [rows, K/2] bytes: box 128 bytes x box_rows rows, 128-byte swizzle.
+bool make_codes_map(CUtensorMap* m, const uint8_t* codes, int64_t rows, int64_t K, uint32_t box_rows = 128) {
   const cuuint64_t dims[2] = {static_cast<cuuint64_t>(K / 2), static_cast<cuuint64_t>(rows)};
   const cuuint64_t strides[1] = {static_cast<cuuint64_t>(K / 2)};
-  const cuuint32_t box[2] = {128, 128};
+  const cuuint32_t box[2] = {128, box_rows};
   const cuuint32_t estr[2] = {1, 1};
   return encode_fn()(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(codes), dims, strides,
                      box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                      CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// Scale atoms: [row blocks][K atoms][512 bytes] viewed as u32 {128, KA, RB}; box = 4 atoms.
-bool make_sf_map(CUtensorMap* m, const uint8_t* sf, int64_t rows, int64_t K) {
+// Scale atoms: [row blocks][K atoms][512 bytes] viewed as u32 {128, KA, RB};
+// box = `atoms` atoms of `blocks` consecutive 128-row blocks.
+bool make_sf_map(CUtensorMap* m, const uint8_t* sf, int64_t rows, int64_t K, uint32_t atoms = 4, uint32_t blocks = 1) {
   const int64_t KA = ceil_div(K, 64), RB = ceil_div(rows, 128);
   const cuuint64_t dims[3] = {128, static_cast<cuuint64_t>(KA), static_cast<cuuint64_t>(RB)};
   const cuuint64_t strides[2] = {512, static_cast<cuuint64_t>(KA * 512)};
-  const cuuint32_t box[3] = {128, 4, 1};
+  const cuuint32_t box[3] = {128, atoms, blocks};
   const cuuint32_t estr[3] = {1, 1, 1};
   return encode_fn()(m, CU_TENSOR_MAP_DATA_TYPE_UINT32, 3, const_cast<uint8_t*>(sf), dims, strides,
                      box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
@@ -429,14 +891,25 @@ bool make_sf_map(CUtensorMap* m, const uint8_t* sf, int64_t rows, int64_t K) {
 
 size_t gemm_workspace_bytes(int64_t, int64_t, int64_t) { return 0; }
 
+// Prefill shapes (M > 128) run on CTA pairs unless switched off for comparison.
+#ifndef NVFP4_PAIR_KERNEL
+#define NVFP4_PAIR_KERNEL 1
+#endif
+bool g_use_pair_kernel = NVFP4_PAIR_KERNEL;
+
+bool decode_path_applies(const GemmProblem& p);
+cudaError_t launch_gemm_decode(const GemmProblem& p, cudaStream_t stream);
+
 cudaError_t launch_gemm(const GemmProblem& p, void*, size_t, cudaStream_t stream) {
   using namespace gk;
   if (encode_fn() == nullptr) return cudaErrorNotSupported;
+  if (decode_path_applies(p)) return launch_gemm_decode(p, stream);
   CUtensorMap tm_a, tm_b, tm_sfa, tm_sfb;
   if (!make_codes_map(&tm_a, p.a_codes, p.M, p.K) || !make_codes_map(&tm_b, p.w_codes, p.N, p.K) ||
       !make_sf_map(&tm_sfa, p.a_sf, p.M, p.K) || !make_sf_map(&tm_sfb, p.w_sf, p.N, p.K))
     return cudaErrorInvalidValue;
 
+  const bool pair_kernel = p.M > 128 && g_use_pair_kernel;
   KernelArgs a{};
   a.M = p.M;
   a.N = p.N;
@@ -444,10 +917,10 @@ cudaError_t launch_gemm(const GemmProblem& p, void*, size_t, cudaStream_t stream
   a.swiglu = p.swiglu ? 1 : 0;
   a.n_out = p.swiglu ? p.N / 2 : p.N;
   a.up_row0 = p.swiglu ? p.N / 2 : 0;
-  a.num_m_blocks = static_cast<int>(ceil_div(p.M, BM));
+  a.num_m_blocks = static_cast<int>(ceil_div(p.M, pair_kernel ? 2 * BM : BM));
   a.num_n_blocks = static_cast<int>(p.swiglu ? ceil_div(p.N / 2, 128) : ceil_div(p.N, BN));
   a.num_k_stages = static_cast<int>(ceil_div(p.K, BK));
-  a.group_m = 16;
+  a.group_m = pair_kernel ? 8 : 16;
   a.g_a = p.g_a;
   a.seg_scale = p.seg_scale;
   a.nseg = p.nseg;
@@ -456,17 +929,71 @@ cudaError_t launch_gemm(const GemmProblem& p, void*, size_t, cudaStream_t stream
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
   const int tiles = a.num_m_blocks * a.num_n_blocks;
   if (tiles == 0) return cudaSuccess;
-  const int grid = tiles < sms ? tiles : sms;
-  gemm_kernel<<<grid, kThreads, kSmemBytes, stream>>>(tm_a, tm_b, tm_sfa, tm_sfb, a);
-  return cudaGetLastError();
+  if (!pair_kernel) {
+    static bool attr_set = false;
+    if (!attr_set) {
+      cudaError_t e = cudaFuncSetAttribute(gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+      if (e != cudaSuccess) return e;
+      attr_set = true;
+    }
+    const int grid = tiles < sms ? tiles : sms;
+    gemm_kernel<<<grid, kThreads, kSmemBytes, stream>>>(tm_a, tm_b, tm_sfa, tm_sfb, a);
+    return cudaGetLastError();
+  }
+  if (!p.swiglu) {
+    KernelArgs b = a;
+    b.num_n_blocks = static_cast<int>(ceil_div(p.N, BN3));
+    CUtensorMap tm_b3, tm_sfb3;
+    if (!make_codes_map(&tm_b3, p.w_codes, p.N, p.K, kBRows3) || !make_sf_map(&tm_sfb3, p.w_sf, p.N, p.K, 4, kSFBBlocks3))
+      return cudaErrorInvalidValue;
+    static bool attr3_set = false;
+    if (!attr3_set) {
+      cudaError_t e = cudaFuncSetAttribute(gemm_pair_db_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes3);
+      if (e != cudaSuccess) return e;
+      attr3_set = true;
+    }
+    const int tiles3 = b.num_m_blocks * b.num_n_blocks;
+    const int pairs3 = tiles3 < sms / 2 ? tiles3 : sms / 2;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2 * pairs3);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = kSmemBytes3;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, gemm_pair_db_kernel, tm_a, tm_b3, tm_sfa, tm_sfb3, b);
+  }
+  CUtensorMap tm_sfa4, tm_sfb4, tm_sfb8;
+  if (!make_sf_map(&tm_sfa4, p.a_sf, p.M, p.K, 4 * kSFGroup, 1) || !make_sf_map(&tm_sfb4, p.w_sf, p.N, p.K, 4 * kSFGroup, 1) ||
+      !make_sf_map(&tm_sfb8, p.w_sf, p.N, p.K, 4 * kSFGroup, 2))
+    return cudaErrorInvalidValue;
+  static bool attr2_set = false;
+  if (!attr2_set) {
+    cudaError_t e = cudaFuncSetAttribute(gemm_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes2);
+    if (e != cudaSuccess) return e;
+    attr2_set = true;
+  }
+  const int pairs = tiles < sms / 2 ? tiles : sms / 2;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * pairs);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = kSmemBytes2;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, gemm_pair_kernel, tm_a, tm_b, tm_sfa4, tm_sfb4, tm_sfb8, a);
 }
 
 }  // namespace nvfp4

@@ -1,0 +1,351 @@
+// Weight-streaming NVFP4 GEMM for few tokens (M <= 64), sm_100a.
+//
+// Same arithmetic as the prefill kernel ("Why Gated DeltaNet Survives 4-Bit
+// Quantization", ai.info summary, "Methodology in Plain English"; "Main
+// Findings": per-module global scales and gate nonlinearities), shaped for
+// decode, where the GEMM is bound by reading W from HBM ("Main Findings",
+// efficiency bullet: decode is weight-bandwidth-bound).
+//
+//  * Swap AB: 128 weight rows fill the MMA M dimension, the (<= 64) tokens sit
+//    in N = 64, so out^T[n, m] = W[n, :] . X[m, :] accumulates in TMEM with one
+//    TMEM lane per weight row.
+//  * Split K over a thread-block cluster: the S CTAs of a cluster share one
+//    128-row block of W and each streams 1/S of K, so about S * N/128 CTAs
+//    stream W at once.
+//  * The S partial accumulators are summed through distributed shared memory:
+//    peers stage their FP32 partial in their own shared memory and arrive on
+//    the leader's mbarrier; the leader adds them in rank order (deterministic),
+//    applies the global scales and the segment's epilogue, stores, and then
+//    releases the peers.  No workspace, no atomics.  All waits are bounded.
+//
+// Warps: 0 TMA producer, 1 TMEM owner + MMA issuer, 2..5 epilogue (one TMEM
+// lane quadrant each).
+#include <cfloat>
+#include <cstdint>
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "internal.h"
+#include "ptx.cuh"
+
+namespace nvfp4 {
+namespace dk {
+
+constexpr int BM = 128;  // weight rows per CTA (MMA M)
+constexpr int BK = 256;
+constexpr int kWBytes = BM * BK / 2;     // 16 KB
+constexpr int kSFWBytes = BM * BK / 16;  // 2 KB
+constexpr int kSFXBytes = 128 * BK / 16; // 2 KB (one 128-row atom per 64 K)
+constexpr int kEpiWarps = 4;
+constexpr int kThreads = 64 + kEpiWarps * 32;
+constexpr uint32_t kTmemCols = 128;
+constexpr int kSmemBudget = 200 * 1024;
+
+// BN token columns (MMA N = 16, 32 or 64; tokens beyond M are zero rows of X).
+// The stage count fills the shared-memory budget, so fewer tokens means more
+// weight bytes in flight per CTA.
+template <int BN>
+struct DCfg {
+  static constexpr int kXBytes = BN * BK / 2;
+  static constexpr int kStageRaw = kWBytes + kXBytes + kSFWBytes + kSFXBytes;
+  static constexpr int kStageBytes = (kStageRaw + 1023) / 1024 * 1024;
+  static constexpr int kStages = kSmemBudget / kStageBytes;
+  static constexpr uint32_t kColAcc = 0, kColSFW = 64, kColSFX = 80;
+  static constexpr int kPartialBytes = BN * BM * 4;  // staged over the first stages
+  static constexpr int kSmemBytes = kStages * kStageBytes + 1024 + 512;
+  static_assert(kPartialBytes <= kStages * kStageBytes, "partial fits in the stage buffers");
+};
+constexpr int kMaxStages = kSmemBudget / ((kWBytes + 16 * BK / 2 + kSFWBytes + kSFXBytes + 1023) / 1024 * 1024);
+
+struct DecodeArgs {
+  int64_t M, N, K;
+  int num_k_stages, split;
+  const float* g_a;
+  const float* seg_scale;
+  int nseg;
+  EpiSegment seg[kMaxSeg];
+};
+
+struct Tail {
+  uint64_t full[kMaxStages];
+  uint64_t empty[kMaxStages];
+  uint64_t tmem_full;
+  uint64_t ready;  // leader: peers' partials staged
+  uint64_t done;   // peer: leader finished reading
+  uint64_t drain;
+  uint32_t tmem_base;
+  int abort_flag;
+};
+
+__device__ __forceinline__ float sigmoid_f(float y) { return 1.0f / (1.0f + expf(-y)); }
+__device__ __forceinline__ float softplus_f(float t) {
+  return t > 0.0f ? t + log1pf(expf(-t)) : log1pf(expf(t));
+}
+
+template <int BN>
+__global__ void __launch_bounds__(kThreads, 1)
+    decode_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_x,
+                  const __grid_constant__ CUtensorMap tm_sfw, const __grid_constant__ CUtensorMap tm_sfx,
+                  const __grid_constant__ DecodeArgs args) {
+  using C = DCfg<BN>;
+  constexpr int kStages = C::kStages;
+  constexpr int kStageBytes = C::kStageBytes;
+  constexpr int kXBytes = C::kXBytes;
+  constexpr uint32_t kColAcc = C::kColAcc, kColSFW = C::kColSFW, kColSFX = C::kColSFX;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  Tail* tail = reinterpret_cast<Tail*>(smem + kStages * kStageBytes);
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_rank();
+  const int S = args.split;
+  const int rb = blockIdx.x / S;
+  const int ks0 = static_cast<int>((static_cast<int64_t>(rank) * args.num_k_stages) / S);
+  const int ks1 = static_cast<int>((static_cast<int64_t>(rank + 1) * args.num_k_stages) / S);
+  volatile int* abort_flag = &tail->abort_flag;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&tail->full[s], 1);
+      mbar_init(&tail->empty[s], 1);
+    }
+    mbar_init(&tail->tmem_full, 1);
+    mbar_init(&tail->ready, S > 1 ? kEpiWarps * 32 * (S - 1) : 1);
+    mbar_init(&tail->done, 1);
+    mbar_init(&tail->drain, 1);
+    tail->abort_flag = 0;
+    fence_mbarrier_init();
+    prefetch_tmap(&tm_w);
+    prefetch_tmap(&tm_x);
+    prefetch_tmap(&tm_sfw);
+    prefetch_tmap(&tm_sfx);
+  }
+  if (warp == 1) {
+    tmem_alloc(&tail->tmem_base, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  // every CTA of the cluster has initialised its barriers before any remote arrive
+  cluster_sync_all();
+  tc_fence_after();
+  const uint32_t tmem = tail->tmem_base;
+
+  if (warp == 0) {
+    if (elect_one()) {
+      int stage = 0;
+      uint32_t phase = 0;
+      bool issued[kStages] = {};
+      uint32_t issued_phase[kStages] = {};
+      for (int ks = ks0; ks < ks1; ++ks) {
+        if (!mbar_wait_bounded(&tail->empty[stage], phase ^ 1u, abort_flag)) break;
+        uint8_t* st = smem + stage * kStageBytes;
+        mbar_arrive_expect_tx(&tail->full[stage], C::kStageRaw);
+        const int32_t kx = ks * (BK / 2);
+        tma_load_2d(st, &tm_w, &tail->full[stage], kx, rb * BM);
+        tma_load_2d(st + kWBytes, &tm_x, &tail->full[stage], kx, 0);
+        tma_load_3d(st + kWBytes + kXBytes, &tm_sfw, &tail->full[stage], 0, ks * 4, rb);
+        tma_load_3d(st + kWBytes + kXBytes + kSFWBytes, &tm_sfx, &tail->full[stage], 0, ks * 4, 0);
+        issued[stage] = true;
+        issued_phase[stage] = phase;
+        if (++stage == kStages) { stage = 0; phase ^= 1u; }
+      }
+      if (*abort_flag)
+        for (int s = 0; s < kStages; ++s)
+          if (issued[s]) mbar_wait_bounded(&tail->full[s], issued_phase[s], nullptr, 200000000ull);
+    }
+  } else if (warp == 1) {
+    if (elect_one()) {
+      // E2M1 x E2M1, UE4M3 scales, K-major, M = 128 (weights), N = 64 (tokens)
+      const uint32_t idesc = (1u << 7) | (1u << 10) | (static_cast<uint32_t>(BN >> 3) << 17) |
+                             (static_cast<uint32_t>(BM >> 4) << 24);
+      const uint32_t base = smem_u32(smem);
+      int stage = 0;
+      uint32_t phase = 0;
+      bool any = false;
+      for (int ks = ks0; ks < ks1; ++ks) {
+        if (!mbar_wait_bounded(&tail->full[stage], phase, abort_flag)) break;
+        tc_fence_after();
+        const uint32_t sw = base + stage * kStageBytes;
+        const uint32_t sx = sw + kWBytes;
+        const uint32_t ssfw = sx + kXBytes;
+        const uint32_t ssfx = ssfw + kSFWBytes;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          tmem_cp_32x128b_warpx4(tmem + kColSFW + 4 * j, make_smem_desc(ssfw + 512 * j, 0, 128, kLayoutSwizzleNone));
+          tmem_cp_32x128b_warpx4(tmem + kColSFX + 4 * j, make_smem_desc(ssfx + 512 * j, 0, 128, kLayoutSwizzleNone));
+        }
+        const uint64_t wdesc = make_smem_desc(sw, 16, 1024, kLayoutSwizzle128B);
+        const uint64_t xdesc = make_smem_desc(sx, 16, 1024, kLayoutSwizzle128B);
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          mma_mxf4nvf4(tmem + kColAcc, wdesc + 2 * j, xdesc + 2 * j, idesc, tmem + kColSFW + 4 * j,
+                       tmem + kColSFX + 4 * j, (ks > ks0 || j > 0) ? 1u : 0u);
+        any = true;
+        tc_commit(&tail->empty[stage]);
+        if (++stage == kStages) { stage = 0; phase ^= 1u; }
+      }
+      if (any) tc_commit(&tail->tmem_full);  // also the drain point on abort
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int q = warp & 3;
+    const int row_local = q * 32 + lane;
+    const int64_t n = static_cast<int64_t>(rb) * BM + row_local;
+    float acc[BN];
+    bool have = (ks1 > ks0) && mbar_wait_bounded(&tail->tmem_full, 0, abort_flag);
+    if (have) {
+      tc_fence_after();
+      const uint32_t lane_addr = tmem + (static_cast<uint32_t>(q * 32) << 16);
+      if constexpr (BN == 64) {
+        uint32_t r0[32], r1[32];
+        tmem_ld_32x32b_x32(lane_addr + kColAcc, r0);
+        tmem_ld_32x32b_x32(lane_addr + kColAcc + 32, r1);
+        tmem_ld_wait();
+#pragma unroll
+        for (int t = 0; t < 32; ++t) {
+          acc[t] = __uint_as_float(r0[t]);
+          acc[32 + t] = __uint_as_float(r1[t]);
+        }
+      } else if constexpr (BN == 32) {
+        uint32_t r0[32];
+        tmem_ld_32x32b_x32(lane_addr + kColAcc, r0);
+        tmem_ld_wait();
+#pragma unroll
+        for (int t = 0; t < 32; ++t) acc[t] = __uint_as_float(r0[t]);
+      } else {
+        uint32_t r0[16];
+        tmem_ld_32x32b_x16(lane_addr + kColAcc, r0);
+        tmem_ld_wait();
+#pragma unroll
+        for (int t = 0; t < 16; ++t) acc[t] = __uint_as_float(r0[t]);
+      }
+    } else {
+#pragma unroll
+      for (int t = 0; t < BN; ++t) acc[t] = 0.0f;
+    }
+    tc_fence_before();
+    float* partial = reinterpret_cast<float*>(smem);  // [token][row], reuses stage buffers
+    const uint32_t ready_local = smem_u32(&tail->ready);
+    if (rank != 0) {
+#pragma unroll
+      for (int t = 0; t < BN; ++t)
+        if (t < args.M) partial[t * BM + row_local] = acc[t];
+      mbar_arrive_remote(map_to_rank(ready_local, 0));
+      mbar_wait_cluster_bounded(&tail->done, 0);
+    } else {
+      const bool ok = S == 1 || mbar_wait_cluster_bounded(&tail->ready, 0);
+      if (ok) {
+        for (int p = 1; p < S; ++p) {
+          const uint32_t peer = map_to_rank(smem_u32(partial), p) + 4u * row_local;
+          // issue every remote load of this peer before the first add
+          float v[BN];
+#pragma unroll
+          for (int t = 0; t < BN; ++t) v[t] = t < args.M ? ld_shared_cluster_f32(peer + 4u * (t * BM)) : 0.0f;
+#pragma unroll
+          for (int t = 0; t < BN; ++t) acc[t] += v[t];
+        }
+      }
+      if (ok && n < args.N) {
+        int s = 0;
+#pragma unroll
+        for (int i = 1; i < kMaxSeg; ++i)
+          if (i < args.nseg && n >= args.seg[i].n_begin) s = i;
+        const EpiSegment& sg = args.seg[s];
+        const float scale = __ldg(args.g_a) * __ldg(args.seg_scale + s);
+        const int64_t j = n - sg.n_begin;
+        float a_log = 0.0f, dt = 0.0f;
+        if (sg.kind == NVFP4_EPI_GDN_DECAY_F32) {
+          a_log = -expf(__ldg(sg.a_log + j));
+          dt = __ldg(sg.dt_bias + j);
+        }
+#pragma unroll
+        for (int t = 0; t < BN; ++t) {
+          if (t >= args.M) break;
+          const float y = acc[t] * scale;
+          if (sg.kind == NVFP4_EPI_IDENTITY_BF16) {
+            static_cast<__nv_bfloat16*>(sg.out)[t * sg.ld_out + j] = __float2bfloat16_rn(y);
+          } else {
+            float o = y;
+            if (sg.kind == NVFP4_EPI_SIGMOID_F32) o = sigmoid_f(y);
+            else if (sg.kind == NVFP4_EPI_GDN_DECAY_F32) o = a_log * softplus_f(y + dt);
+            static_cast<float*>(sg.out)[t * sg.ld_out + j] = o;
+          }
+        }
+      }
+      // every epilogue thread of the leader has finished reading the peers
+      named_barrier_sync(1, kEpiWarps * 32);
+      if (threadIdx.x == 64)
+        for (int p = 1; p < S; ++p) mbar_arrive_remote(map_to_rank(smem_u32(&tail->done), p));
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+}  // namespace dk
+
+bool decode_path_applies(const GemmProblem& p) { return p.M >= 1 && p.M <= 64 && !p.swiglu; }
+
+namespace dk {
+template <int BN>
+cudaError_t launch_bn(const GemmProblem& p, cudaStream_t stream) {
+  using C = DCfg<BN>;
+  CUtensorMap tm_w, tm_x, tm_sfw, tm_sfx;
+  if (!gk::make_codes_map(&tm_w, p.w_codes, p.N, p.K, BM) || !gk::make_codes_map(&tm_x, p.a_codes, p.M, p.K, BN) ||
+      !gk::make_sf_map(&tm_sfw, p.w_sf, p.N, p.K) || !gk::make_sf_map(&tm_sfx, p.a_sf, p.M, p.K))
+    return cudaErrorInvalidValue;
+  DecodeArgs a{};
+  a.M = p.M;
+  a.N = p.N;
+  a.K = p.K;
+  a.num_k_stages = static_cast<int>(ceil_div(p.K, BK));
+  a.g_a = p.g_a;
+  a.seg_scale = p.seg_scale;
+  a.nseg = p.nseg;
+  for (int i = 0; i < p.nseg; ++i) a.seg[i] = p.seg[i];
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int rbs = static_cast<int>(ceil_div(p.N, BM));
+  int S = sms / rbs;
+  if (S > 8) S = 8;
+  if (S > a.num_k_stages) S = a.num_k_stages;
+  if (S < 1) S = 1;
+  a.split = S;
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(decode_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(rbs * S);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = C::kSmemBytes;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = S;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, decode_kernel<BN>, tm_w, tm_x, tm_sfw, tm_sfx, a);
+}
+}  // namespace dk
+
+cudaError_t launch_gemm_decode(const GemmProblem& p, cudaStream_t stream) {
+  if (p.M <= 16) return dk::launch_bn<16>(p, stream);
+  if (p.M <= 32) return dk::launch_bn<32>(p, stream);
+  return dk::launch_bn<64>(p, stream);
+}
+
+}  // namespace nvfp4

@@ -22,16 +22,17 @@ inline size_t sf_bytes(int64_t rows, int64_t K) {
   return static_cast<size_t>(ceil_div(rows, 128) * 128) * static_cast<size_t>(ceil_div(K, 64) * 4);
 }
 
-// amax over each row range into ws_bits[s] (float bits, pre-zeroed).
-cudaError_t launch_amax(const void* x, int dtype, int64_t K, int64_t ld, const RowSegments& segs,
-                        unsigned int* ws_bits, cudaStream_t stream);
+// Scratch words a device-computed scale needs: one amax word per segment and
+// one grid-barrier counter.
+size_t quantize_scratch_words(int nseg);
 
-// Quantise rows [0, M) (scale layout padded to 128 rows).  Scale of segment s:
-// g_in[s] if g_in, else (float bits ws_bits[s]) / 2688.  Writes g_out[s].
+// Quantise rows [0, M) (scale layout padded to 128 rows).  Global scale of
+// segment s: g_in[s] if g_in, else amax over the segment's rows / 2688,
+// computed in the same launch with `ws` (quantize_scratch_words(segs.n) words,
+// cleared here) as scratch.  Writes g_out[s].
 cudaError_t launch_quantize(const void* x, int dtype, int64_t M, int64_t K, int64_t ld,
-                            const RowSegments& segs, const float* g_in,
-                            const unsigned int* ws_bits, float* g_out, uint8_t* codes,
-                            uint8_t* sf, cudaStream_t stream);
+                            const RowSegments& segs, const float* g_in, unsigned int* ws,
+                            float* g_out, uint8_t* codes, uint8_t* sf, cudaStream_t stream);
 
 // GEMM epilogue description handed to the kernels.
 struct EpiSegment {

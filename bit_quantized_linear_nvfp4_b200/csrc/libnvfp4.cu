@@ -2,5 +2,6 @@
 // word, so they are compiled together without relocatable device code.
 #include "quantize.cu"
 #include "gemm.cu"
+#include "gemm_decode.cu"
 #include "api.cu"
 #include "noalloc.cu"

@@ -62,9 +62,7 @@ extern "C" int nvfp4_quantize_noalloc(const void* x, int x_dtype, int64_t M, int
   segs.begin[0] = 0;
   segs.begin[1] = M;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  // launch_amax clears the scratch word before accumulating into it
-  e = nvfp4::launch_amax(x, x_dtype, K, ld_x, segs, scratch, s);
-  if (e != cudaSuccess) return cuda_fail(e);
+  // launch_quantize clears the scratch words before accumulating into them
   e = nvfp4::launch_quantize(x, x_dtype, M, K, ld_x, segs, nullptr, scratch, g_out, codes, sf, s);
   if (e != cudaSuccess) return cuda_fail(e);
   return NVFP4_OK;

@@ -6,15 +6,19 @@
 // ("Main Findings", fused-GEMM bullet).  Per block of 16, in FP32:
 //   s = (amax_b / 6) / g;  sf = E4M3_rn_satfinite(s);  S = decode(sf)
 //   inv = S*g > 0 ? 1/(S*g) : 0, at most FLT_MAX;  code = E2M1_rn_satfinite(x*inv)
+// with g = amax|x| / (6 * 448) per tensor (or per row range) when not given.
 //
-// HBM-bound design: a warp takes one row and up to 4 consecutive chunks of 256
-// elements; lane l holds elements [8l, 8l+8) of a chunk (one 16-byte load for
-// BF16), so a lane pair holds one 16-block and one shuffle gives its amax.
-// Each lane stores its 8 codes as one 32-bit word (a warp writes 128
-// contiguous bytes); the 4 scales of a 64-element group are gathered by
-// shuffles into one 32-bit word stored at its place in the tcgen05 scale
-// layout.  The padding of the scale layout (rows up to 128, K/16 up to 4) is
-// written with zeros.
+// HBM-bound design.  A warp takes a chunk of 512 consecutive elements of one
+// row; lane l owns the 16-block l of the chunk (one 256-bit load for BF16),
+// so the block amax, scale and codes need no cross-lane traffic.  Each lane
+// stores its 16 codes as 8 contiguous bytes (a warp writes 256 bytes), and
+// four lanes' scale bytes are gathered by shuffles into one 32-bit word
+// stored at its place in the tcgen05 block-scale layout; layout padding
+// (rows up to 128, K/16 up to 4) is written with zeros.
+//
+// With a device-computed scale the kernel runs two passes in one cooperative
+// launch: amax over the rows, a grid barrier (bounded wait), then the
+// quantisation pass, which re-reads x from L2 when x fits there.
 #include <cfloat>
 #include <cstdint>
 
@@ -25,63 +29,86 @@
 #include "ptx.cuh"
 
 namespace nvfp4 {
-
 namespace qk {
 
-constexpr int kChunk = 256;        // elements per warp per chunk
-constexpr int kChunksPerItem = 4;  // chunks of one row per warp item
-constexpr int kThreads = 256;
+constexpr int kChunk = 512;  // elements per warp per chunk (32 lanes x 16)
+// Large blocks keep the number of blocks (and so of same-address atomics in
+// the amax reduction and the grid barrier) near the SM count; FP32 input
+// needs more registers per lane and uses smaller blocks.
+template <int DTYPE>
+struct Cfg {
+  static constexpr int kThreads = DTYPE == NVFP4_DTYPE_BF16 ? 1024 : 256;
+  static constexpr int kWarps = kThreads / 32;
+};
+constexpr int kUnrollQ = 2;  // chunks per warp iteration, quantisation pass
+constexpr int kUnrollA = 4;  // chunks per warp iteration, amax pass
 
-struct SegParams {
-  int n;
-  int64_t begin[kMaxSeg + 1];
+struct QuantArgs {
+  const uint8_t* x;
+  int64_t ld_bytes;
+  int32_t M, K, rows_pad, cpr;  // cpr: chunks per row
+  int32_t items_q, items_a;     // rows_pad * cpr, M * cpr
+  int nseg;
+  int32_t seg_begin[kMaxSeg + 1];
+  const float* g_in;
+  unsigned int* ws;  // [nseg] amax bits, [nseg] grid-barrier counter (dynamic only)
+  float* g_out;
+  uint8_t* codes;
+  uint8_t* sf;
 };
 
-__device__ __forceinline__ uint4 ld_stream_v4(const void* p) {
-  uint4 r;
-  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
-               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+__device__ __forceinline__ void ld_v8(const void* p, uint32_t* r) {
+  asm volatile("ld.global.nc.L1::no_allocate.v8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]),
+                 "=r"(r[6]), "=r"(r[7])
                : "l"(p));
-  return r;
+}
+__device__ __forceinline__ void ld_v4(const void* p, uint32_t* r) {
+  asm volatile("ld.global.nc.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "l"(p));
 }
 
-__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
-__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+// Raw 16-element block of one lane: 8 words (BF16) or 16 words (F32).
+template <int DTYPE>
+struct Block {
+  static constexpr int kWords = DTYPE == NVFP4_DTYPE_BF16 ? 8 : 16;
+  uint32_t w[kWords];
+};
+
+template <int DTYPE, bool WIDE>
+__device__ __forceinline__ void load_block(const uint8_t* p, Block<DTYPE>& b) {
+  if constexpr (DTYPE == NVFP4_DTYPE_BF16) {
+    if constexpr (WIDE) {
+      ld_v8(p, b.w);
+    } else {
+      ld_v4(p, b.w);
+      ld_v4(p + 16, b.w + 4);
+    }
+  } else {
+    if constexpr (WIDE) {
+      ld_v8(p, b.w);
+      ld_v8(p + 32, b.w + 8);
+    } else {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) ld_v4(p + 16 * i, b.w + 4 * i);
+    }
+  }
+}
 
 template <int DTYPE>
-struct Loader;
-
-template <>
-struct Loader<NVFP4_DTYPE_BF16> {
-  static constexpr int kBytes = 2;
-  struct Raw {
-    uint4 a;
-  };
-  __device__ __forceinline__ static Raw load(const uint8_t* p) { return Raw{ld_stream_v4(p)}; }
-  __device__ __forceinline__ static void unpack(const Raw& r, float (&v)[8]) {
-    v[0] = bf16_lo(r.a.x); v[1] = bf16_hi(r.a.x);
-    v[2] = bf16_lo(r.a.y); v[3] = bf16_hi(r.a.y);
-    v[4] = bf16_lo(r.a.z); v[5] = bf16_hi(r.a.z);
-    v[6] = bf16_lo(r.a.w); v[7] = bf16_hi(r.a.w);
+__device__ __forceinline__ void unpack(const Block<DTYPE>& b, float (&v)[16]) {
+  if constexpr (DTYPE == NVFP4_DTYPE_BF16) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      v[2 * i] = __uint_as_float(b.w[i] << 16);
+      v[2 * i + 1] = __uint_as_float(b.w[i] & 0xFFFF0000u);
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(b.w[i]);
   }
-};
-
-template <>
-struct Loader<NVFP4_DTYPE_F32> {
-  static constexpr int kBytes = 4;
-  struct Raw {
-    uint4 a, b;
-  };
-  __device__ __forceinline__ static Raw load(const uint8_t* p) {
-    return Raw{ld_stream_v4(p), ld_stream_v4(p + 16)};
-  }
-  __device__ __forceinline__ static void unpack(const Raw& r, float (&v)[8]) {
-    v[0] = __uint_as_float(r.a.x); v[1] = __uint_as_float(r.a.y);
-    v[2] = __uint_as_float(r.a.z); v[3] = __uint_as_float(r.a.w);
-    v[4] = __uint_as_float(r.b.x); v[5] = __uint_as_float(r.b.y);
-    v[6] = __uint_as_float(r.b.z); v[7] = __uint_as_float(r.b.w);
-  }
-};
+}
 
 // E4M3 (satfinite, round to nearest even) of a non-negative float: low byte.
 __device__ __forceinline__ uint32_t to_e4m3(float s) {
@@ -98,7 +125,7 @@ __device__ __forceinline__ float e4m3_value(uint32_t b) {
 }
 
 // Eight E2M1 codes (satfinite, round to nearest even), element 2j in the low nibble.
-__device__ __forceinline__ uint32_t to_e2m1x8(const float (&q)[8]) {
+__device__ __forceinline__ uint32_t to_e2m1x8(const float* q) {
   uint32_t out;
   asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
       "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
@@ -111,200 +138,258 @@ __device__ __forceinline__ uint32_t to_e2m1x8(const float (&q)[8]) {
   return out;
 }
 
-__device__ __forceinline__ int find_segment(const SegParams& sp, int64_t row) {
+__device__ __forceinline__ int find_segment(const QuantArgs& a, int32_t row) {
   int s = 0;
 #pragma unroll
   for (int i = 1; i < kMaxSeg; ++i)
-    if (i < sp.n && row >= sp.begin[i]) s = i;
+    if (i < a.nseg && row >= a.seg_begin[i]) s = i;
   return s;
 }
 
-// ------------------------------------------------------------------ amax
+__device__ __forceinline__ unsigned int ld_acquire_u32(const unsigned int* p) {
+  unsigned int v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
 
-template <int DTYPE>
-__global__ void __launch_bounds__(kThreads) amax_kernel(const uint8_t* __restrict__ x, int64_t K,
-                                                        int64_t ld_bytes, int64_t row_begin,
-                                                        int64_t rows, unsigned int* __restrict__ out) {
-  using L = Loader<DTYPE>;
+// Pass 1: per-segment amax of rows [0, M), one atomicMax per block and segment.
+template <int DTYPE, bool WIDE>
+__device__ __forceinline__ void amax_pass(const QuantArgs& a) {
+  constexpr int kWarps = Cfg<DTYPE>::kWarps;
   const int lane = threadIdx.x & 31;
-  const int64_t nchunks = (K + kChunk - 1) / kChunk;
-  const int64_t groups = (nchunks + kChunksPerItem - 1) / kChunksPerItem;
-  const int64_t items = rows * groups;
-  const int64_t warp0 = (static_cast<int64_t>(blockIdx.x) * kThreads + threadIdx.x) >> 5;
-  const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * kThreads) >> 5;
-  float m = 0.0f;
-  for (int64_t item = warp0; item < items; item += nwarps) {
-    const int64_t row = row_begin + item / groups;
-    const int64_t c0 = (item % groups) * kChunksPerItem;
-    const uint8_t* rp = x + row * ld_bytes;
-    typename L::Raw raw[kChunksPerItem];
-    bool act[kChunksPerItem];
+  const int warp = threadIdx.x >> 5;
+  const int32_t gwarp = blockIdx.x * kWarps + warp;
+  const int32_t nwarps = gridDim.x * kWarps;
+  constexpr int kEsz = DTYPE == NVFP4_DTYPE_BF16 ? 2 : 4;
+  float lm[kMaxSeg];
 #pragma unroll
-    for (int u = 0; u < kChunksPerItem; ++u) {
-      const int64_t col = (c0 + u) * kChunk + lane * 8;
-      act[u] = col < K;
-      if (act[u]) raw[u] = L::load(rp + col * L::kBytes);
+  for (int s = 0; s < kMaxSeg; ++s) lm[s] = 0.0f;
+  for (int32_t base = gwarp * kUnrollA; base < a.items_a; base += nwarps * kUnrollA) {
+    Block<DTYPE> blk[kUnrollA];
+    int32_t rows[kUnrollA];
+    bool act[kUnrollA];
+#pragma unroll
+    for (int u = 0; u < kUnrollA; ++u) {
+      const int32_t item = base + u;
+      const int32_t row = item / a.cpr;
+      const int32_t col = (item - row * a.cpr) * kChunk + lane * 16;
+      rows[u] = row;
+      act[u] = item < a.items_a && col < a.K;
+      if (act[u]) load_block<DTYPE, WIDE>(a.x + row * a.ld_bytes + static_cast<int64_t>(col) * kEsz, blk[u]);
     }
 #pragma unroll
-    for (int u = 0; u < kChunksPerItem; ++u) {
+    for (int u = 0; u < kUnrollA; ++u) {
       if (!act[u]) continue;
-      float v[8];
-      L::unpack(raw[u], v);
+      float v[16];
+      unpack<DTYPE>(blk[u], v);
+      float m = 0.0f;
 #pragma unroll
-      for (int i = 0; i < 8; ++i) m = fmaxf(m, fabsf(v[i]));
+      for (int i = 0; i < 16; ++i) m = fmaxf(m, fabsf(v[i]));
+      const int s = find_segment(a, rows[u]);
+#pragma unroll
+      for (int i = 0; i < kMaxSeg; ++i)
+        if (i == s) lm[i] = fmaxf(lm[i], m);
     }
   }
+  __shared__ float red[kWarps][kMaxSeg];
 #pragma unroll
-  for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
-  __shared__ float red[kThreads / 32];
-  if (lane == 0) red[threadIdx.x >> 5] = m;
+  for (int s = 0; s < kMaxSeg; ++s) {
+    float m = lm[s];
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+    if (lane == 0) red[warp][s] = m;
+  }
   __syncthreads();
-  if (threadIdx.x == 0) {
-    float b = 0.0f;
+  if (threadIdx.x < a.nseg) {
+    float m = 0.0f;
 #pragma unroll
-    for (int w = 0; w < kThreads / 32; ++w) b = fmaxf(b, red[w]);
-    if (b > 0.0f) atomicMax(out, __float_as_uint(b));  // non-negative floats order as integers
+    for (int w = 0; w < kWarps; ++w) m = fmaxf(m, red[w][threadIdx.x]);
+    if (m > 0.0f) atomicMax(a.ws + threadIdx.x, __float_as_uint(m));  // non-negative floats order as integers
   }
 }
 
-// -------------------------------------------------------------- quantise
-
-template <int DTYPE>
-__global__ void __launch_bounds__(kThreads) quantize_kernel(
-    const uint8_t* __restrict__ x, int64_t M, int64_t K, int64_t ld_bytes, SegParams sp,
-    const float* __restrict__ g_in, const unsigned int* __restrict__ ws_bits,
-    float* __restrict__ g_out, uint8_t* __restrict__ codes, uint8_t* __restrict__ sf) {
-  using L = Loader<DTYPE>;
-  __shared__ float g_sh[kMaxSeg];
-  if (threadIdx.x < sp.n) {
-    float g = g_in ? g_in[threadIdx.x] : __uint_as_float(ws_bits[threadIdx.x]) / 2688.0f;
-    g_sh[threadIdx.x] = g;
-    if (blockIdx.x == 0) g_out[threadIdx.x] = g;
-  }
-  __syncthreads();
-
+// Pass 2: quantise rows [0, rows_pad) (rows >= M only zero their scale words).
+template <int DTYPE, bool WIDE>
+__device__ __forceinline__ void quant_pass(const QuantArgs& a, const float* g_sh) {
+  constexpr int kWarps = Cfg<DTYPE>::kWarps;
   const int lane = threadIdx.x & 31;
-  const int64_t rows_pad = (M + 127) / 128 * 128;
-  const int64_t nchunks = (K + kChunk - 1) / kChunk;
-  const int64_t groups = (nchunks + kChunksPerItem - 1) / kChunksPerItem;
-  const int64_t KA = (K + 63) / 64;  // scale atoms per 128-row block
-  const int64_t code_ld = K / 2;
-  const int64_t items = rows_pad * groups;
-  const int64_t warp0 = (static_cast<int64_t>(blockIdx.x) * kThreads + threadIdx.x) >> 5;
-  const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * kThreads) >> 5;
-
-  for (int64_t item = warp0; item < items; item += nwarps) {
-    const int64_t row = item / groups;
-    const int64_t c0 = (item % groups) * kChunksPerItem;
-    const bool real_row = row < M;
-    const float g = real_row ? g_sh[find_segment(sp, row)] : 0.0f;
-    const bool live = real_row && (g > 0.0f);
-    const uint8_t* rp = x + row * ld_bytes;
-
-    typename L::Raw raw[kChunksPerItem];
-    bool act[kChunksPerItem];
+  const int32_t gwarp = blockIdx.x * kWarps + (threadIdx.x >> 5);
+  const int32_t nwarps = gridDim.x * kWarps;
+  constexpr int kEsz = DTYPE == NVFP4_DTYPE_BF16 ? 2 : 4;
+  const int32_t KA = (a.K + 63) / 64;
+  const int64_t code_ld = a.K / 2;
+  for (int32_t base = gwarp * kUnrollQ; base < a.items_q; base += nwarps * kUnrollQ) {
+    Block<DTYPE> blk[kUnrollQ];
+    int32_t rows[kUnrollQ], cols[kUnrollQ];
+    bool act[kUnrollQ];
+    float gs[kUnrollQ];
 #pragma unroll
-    for (int u = 0; u < kChunksPerItem; ++u) {
-      const int64_t col = (c0 + u) * kChunk + lane * 8;
-      act[u] = live && col < K;
-      if (act[u]) raw[u] = L::load(rp + col * L::kBytes);
+    for (int u = 0; u < kUnrollQ; ++u) {
+      const int32_t item = base + u;
+      const int32_t row = item / a.cpr;
+      const int32_t col = (item - row * a.cpr) * kChunk + lane * 16;
+      rows[u] = row;
+      cols[u] = col;
+      gs[u] = row < a.M ? g_sh[find_segment(a, row)] : 0.0f;
+      act[u] = item < a.items_q && row < a.M && col < a.K && gs[u] > 0.0f;
+      if (act[u]) load_block<DTYPE, WIDE>(a.x + row * a.ld_bytes + static_cast<int64_t>(col) * kEsz, blk[u]);
     }
-    // scale-layout address pieces of this row
-    const int64_t rb = row >> 7;
-    const uint32_t in_atom = static_cast<uint32_t>((row & 31) * 16 + ((row >> 5) & 3) * 4);
-
 #pragma unroll
-    for (int u = 0; u < kChunksPerItem; ++u) {
-      const int64_t chunk = c0 + u;
-      if (chunk >= nchunks) break;  // uniform across the warp
-      const int64_t col = chunk * kChunk + lane * 8;
-      float v[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-      if (act[u]) L::unpack(raw[u], v);
-      float m = 0.0f;
-#pragma unroll
-      for (int i = 0; i < 8; ++i) m = fmaxf(m, fabsf(v[i]));
-      m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));  // the lane pair holds one 16-block
-      uint32_t sfb = 0, word = 0;
+    for (int u = 0; u < kUnrollQ; ++u) {
+      const int32_t item = base + u;
+      if (item >= a.items_q) break;  // uniform across the warp
+      const int32_t row = rows[u], col = cols[u];
+      uint32_t sfb = 0;
+      uint2 word = make_uint2(0u, 0u);
       if (act[u]) {
+        const float g = gs[u];
+        float v[16];
+        unpack<DTYPE>(blk[u], v);
+        float m = 0.0f;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) m = fmaxf(m, fabsf(v[i]));
         const float s = (m / 6.0f) / g;
         sfb = to_e4m3(s);
         const float denom = e4m3_value(sfb) * g;
         float inv = denom > 0.0f ? 1.0f / denom : 0.0f;
         inv = fminf(inv, FLT_MAX);
-        float q[8];
+        float q[16];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) q[i] = v[i] * inv;
-        word = to_e2m1x8(q);
+        for (int i = 0; i < 16; ++i) q[i] = v[i] * inv;
+        word.x = to_e2m1x8(q);
+        word.y = to_e2m1x8(q + 8);
       }
-      if (real_row && col < K) *reinterpret_cast<uint32_t*>(codes + row * code_ld + col / 2) = word;
-      // gather the 4 scale bytes of each 64-element group into lane 8a
-      const int base = lane & ~7;
-      const uint32_t s1 = __shfl_sync(0xffffffffu, sfb, base + 2);
-      const uint32_t s2 = __shfl_sync(0xffffffffu, sfb, base + 4);
-      const uint32_t s3 = __shfl_sync(0xffffffffu, sfb, base + 6);
-      const int64_t kb = chunk * 4 + (lane >> 3);
-      if ((lane & 7) == 0 && kb < KA) {
-        const uint32_t w4 = sfb | (s1 << 8) | (s2 << 16) | (s3 << 24);
-        *reinterpret_cast<uint32_t*>(sf + (rb * KA + kb) * 512 + in_atom) = w4;
+      if (row < a.M && col < a.K)
+        *reinterpret_cast<uint2*>(a.codes + row * code_ld + col / 2) = word;
+      // four lanes' scale bytes -> one 32-bit word of the block-scale layout
+      const uint32_t s1 = __shfl_down_sync(0xffffffffu, sfb, 1);
+      const uint32_t s2 = __shfl_down_sync(0xffffffffu, sfb, 2);
+      const uint32_t s3 = __shfl_down_sync(0xffffffffu, sfb, 3);
+      const int32_t kb = col / 64;
+      if ((lane & 3) == 0 && kb < KA) {
+        const int64_t off = (static_cast<int64_t>(row >> 7) * KA + kb) * 512 + (row & 31) * 16 + ((row >> 5) & 3) * 4;
+        *reinterpret_cast<uint32_t*>(a.sf + off) = sfb | (s1 << 8) | (s2 << 16) | (s3 << 24);
       }
     }
   }
 }
 
-int grid_for(int64_t warp_items) {
+template <int DTYPE, bool WIDE, bool DYNAMIC>
+__global__ void __launch_bounds__(Cfg<DTYPE>::kThreads) quantize_kernel(const __grid_constant__ QuantArgs a) {
+  __shared__ float g_sh[kMaxSeg];
+  __shared__ int abort_sh;
+  if constexpr (DYNAMIC) {
+    amax_pass<DTYPE, WIDE>(a);
+    // grid barrier: every block's amax is published before any block reads it
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      abort_sh = 0;
+      unsigned int* counter = a.ws + a.nseg;
+      __threadfence();
+      atomicAdd(counter, 1u);
+      const uint64_t t0 = global_timer_ns();
+      while (ld_acquire_u32(counter) < gridDim.x) {
+        if (global_timer_ns() - t0 > 2000000000ull) {
+          atomicOr(&g_device_error, kErrTimeout);
+          abort_sh = 1;
+          break;
+        }
+        __nanosleep(64);
+      }
+    }
+    __syncthreads();
+    if (abort_sh) return;
+    if (threadIdx.x < a.nseg) {
+      const float g = __uint_as_float(ld_acquire_u32(a.ws + threadIdx.x)) / 2688.0f;
+      g_sh[threadIdx.x] = g;
+      if (blockIdx.x == 0) a.g_out[threadIdx.x] = g;
+    }
+  } else {
+    if (threadIdx.x < a.nseg) {
+      const float g = a.g_in[threadIdx.x];
+      g_sh[threadIdx.x] = g;
+      if (blockIdx.x == 0) a.g_out[threadIdx.x] = g;
+    }
+  }
+  __syncthreads();
+  quant_pass<DTYPE, WIDE>(a, g_sh);
+}
+
+int num_sms() {
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  const int64_t want = (warp_items + (kThreads / 32) - 1) / (kThreads / 32);
-  const int64_t cap = static_cast<int64_t>(sms) * 8;  // 8 resident blocks of 256 threads
-  int64_t g = want < cap ? want : cap;
-  return static_cast<int>(g < 1 ? 1 : g);
+  return sms;
+}
+
+template <int DTYPE, bool WIDE, bool DYNAMIC>
+cudaError_t launch_t(const QuantArgs& a, cudaStream_t stream) {
+  constexpr int kThreads = Cfg<DTYPE>::kThreads;
+  constexpr int kWarps = Cfg<DTYPE>::kWarps;
+  auto kern = quantize_kernel<DTYPE, WIDE, DYNAMIC>;
+  int per_sm = 0;
+  cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kThreads, 0);
+  if (e != cudaSuccess) return e;
+  if (per_sm < 1) per_sm = 1;
+  const int64_t cap = static_cast<int64_t>(num_sms()) * per_sm;
+  const int64_t want = (static_cast<int64_t>(a.items_q) + kWarps * kUnrollQ - 1) / (kWarps * kUnrollQ);
+  int grid = static_cast<int>(want < cap ? want : cap);
+  if (grid < 1) grid = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = DYNAMIC ? 1 : 0;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, a);
 }
 
 }  // namespace qk
 
-cudaError_t launch_amax(const void* x, int dtype, int64_t K, int64_t ld, const RowSegments& segs,
-                        unsigned int* ws_bits, cudaStream_t stream) {
-  using namespace qk;
-  cudaError_t e = cudaMemsetAsync(ws_bits, 0, sizeof(unsigned int) * segs.n, stream);
-  if (e != cudaSuccess) return e;
-  const int esz = dtype == NVFP4_DTYPE_BF16 ? 2 : 4;
-  const int64_t groups = ceil_div(ceil_div(K, kChunk), kChunksPerItem);
-  for (int s = 0; s < segs.n; ++s) {
-    const int64_t rows = segs.begin[s + 1] - segs.begin[s];
-    if (rows <= 0 || K <= 0) continue;
-    const int grid = grid_for(rows * groups);
-    if (dtype == NVFP4_DTYPE_BF16)
-      amax_kernel<NVFP4_DTYPE_BF16><<<grid, kThreads, 0, stream>>>(
-          static_cast<const uint8_t*>(x), K, ld * esz, segs.begin[s], rows, ws_bits + s);
-    else
-      amax_kernel<NVFP4_DTYPE_F32><<<grid, kThreads, 0, stream>>>(
-          static_cast<const uint8_t*>(x), K, ld * esz, segs.begin[s], rows, ws_bits + s);
-    e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
-  }
-  return cudaSuccess;
-}
+size_t quantize_scratch_words(int nseg) { return static_cast<size_t>(nseg) + 1; }
 
 cudaError_t launch_quantize(const void* x, int dtype, int64_t M, int64_t K, int64_t ld,
-                            const RowSegments& segs, const float* g_in,
-                            const unsigned int* ws_bits, float* g_out, uint8_t* codes,
-                            uint8_t* sf, cudaStream_t stream) {
+                            const RowSegments& segs, const float* g_in, unsigned int* ws,
+                            float* g_out, uint8_t* codes, uint8_t* sf, cudaStream_t stream) {
   using namespace qk;
-  SegParams sp;
-  sp.n = segs.n;
-  for (int i = 0; i <= kMaxSeg; ++i) sp.begin[i] = i <= segs.n ? segs.begin[i] : segs.begin[segs.n];
+  QuantArgs a{};
   const int esz = dtype == NVFP4_DTYPE_BF16 ? 2 : 4;
-  const int64_t groups = ceil_div(ceil_div(K, kChunk), kChunksPerItem);
-  const int64_t rows_pad = ceil_div(M, 128) * 128;
-  const int grid = grid_for(rows_pad * groups);
-  if (dtype == NVFP4_DTYPE_BF16)
-    quantize_kernel<NVFP4_DTYPE_BF16><<<grid, kThreads, 0, stream>>>(
-        static_cast<const uint8_t*>(x), M, K, ld * esz, sp, g_in, ws_bits, g_out, codes, sf);
-  else
-    quantize_kernel<NVFP4_DTYPE_F32><<<grid, kThreads, 0, stream>>>(
-        static_cast<const uint8_t*>(x), M, K, ld * esz, sp, g_in, ws_bits, g_out, codes, sf);
-  return cudaGetLastError();
+  a.x = static_cast<const uint8_t*>(x);
+  a.ld_bytes = ld * esz;
+  a.M = static_cast<int32_t>(M);
+  a.K = static_cast<int32_t>(K);
+  a.rows_pad = static_cast<int32_t>(ceil_div(M, 128) * 128);
+  a.cpr = static_cast<int32_t>(ceil_div(K, kChunk));
+  a.items_q = a.rows_pad * a.cpr;
+  a.items_a = a.M * a.cpr;
+  a.nseg = segs.n;
+  for (int i = 0; i <= kMaxSeg; ++i)
+    a.seg_begin[i] = static_cast<int32_t>(i <= segs.n ? segs.begin[i] : segs.begin[segs.n]);
+  a.g_in = g_in;
+  a.ws = ws;
+  a.g_out = g_out;
+  a.codes = codes;
+  a.sf = sf;
+  const bool dynamic = g_in == nullptr;
+  if (dynamic) {
+    cudaError_t e = cudaMemsetAsync(ws, 0, sizeof(unsigned int) * quantize_scratch_words(segs.n), stream);
+    if (e != cudaSuccess) return e;
+  }
+  const bool wide = (reinterpret_cast<uintptr_t>(x) % 32 == 0) && (a.ld_bytes % 32 == 0);
+  if (dtype == NVFP4_DTYPE_BF16) {
+    if (dynamic) return wide ? launch_t<NVFP4_DTYPE_BF16, true, true>(a, stream)
+                             : launch_t<NVFP4_DTYPE_BF16, false, true>(a, stream);
+    return wide ? launch_t<NVFP4_DTYPE_BF16, true, false>(a, stream)
+                : launch_t<NVFP4_DTYPE_BF16, false, false>(a, stream);
+  }
+  if (dynamic) return wide ? launch_t<NVFP4_DTYPE_F32, true, true>(a, stream)
+                           : launch_t<NVFP4_DTYPE_F32, false, true>(a, stream);
+  return wide ? launch_t<NVFP4_DTYPE_F32, true, false>(a, stream)
+              : launch_t<NVFP4_DTYPE_F32, false, false>(a, stream);
 }
 
 }  // namespace nvfp4

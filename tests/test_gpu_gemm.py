@@ -184,7 +184,7 @@ def test_swiglu_reduced():
 
 
 @pytest.mark.slow
-def test_oproj_full_size_sampled_rows():
+def test_full_size_oproj_sampled_rows():
     """Prefill o_proj 4096x5120x5120 at full size; 256 sampled rows x all columns."""
     w = wl.OPROJ
     x = wl.make_x(w)
@@ -201,3 +201,68 @@ def test_oproj_full_size_sampled_rows():
     acc, mag = o.gemm(aq[0], aq[1], wq[0], wq[1])
     s = float(g_a) * float(wq[2])
     check_bf16(to_np(out[torch.from_numpy(rows).to(DEV)]), acc * s, TOL_ACC * mag * s, "oproj")
+
+
+# ---------------------------------------------------------------- decode path (M <= 64)
+
+@pytest.mark.parametrize("M", [1, 5, 8, 64])
+@pytest.mark.parametrize("N,K", [(640, 2048), (200, 256), (128, 5376)])
+def test_decode_path(M, N, K):
+    """Few tokens: swap-AB, split-K over a cluster, DSMEM reduction."""
+    x = _rand(M, K, 3 * M + N, outliers=2)
+    wt = _rand(N, K, 5 * N + K, scale=0.02)
+    A, ga = nv.nvfp4_quantize(_dev(x))
+    W, gw = nv.nvfp4_quantize(_dev(wt))
+    out32 = nv.nvfp4_gemm(A, ga, W, gw, out_dtype=torch.float32)
+    out16 = nv.nvfp4_gemm(A, ga, W, gw, out_dtype=torch.bfloat16)
+    torch.cuda.synchronize()
+    y, mag, _, _ = o.linear(x, wt)
+    check_fp32(to_np(out32), y, mag, f"decode f32 {M}x{N}x{K}")
+    check_bf16(to_np(out16), y, TOL_ACC * mag, f"decode bf16 {M}x{N}x{K}")
+
+
+@pytest.mark.parametrize("M", [1, 8, 64])
+def test_decode_path_gdn_segments(M):
+    """GDN-style segments (identity, write strength, decay) through the decode epilogue."""
+    w = wl.GDN
+    rng = np.random.default_rng(31 + M)
+    K = 1024
+    x = _rand(M, K, 40 + M, outliers=3)
+    widths = [256, 32, 32]
+    segs = [wl.round_to_bf16((0.02 * (i + 1) * rng.standard_normal((n, K))).astype(np.float32)) for i, n in enumerate(widths)]
+    a_log, dt_bias = wl.make_gate_params(w)
+    bounds = [0, 256, 288, 320]
+    A, ga = nv.nvfp4_quantize(_dev(x))
+    W, gw = nv.nvfp4_quantize_segments(_dev(np.concatenate(segs)), bounds)
+    q = torch.empty((M, 256), dtype=torch.bfloat16, device=DEV)
+    beta = torch.empty((M, 32), dtype=torch.float32, device=DEV)
+    dec = torch.empty((M, 32), dtype=torch.float32, device=DEV)
+    nv.nvfp4_fused_proj(A, ga, W, gw, [
+        nv.Segment(0, 256, "identity_bf16", q), nv.Segment(256, 288, "sigmoid", beta),
+        nv.Segment(288, 320, "gdn_decay", dec, A_log=torch.from_numpy(a_log).to(DEV),
+                   dt_bias=torch.from_numpy(dt_bias).to(DEV))])
+    torch.cuda.synchronize()
+    aq = o.quantize(x)
+    wq = [o.quantize(s) for s in segs]
+    outs, pre = o.fused_projection(aq, [(c, s) for c, s, _ in wq], [g for _, _, g in wq],
+                                   ["identity", "sigmoid", "gdn_decay"], (a_log, dt_bias))
+    check_bf16(to_np(q), outs[0], TOL_ACC * pre[0][1], "q")
+    assert np.all(np.abs(to_np(beta) - outs[1]) <= TOL_ACC * pre[1][1] / 4 + 4 * f32_ulp(outs[1]))
+    t = pre[2][0] + dt_bias[None, :]
+    bound = np.exp(a_log)[None, :] * o.sigmoid(t) * (TOL_ACC * pre[2][1] + f32_ulp(t)) + 8 * f32_ulp(outs[2])
+    assert np.all(np.abs(to_np(dec) - outs[2]) <= bound)
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("M", [1, 8, 64])
+def test_full_size_decode(M):
+    """Decode down_proj W[5120,17408], every output element."""
+    w = wl.decode_workload(M)
+    x = wl.make_x(w)
+    wt = wl.make_w_segment(w, 0)
+    A, ga = nv.nvfp4_quantize(_dev(x))
+    W, gw = nv.nvfp4_quantize(_dev(wt))
+    out = nv.nvfp4_gemm(A, ga, W, gw)
+    torch.cuda.synchronize()
+    y, mag, _, _ = o.linear(x, wt)
+    check_bf16(to_np(out), y, TOL_ACC * mag, f"decode M={M}")
