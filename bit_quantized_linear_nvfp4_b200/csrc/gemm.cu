@@ -110,6 +110,12 @@ __device__ __forceinline__ bool epi_is_bf16(int kind) {
   return kind == NVFP4_EPI_IDENTITY_BF16 || kind == NVFP4_EPI_SWIGLU_GATE;
 }
 
+__device__ __forceinline__ void st_global_v8(void* p, const uint32_t* w) {
+  asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(p), "r"(w[0]), "r"(w[1]),
+               "r"(w[2]), "r"(w[3]), "r"(w[4]), "r"(w[5]), "r"(w[6]), "r"(w[7])
+               : "memory");
+}
+
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<const uint32_t*>(&v);
@@ -130,25 +136,34 @@ __device__ __forceinline__ void store_chunk(const KernelArgs& a, int64_t row, in
     const int64_t j0 = n0 - sg.n_begin;
     if (bf16) {
       __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(sg.out) + row * sg.ld_out + j0;
+      const bool wide = (reinterpret_cast<uintptr_t>(dst) & 31u) == 0;
 #pragma unroll
-      for (int v = 0; v < 4; ++v) {
-        uint4 w;
-        w.x = pack_bf16(__uint_as_float(r[8 * v + 0]) * scale, __uint_as_float(r[8 * v + 1]) * scale);
-        w.y = pack_bf16(__uint_as_float(r[8 * v + 2]) * scale, __uint_as_float(r[8 * v + 3]) * scale);
-        w.z = pack_bf16(__uint_as_float(r[8 * v + 4]) * scale, __uint_as_float(r[8 * v + 5]) * scale);
-        w.w = pack_bf16(__uint_as_float(r[8 * v + 6]) * scale, __uint_as_float(r[8 * v + 7]) * scale);
-        *reinterpret_cast<uint4*>(dst + 8 * v) = w;
+      for (int g = 0; g < 2; ++g) {  // 16 values = one 32-byte sector per group
+        uint32_t w[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+          w[i] = pack_bf16(__uint_as_float(r[16 * g + 2 * i]) * scale, __uint_as_float(r[16 * g + 2 * i + 1]) * scale);
+        if (wide) {
+          st_global_v8(dst + 16 * g, w);
+        } else {
+          *reinterpret_cast<uint4*>(dst + 16 * g) = make_uint4(w[0], w[1], w[2], w[3]);
+          *reinterpret_cast<uint4*>(dst + 16 * g + 8) = make_uint4(w[4], w[5], w[6], w[7]);
+        }
       }
     } else {
       float* dst = static_cast<float*>(sg.out) + row * sg.ld_out + j0;
+      const bool wide = (reinterpret_cast<uintptr_t>(dst) & 31u) == 0;
 #pragma unroll
-      for (int v = 0; v < 8; ++v) {
-        float4 w;
-        w.x = apply_epi(sg, __uint_as_float(r[4 * v + 0]) * scale, j0 + 4 * v + 0);
-        w.y = apply_epi(sg, __uint_as_float(r[4 * v + 1]) * scale, j0 + 4 * v + 1);
-        w.z = apply_epi(sg, __uint_as_float(r[4 * v + 2]) * scale, j0 + 4 * v + 2);
-        w.w = apply_epi(sg, __uint_as_float(r[4 * v + 3]) * scale, j0 + 4 * v + 3);
-        *reinterpret_cast<float4*>(dst + 4 * v) = w;
+      for (int g = 0; g < 4; ++g) {
+        uint32_t w[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) w[i] = __float_as_uint(apply_epi(sg, __uint_as_float(r[8 * g + i]) * scale, j0 + 8 * g + i));
+        if (wide) {
+          st_global_v8(dst + 8 * g, w);
+        } else {
+          *reinterpret_cast<uint4*>(dst + 8 * g) = make_uint4(w[0], w[1], w[2], w[3]);
+          *reinterpret_cast<uint4*>(dst + 8 * g + 4) = make_uint4(w[4], w[5], w[6], w[7]);
+        }
       }
     }
     return;
@@ -187,14 +202,16 @@ __device__ __forceinline__ void store_swiglu(const KernelArgs& a, int64_t row, i
   }
   __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(sg.out) + row * sg.ld_out + o0;
   if (o0 + 31 < a.n_out && (o0 % 8) == 0) {
+    uint32_t w[16];
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      uint4 w;
-      w.x = pack_bf16(v[8 * q + 0], v[8 * q + 1]);
-      w.y = pack_bf16(v[8 * q + 2], v[8 * q + 3]);
-      w.z = pack_bf16(v[8 * q + 4], v[8 * q + 5]);
-      w.w = pack_bf16(v[8 * q + 6], v[8 * q + 7]);
-      *reinterpret_cast<uint4*>(dst + 8 * q) = w;
+    for (int i = 0; i < 16; ++i) w[i] = pack_bf16(v[2 * i], v[2 * i + 1]);
+    if ((reinterpret_cast<uintptr_t>(dst) & 31u) == 0) {
+      st_global_v8(dst, w);
+      st_global_v8(dst + 16, w + 8);
+    } else {
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+        *reinterpret_cast<uint4*>(dst + 8 * q) = make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
     }
   } else {
 #pragma unroll
@@ -406,13 +423,21 @@ constexpr int kSFSlotBytes = kSFASlotBytes + kSFBSlotBytes;
 constexpr int kSmemBytes2 = kStages2 * kCodeStage2 + kSFSlots * kSFSlotBytes + 1024 + 256;
 static_assert(kCodeStage2 % 1024 == 0 && kSFSlotBytes % 1024 == 0, "buffers keep 1024-byte alignment");
 
+// Two accumulators that share 64 TMEM columns: buffer 0 is columns
+// [0, 256), buffer 1 is [192, 448), scales follow at 448.  The epilogue reads
+// the shared columns first and releases them on ovl_free, so the next tile's
+// MMAs (which overwrite them) wait for a 64-column read, not the whole drain.
+constexpr uint32_t kColSFA2 = 448, kColSFB2 = 464;
+__device__ __forceinline__ uint32_t col_acc2(int buf) { return buf ? 192u : 0u; }
+
 struct SharedTail2 {
   uint64_t full[kStages2];
   uint64_t empty[kStages2];
   uint64_t sf_full[kSFSlots];
   uint64_t sf_empty[kSFSlots];
-  uint64_t tmem_full;
-  uint64_t tmem_empty;
+  uint64_t tmem_full[2];
+  uint64_t tmem_empty[2];
+  uint64_t ovl_free[2];
   uint64_t drain;
   uint32_t tmem_base;
   int abort_flag;
@@ -446,8 +471,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&tail->sf_full[s], 1);
       mbar_init(&tail->sf_empty[s], 1);
     }
-    mbar_init(&tail->tmem_full, 1);
-    mbar_init(&tail->tmem_empty, 2 * kNumEpiWarps);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&tail->tmem_full[b], 1);
+      mbar_init(&tail->tmem_empty[b], 2 * kNumEpiWarps);
+      mbar_init(&tail->ovl_free[b], kNumEpiWarps);  // the 4 warps per CTA holding the shared columns
+    }
     mbar_init(&tail->drain, 1);
     tail->abort_flag = 0;
     fence_mbarrier_init();
@@ -535,9 +563,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = true;
       bool any_issued = false;
       for (int t = pair; t < num_tiles && ok; t += num_pairs, ++local) {
-        if (local > 0) {
-          if (!mbar_wait_bounded(&tail->tmem_empty, (local - 1) & 1, abort_flag)) { ok = false; break; }
-        }
+        const int buf = local & 1;
+        // shared columns read by the previous tile's epilogue; own columns drained two tiles ago
+        if (local >= 1 &&
+            !mbar_wait_bounded(&tail->ovl_free[buf ^ 1], ((local - 1) >> 1) & 1, abort_flag)) { ok = false; break; }
+        if (local >= 2 &&
+            !mbar_wait_bounded(&tail->tmem_empty[buf], ((local - 2) >> 1) & 1, abort_flag)) { ok = false; break; }
         tc_fence_after();
         for (int ks = 0; ks < KS; ++ks) {
           const int j = ks % kSFGroup;
@@ -553,16 +584,16 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t ssfb1 = ssfb0 + kSFBSlotBytes / 2;
 #pragma unroll
           for (int kb = 0; kb < 4; ++kb) {
-            tmem_cp_32x128b_warpx4_pair(tmem + kColSFA + 4 * kb, make_smem_desc(ssfa + 512 * kb, 0, 128, kLayoutSwizzleNone));
-            tmem_cp_32x128b_warpx4_pair(tmem + kColSFB + 8 * kb, make_smem_desc(ssfb0 + 512 * kb, 0, 128, kLayoutSwizzleNone));
-            tmem_cp_32x128b_warpx4_pair(tmem + kColSFB + 8 * kb + 4, make_smem_desc(ssfb1 + 512 * kb, 0, 128, kLayoutSwizzleNone));
+            tmem_cp_32x128b_warpx4_pair(tmem + kColSFA2 + 4 * kb, make_smem_desc(ssfa + 512 * kb, 0, 128, kLayoutSwizzleNone));
+            tmem_cp_32x128b_warpx4_pair(tmem + kColSFB2 + 8 * kb, make_smem_desc(ssfb0 + 512 * kb, 0, 128, kLayoutSwizzleNone));
+            tmem_cp_32x128b_warpx4_pair(tmem + kColSFB2 + 8 * kb + 4, make_smem_desc(ssfb1 + 512 * kb, 0, 128, kLayoutSwizzleNone));
           }
           const uint64_t adesc = make_smem_desc(sa, 16, 1024, kLayoutSwizzle128B);
           const uint64_t bdesc = make_smem_desc(sb, 16, 1024, kLayoutSwizzle128B);
 #pragma unroll
           for (int kb = 0; kb < 4; ++kb)
-            mma_mxf4nvf4_pair(tmem + kColAcc, adesc + 2 * kb, bdesc + 2 * kb, idesc, tmem + kColSFA + 4 * kb,
-                              tmem + kColSFB + 8 * kb, (ks | kb) != 0 ? 1u : 0u);
+            mma_mxf4nvf4_pair(tmem + col_acc2(buf), adesc + 2 * kb, bdesc + 2 * kb, idesc, tmem + kColSFA2 + 4 * kb,
+                              tmem + kColSFB2 + 8 * kb, (ks | kb) != 0 ? 1u : 0u);
           any_issued = true;
           tc_commit_pair_mc(&tail->empty[stage], 0x3);
           if (++stage == kStages2) { stage = 0; phase ^= 1u; }
@@ -572,7 +603,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         if (!ok) break;
-        tc_commit_pair_mc(&tail->tmem_full, 0x3);
+        tc_commit_pair_mc(&tail->tmem_full[buf], 0x3);
       }
       if (*abort_flag && any_issued) {
         tc_commit_pair_mc(&tail->drain, 0x1);
@@ -583,30 +614,59 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------ epilogue (both CTAs)
     const int q = warp & 3;
     const int h = (warp - 2) >> 2;
-    const uint32_t empty_leader = map_to_rank(smem_u32(&tail->tmem_empty), 0);
+    uint32_t empty_leader[2], ovl_leader[2];
+    for (int b = 0; b < 2; ++b) {
+      empty_leader[b] = map_to_rank(smem_u32(&tail->tmem_empty[b]), 0);
+      ovl_leader[b] = map_to_rank(smem_u32(&tail->ovl_free[b]), 0);
+    }
+    // chunk c of this warp sits at buffer column cc[c]; the shared columns are
+    // buffer 0's [192, 256) (chunks 2, 3 of the h = 1 warps) and buffer 1's
+    // [0, 64) (chunks 0, 1 of the h = 0 warps), in both layouts
+    uint32_t cc[4];
+    if (!args.swiglu) {
+      cc[0] = h * 128; cc[1] = h * 128 + 32; cc[2] = h * 128 + 64; cc[3] = h * 128 + 96;
+    } else {
+      cc[0] = h * 64; cc[1] = h * 64 + 32; cc[2] = 128 + h * 64; cc[3] = 128 + h * 64 + 32;
+    }
     int local = 0;
     for (int t = pair; t < num_tiles; t += num_pairs, ++local) {
       int m_blk, n_blk;
       tile_coords(args, t, m_blk, n_blk);
-      if (!mbar_wait_bounded(&tail->tmem_full, local & 1, abort_flag)) break;
+      const int buf = local & 1;
+      if (!mbar_wait_bounded(&tail->tmem_full[buf], (local >> 1) & 1, abort_flag)) break;
       tc_fence_after();
-      const uint32_t lane_addr = tmem + (static_cast<uint32_t>(q * 32) << 16);
+      const uint32_t base = tmem + (static_cast<uint32_t>(q * 32) << 16) + col_acc2(buf);
       uint32_t r0[32], r1[32], r2[32], r3[32];
-      if (!args.swiglu) {
-        tmem_ld_32x32b_x32(lane_addr + kColAcc + h * 128 + 0, r0);
-        tmem_ld_32x32b_x32(lane_addr + kColAcc + h * 128 + 32, r1);
-        tmem_ld_32x32b_x32(lane_addr + kColAcc + h * 128 + 64, r2);
-        tmem_ld_32x32b_x32(lane_addr + kColAcc + h * 128 + 96, r3);
+      const bool shared = h == (buf ? 0 : 1);
+      if (shared) {
+        if (buf == 0) {
+          tmem_ld_32x32b_x32(base + cc[2], r2);
+          tmem_ld_32x32b_x32(base + cc[3], r3);
+        } else {
+          tmem_ld_32x32b_x32(base + cc[0], r0);
+          tmem_ld_32x32b_x32(base + cc[1], r1);
+        }
+        tmem_ld_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_remote(ovl_leader[buf]);
+        if (buf == 0) {
+          tmem_ld_32x32b_x32(base + cc[0], r0);
+          tmem_ld_32x32b_x32(base + cc[1], r1);
+        } else {
+          tmem_ld_32x32b_x32(base + cc[2], r2);
+          tmem_ld_32x32b_x32(base + cc[3], r3);
+        }
       } else {
-        tmem_ld_32x32b_x32(lane_addr + kColAcc + h * 64 + 0, r0);
-        tmem_ld_32x32b_x32(lane_addr + kColAcc + h * 64 + 32, r1);
-        tmem_ld_32x32b_x32(lane_addr + kColAcc + 128 + h * 64 + 0, r2);
-        tmem_ld_32x32b_x32(lane_addr + kColAcc + 128 + h * 64 + 32, r3);
+        tmem_ld_32x32b_x32(base + cc[0], r0);
+        tmem_ld_32x32b_x32(base + cc[1], r1);
+        tmem_ld_32x32b_x32(base + cc[2], r2);
+        tmem_ld_32x32b_x32(base + cc[3], r3);
       }
       tmem_ld_wait();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive_remote(empty_leader);
+      if (lane == 0) mbar_arrive_remote(empty_leader[buf]);
 
       const int64_t row = static_cast<int64_t>(m_blk) * 256 + rank * 128 + q * 32 + lane;
       if (row < args.M) {
@@ -942,7 +1002,19 @@ cudaError_t launch_gemm(const GemmProblem& p, void*, size_t, cudaStream_t stream
     gemm_kernel<<<grid, kThreads, kSmemBytes, stream>>>(tm_a, tm_b, tm_sfa, tm_sfb, a);
     return cudaGetLastError();
   }
+  // Non-SwiGLU projections run either 192-wide double-buffered tiles or
+  // 256-wide tiles with overlapping accumulators.  The 256-wide tile moves
+  // about 17% fewer operand bytes per MMA clock; the 192-wide tile can fill
+  // the last wave better.  Pick the smaller estimated time.
+  bool n192 = false;
   if (!p.swiglu) {
+    const int64_t pairs_avail = sms / 2;
+    const int64_t mb = ceil_div(p.M, 256);
+    const double t192 = static_cast<double>(ceil_div(mb * ceil_div(p.N, BN3), pairs_avail)) * 192.0;
+    const double t256 = static_cast<double>(ceil_div(mb * ceil_div(p.N, BN), pairs_avail)) * 256.0 * 0.9;
+    n192 = t192 < t256;
+  }
+  if (n192) {
     KernelArgs b = a;
     b.num_n_blocks = static_cast<int>(ceil_div(p.N, BN3));
     CUtensorMap tm_b3, tm_sfb3;
