@@ -1011,7 +1011,7 @@ cudaError_t launch_gemm(const GemmProblem& p, void*, size_t, cudaStream_t stream
     const int64_t pairs_avail = sms / 2;
     const int64_t mb = ceil_div(p.M, 256);
     const double t192 = static_cast<double>(ceil_div(mb * ceil_div(p.N, BN3), pairs_avail)) * 192.0;
-    const double t256 = static_cast<double>(ceil_div(mb * ceil_div(p.N, BN), pairs_avail)) * 256.0 * 0.9;
+    const double t256 = static_cast<double>(ceil_div(mb * ceil_div(p.N, BN), pairs_avail)) * 256.0 * 0.95;
     n192 = t192 < t256;
   }
   if (n192) {

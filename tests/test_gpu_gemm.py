@@ -266,3 +266,23 @@ def test_full_size_decode(M):
     torch.cuda.synchronize()
     y, mag, _, _ = o.linear(x, wt)
     check_bf16(to_np(out), y, TOL_ACC * mag, f"decode M={M}")
+
+
+def test_wide_tiles_two_segments():
+    """A shape that runs the 256-wide overlapped-accumulator kernel for a
+    non-SwiGLU projection (one M block, N just above 74 x 192), with a BF16
+    and an FP32 segment."""
+    M, K, N = 200, 256, 14336
+    x = _rand(M, K, 61, outliers=2)
+    w0 = _rand(8192, K, 62, 0.02)
+    w1 = _rand(N - 8192, K, 63, 0.05)
+    A, ga = nv.nvfp4_quantize(_dev(x))
+    W, gw = nv.nvfp4_quantize_segments(_dev(np.concatenate([w0, w1])), [0, 8192, N])
+    o0 = torch.empty((M, 8192), dtype=torch.bfloat16, device=DEV)
+    o1 = torch.empty((M, N - 8192), dtype=torch.float32, device=DEV)
+    nv.nvfp4_fused_proj(A, ga, W, gw, [nv.Segment(0, 8192, "identity_bf16", o0), nv.Segment(8192, N, "identity_f32", o1)])
+    torch.cuda.synchronize()
+    y0, m0, _, _ = o.linear(x, w0)
+    y1, m1, _, _ = o.linear(x, w1)
+    check_bf16(to_np(o0), y0, TOL_ACC * m0, "wide bf16")
+    check_fp32(to_np(o1), y1, m1, "wide f32")
