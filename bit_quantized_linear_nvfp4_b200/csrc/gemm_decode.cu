@@ -34,30 +34,36 @@ namespace nvfp4 {
 namespace dk {
 
 constexpr int BM = 128;  // weight rows per CTA (MMA M)
-constexpr int BK = 256;
-constexpr int kWBytes = BM * BK / 2;     // 16 KB
-constexpr int kSFWBytes = BM * BK / 16;  // 2 KB
-constexpr int kSFXBytes = 128 * BK / 16; // 2 KB (one 128-row atom per 64 K)
+constexpr int BK = 256;  // K elements per 128-byte chunk of a row
 constexpr int kEpiWarps = 4;
 constexpr int kThreads = 64 + kEpiWarps * 32;
-constexpr uint32_t kTmemCols = 128;
+constexpr uint32_t kTmemCols = 256;
 constexpr int kSmemBudget = 200 * 1024;
 
-// BN token columns (MMA N = 16, 32 or 64; tokens beyond M are zero rows of X).
-// The stage count fills the shared-memory budget, so fewer tokens means more
-// weight bytes in flight per CTA.
-template <int BN>
+// BN token columns (MMA N = 16, 32 or 64; tokens beyond M are zero rows of X)
+// and CH K-chunks of 256 per stage.  Each stage is four TMA copies (W codes,
+// X codes, W scales, X scales); a copy costs about the same whatever its
+// size, so with CH = 4 one 64 KB weight box carries four chunks at once.  CH
+// > 1 views the codes as 3-D {128 B, rows, K/256} and needs K % 256 == 0;
+// CH = 1 uses the row-clipped 2-D view.
+template <int BN, int CH>
 struct DCfg {
-  static constexpr int kXBytes = BN * BK / 2;
+  static constexpr int kWBytes = BM * BK / 2 * CH;
+  static constexpr int kXPlane = BN * BK / 2;  // one chunk of X
+  static constexpr int kXBytes = kXPlane * CH;
+  static constexpr int kSFWBytes = BM * BK / 16 * CH;
+  static constexpr int kSFXBytes = 128 * BK / 16 * CH;  // 128-row atoms
   static constexpr int kStageRaw = kWBytes + kXBytes + kSFWBytes + kSFXBytes;
   static constexpr int kStageBytes = (kStageRaw + 1023) / 1024 * 1024;
   static constexpr int kStages = kSmemBudget / kStageBytes;
-  static constexpr uint32_t kColAcc = 0, kColSFW = 64, kColSFX = 80;
+  static constexpr uint32_t kColAcc = 0, kColSFW = 64, kColSFX = 64 + 16 * CH;
   static constexpr int kPartialBytes = BN * BM * 4;  // staged over the first stages
   static constexpr int kSmemBytes = kStages * kStageBytes + 1024 + 512;
   static_assert(kPartialBytes <= kStages * kStageBytes, "partial fits in the stage buffers");
+  static_assert(kColSFX + 16 * CH <= kTmemCols, "scales fit in TMEM");
+  static_assert(kStages >= 2, "at least two stages");
 };
-constexpr int kMaxStages = kSmemBudget / ((kWBytes + 16 * BK / 2 + kSFWBytes + kSFXBytes + 1023) / 1024 * 1024);
+constexpr int kMaxStages = 12;
 
 struct DecodeArgs {
   int64_t M, N, K;
@@ -84,15 +90,17 @@ __device__ __forceinline__ float softplus_f(float t) {
   return t > 0.0f ? t + log1pf(expf(-t)) : log1pf(expf(t));
 }
 
-template <int BN>
+template <int BN, int CH>
 __global__ void __launch_bounds__(kThreads, 1)
     decode_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_x,
                   const __grid_constant__ CUtensorMap tm_sfw, const __grid_constant__ CUtensorMap tm_sfx,
                   const __grid_constant__ DecodeArgs args) {
-  using C = DCfg<BN>;
+  using C = DCfg<BN, CH>;
   constexpr int kStages = C::kStages;
   constexpr int kStageBytes = C::kStageBytes;
+  constexpr int kWBytes = C::kWBytes;
   constexpr int kXBytes = C::kXBytes;
+  constexpr int kSFWBytes = C::kSFWBytes;
   constexpr uint32_t kColAcc = C::kColAcc, kColSFW = C::kColSFW, kColSFX = C::kColSFX;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -143,11 +151,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!mbar_wait_bounded(&tail->empty[stage], phase ^ 1u, abort_flag)) break;
         uint8_t* st = smem + stage * kStageBytes;
         mbar_arrive_expect_tx(&tail->full[stage], C::kStageRaw);
-        const int32_t kx = ks * (BK / 2);
-        tma_load_2d(st, &tm_w, &tail->full[stage], kx, rb * BM);
-        tma_load_2d(st + kWBytes, &tm_x, &tail->full[stage], kx, 0);
-        tma_load_3d(st + kWBytes + kXBytes, &tm_sfw, &tail->full[stage], 0, ks * 4, rb);
-        tma_load_3d(st + kWBytes + kXBytes + kSFWBytes, &tm_sfx, &tail->full[stage], 0, ks * 4, 0);
+        if constexpr (CH == 1) {
+          const int32_t kx = ks * (BK / 2);
+          tma_load_2d(st, &tm_w, &tail->full[stage], kx, rb * BM);
+          tma_load_2d(st + kWBytes, &tm_x, &tail->full[stage], kx, 0);
+        } else {
+          tma_load_3d(st, &tm_w, &tail->full[stage], 0, rb * BM, ks * CH);
+          tma_load_3d(st + kWBytes, &tm_x, &tail->full[stage], 0, 0, ks * CH);
+        }
+        tma_load_3d(st + kWBytes + kXBytes, &tm_sfw, &tail->full[stage], 0, ks * 4 * CH, rb);
+        tma_load_3d(st + kWBytes + kXBytes + kSFWBytes, &tm_sfx, &tail->full[stage], 0, ks * 4 * CH, 0);
         issued[stage] = true;
         issued_phase[stage] = phase;
         if (++stage == kStages) { stage = 0; phase ^= 1u; }
@@ -173,16 +186,19 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t ssfw = sx + kXBytes;
         const uint32_t ssfx = ssfw + kSFWBytes;
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          tmem_cp_32x128b_warpx4(tmem + kColSFW + 4 * j, make_smem_desc(ssfw + 512 * j, 0, 128, kLayoutSwizzleNone));
-          tmem_cp_32x128b_warpx4(tmem + kColSFX + 4 * j, make_smem_desc(ssfx + 512 * j, 0, 128, kLayoutSwizzleNone));
+        for (int kb = 0; kb < 4 * CH; ++kb) {
+          tmem_cp_32x128b_warpx4(tmem + kColSFW + 4 * kb, make_smem_desc(ssfw + 512 * kb, 0, 128, kLayoutSwizzleNone));
+          tmem_cp_32x128b_warpx4(tmem + kColSFX + 4 * kb, make_smem_desc(ssfx + 512 * kb, 0, 128, kLayoutSwizzleNone));
         }
-        const uint64_t wdesc = make_smem_desc(sw, 16, 1024, kLayoutSwizzle128B);
-        const uint64_t xdesc = make_smem_desc(sx, 16, 1024, kLayoutSwizzle128B);
 #pragma unroll
-        for (int j = 0; j < 4; ++j)
-          mma_mxf4nvf4(tmem + kColAcc, wdesc + 2 * j, xdesc + 2 * j, idesc, tmem + kColSFW + 4 * j,
-                       tmem + kColSFX + 4 * j, (ks > ks0 || j > 0) ? 1u : 0u);
+        for (int c = 0; c < CH; ++c) {
+          const uint64_t wdesc = make_smem_desc(sw + c * (BM * BK / 2), 16, 1024, kLayoutSwizzle128B);
+          const uint64_t xdesc = make_smem_desc(sx + c * C::kXPlane, 16, 1024, kLayoutSwizzle128B);
+#pragma unroll
+          for (int j = 0; j < 4; ++j)
+            mma_mxf4nvf4(tmem + kColAcc, wdesc + 2 * j, xdesc + 2 * j, idesc, tmem + kColSFW + 4 * (4 * c + j),
+                         tmem + kColSFX + 4 * (4 * c + j), (ks > ks0 || c > 0 || j > 0) ? 1u : 0u);
+        }
         any = true;
         tc_commit(&tail->empty[stage]);
         if (++stage == kStages) { stage = 0; phase ^= 1u; }
@@ -295,18 +311,35 @@ __global__ void __launch_bounds__(kThreads, 1)
 bool decode_path_applies(const GemmProblem& p) { return p.M >= 1 && p.M <= 64 && !p.swiglu; }
 
 namespace dk {
-template <int BN>
+
+// Codes [rows, K/2] viewed as {128 B, rows, K/256}: one box spans CH chunks of
+// box_rows rows (needs K % 256 == 0 so that every chunk lies inside its row).
+bool make_codes_map3(CUtensorMap* m, const uint8_t* codes, int64_t rows, int64_t K, uint32_t box_rows, uint32_t chunks) {
+  const cuuint64_t dims[3] = {128, static_cast<cuuint64_t>(rows), static_cast<cuuint64_t>(K / 256)};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(K / 2), 128};
+  const cuuint32_t box[3] = {128, box_rows, chunks};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return gk::encode_fn()(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<uint8_t*>(codes), dims, strides, box, estr,
+                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int BN, int CH>
 cudaError_t launch_bn(const GemmProblem& p, cudaStream_t stream) {
-  using C = DCfg<BN>;
+  using C = DCfg<BN, CH>;
   CUtensorMap tm_w, tm_x, tm_sfw, tm_sfx;
-  if (!gk::make_codes_map(&tm_w, p.w_codes, p.N, p.K, BM) || !gk::make_codes_map(&tm_x, p.a_codes, p.M, p.K, BN) ||
-      !gk::make_sf_map(&tm_sfw, p.w_sf, p.N, p.K) || !gk::make_sf_map(&tm_sfx, p.a_sf, p.M, p.K))
+  bool ok;
+  if constexpr (CH == 1)
+    ok = gk::make_codes_map(&tm_w, p.w_codes, p.N, p.K, BM) && gk::make_codes_map(&tm_x, p.a_codes, p.M, p.K, BN);
+  else
+    ok = make_codes_map3(&tm_w, p.w_codes, p.N, p.K, BM, CH) && make_codes_map3(&tm_x, p.a_codes, p.M, p.K, BN, CH);
+  if (!ok || !gk::make_sf_map(&tm_sfw, p.w_sf, p.N, p.K, 4 * CH, 1) || !gk::make_sf_map(&tm_sfx, p.a_sf, p.M, p.K, 4 * CH, 1))
     return cudaErrorInvalidValue;
   DecodeArgs a{};
   a.M = p.M;
   a.N = p.N;
   a.K = p.K;
-  a.num_k_stages = static_cast<int>(ceil_div(p.K, BK));
+  a.num_k_stages = static_cast<int>(ceil_div(ceil_div(p.K, BK), CH));
   a.g_a = p.g_a;
   a.seg_scale = p.seg_scale;
   a.nseg = p.nseg;
@@ -322,7 +355,7 @@ cudaError_t launch_bn(const GemmProblem& p, cudaStream_t stream) {
   a.split = S;
   static bool attr_set = false;
   if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(decode_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+    cudaError_t e = cudaFuncSetAttribute(decode_kernel<BN, CH>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
@@ -338,14 +371,15 @@ cudaError_t launch_bn(const GemmProblem& p, cudaStream_t stream) {
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, decode_kernel<BN>, tm_w, tm_x, tm_sfw, tm_sfx, a);
+  return cudaLaunchKernelEx(&cfg, decode_kernel<BN, CH>, tm_w, tm_x, tm_sfw, tm_sfx, a);
 }
 }  // namespace dk
 
 cudaError_t launch_gemm_decode(const GemmProblem& p, cudaStream_t stream) {
-  if (p.M <= 16) return dk::launch_bn<16>(p, stream);
-  if (p.M <= 32) return dk::launch_bn<32>(p, stream);
-  return dk::launch_bn<64>(p, stream);
+  const bool wide = p.K % 256 == 0;
+  if (p.M <= 16) return wide ? dk::launch_bn<16, 4>(p, stream) : dk::launch_bn<16, 1>(p, stream);
+  if (p.M <= 32) return wide ? dk::launch_bn<32, 4>(p, stream) : dk::launch_bn<32, 1>(p, stream);
+  return wide ? dk::launch_bn<64, 2>(p, stream) : dk::launch_bn<64, 1>(p, stream);
 }
 
 }  // namespace nvfp4
