@@ -227,28 +227,40 @@ class ProductStep:
     def gemm(self, s):
         self.nv.nvfp4_fused_proj(s["A"], s["g"], s["W"], s["gw"], s["segs"])
 
+    def linear(self, s):
+        # the whole layer in one call: quantise x, then the fused projection
+        self.nv.nvfp4_linear(s["x"], s["W"], s["gw"], s["segs"], a_codes=s["codes"], a_sf=s["sf"],
+                             g_a=s["g"], workspace=s["ws"])
+
     def launches_per_step(self):
         return 2 if self.w is None else 3  # amax, quantize (+ GEMM)
 
     def capture(self):
         torch = self.torch
-        self.gq, self.gg = [], []
+        self.gq, self.gg, self.gl = [], [], []
         for s in self.sets:  # warm the launch path once outside capture
             self.quantize(s)
             if self.w is not None:
                 self.gemm(s)
+                self.linear(s)
         torch.cuda.synchronize()
+
+        def graph(fn, s):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                fn(s)
+            return g
+
         for s in self.sets:
-            g1 = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(g1):
-                self.quantize(s)
-            self.gq.append(g1)
+            self.gq.append(graph(self.quantize, s))
             if self.w is not None:
-                g2 = torch.cuda.CUDAGraph()
-                with torch.cuda.graph(g2):
-                    self.gemm(s)
-                self.gg.append(g2)
+                self.gg.append(graph(self.gemm, s))
+                self.gl.append(graph(self.linear, s))
         torch.cuda.synchronize()
+
+    def step_graph(self, r):
+        """One pass of the whole path: the layer call (or the quantiser alone)."""
+        return self.gl[r] if self.w is not None else self.gq[r]
 
     def alg_bytes_quant(self):
         # amax pass reads X; the quantiser reads X and writes codes + scales
@@ -283,34 +295,40 @@ def run_product(args):
     K, Wm = args.steps, args.warmup
     R = len(step.sets)
 
-    def one(i, evs=None):
+    def staged(i, evs):
+        # the two stages as separate calls, an event on each side of each
         r = i % R
-        if evs is not None:
-            evs[0].record(stream)
+        evs[0].record(stream)
         step.gq[r].replay()
-        if evs is not None:
-            evs[1].record(stream)
+        evs[1].record(stream)
         if step.w is not None:
             step.gg[r].replay()
-        if evs is not None:
-            evs[2].record(stream)
+        evs[2].record(stream)
 
     for i in range(Wm):
-        one(i)
+        step.step_graph(i % R).replay()
     torch.cuda.synchronize()
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     clocks = ClockSampler(local)
     clocks.start()
     time.sleep(0.3)
+    # timed region: K steps, each one pass of the path (the layer call)
     dist_barrier(dist)
     torch.cuda.synchronize()
     t0.record(stream)
     for i in range(K):
-        one(i, evs[i])
+        step.step_graph(i % R).replay()
     t1.record(stream)
     torch.cuda.synchronize()
     dist_barrier(dist)
+    # per-stage device times (dominant-kernel roofline), same inputs
+    for i in range(min(Wm, 3)):
+        staged(i, evs[i])
+    torch.cuda.synchronize()
+    for i in range(K):
+        staged(i, evs[i])
+    torch.cuda.synchronize()
     clk = clocks.stop()
     total_ms = t0.elapsed_time(t1)
     total_ms = dist_max(dist, total_ms, device)
@@ -365,7 +383,7 @@ def run_product(args):
         line["cpu_baseline"] = cpu_baseline(args.workload, target_s=args.cpu_seconds)
     if rank == 0:
         print(json.dumps(line), flush=True)
-    for g in step.gq + step.gg:
+    for g in step.gq + step.gg + step.gl:
         del g
     if dist is not None:
         dist.destroy_process_group()
@@ -382,9 +400,7 @@ def measure_e2e(step, K, Wm, stream):
 
     def one():
         s["x"].copy_(x_host, non_blocking=True)
-        step.gq[0].replay()
-        if step.w is not None:
-            step.gg[0].replay()
+        step.step_graph(0).replay()
         for dst, src in zip(out_host, outs):
             dst.copy_(src, non_blocking=True)
 

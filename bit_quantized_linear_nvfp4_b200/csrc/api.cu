@@ -61,8 +61,7 @@ int quantize_impl(const void* x, int dtype, int64_t M, int64_t K, int64_t ld,
   st = check_device();
   if (st != NVFP4_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  unsigned int* bits = static_cast<unsigned int*>(ws);
-  cudaError_t e = nvfp4::launch_quantize(x, dtype, M, K, ld, segs, g_in, bits, g_out, codes, sf, s);
+  cudaError_t e = nvfp4::launch_quantize(x, dtype, M, K, ld, segs, g_in, ws, g_out, codes, sf, s);
   if (e != cudaSuccess) return cuda_fail(e);
   return NVFP4_OK;
 }
@@ -105,7 +104,7 @@ size_t nvfp4_sf_bytes(int64_t rows, int64_t K) {
 
 size_t nvfp4_quantize_workspace_bytes(int nseg) {
   if (nseg < 1) nseg = 1;
-  return 16 * ((nvfp4::quantize_scratch_words(nseg) * sizeof(unsigned int) + 15) / 16);
+  return 16 * ((nvfp4::quantize_scratch_bytes(nseg) + 15) / 16);
 }
 
 int nvfp4_quantize(const void* x, int x_dtype, int64_t M, int64_t K, int64_t ld_x,
@@ -139,9 +138,14 @@ size_t nvfp4_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K) {
   return nvfp4::gemm_workspace_bytes(M, N, K);
 }
 
-int nvfp4_fused_proj(const nvfp4_operand* A, const float* g_a, const nvfp4_operand* W,
-                     const float* seg_global_scale, const nvfp4_segment* segs, int nseg,
-                     void* workspace, size_t workspace_bytes, void* stream) {
+}  // extern "C"
+
+namespace {
+
+// Checks the arguments of one fused projection and describes it in *p.
+int build_problem(const nvfp4_operand* A, const float* g_a, const nvfp4_operand* W,
+                  const float* seg_global_scale, const nvfp4_segment* segs, int nseg,
+                  void* workspace, size_t workspace_bytes, nvfp4::GemmProblem* out) {
   int st = check_operand(A);
   if (st != NVFP4_OK) return st;
   st = check_operand(W);
@@ -150,7 +154,8 @@ int nvfp4_fused_proj(const nvfp4_operand* A, const float* g_a, const nvfp4_opera
   if (g_a == nullptr || seg_global_scale == nullptr || segs == nullptr) return NVFP4_ERR_INVALID_ARG;
   if (nseg < 1 || nseg > NVFP4_MAX_SEGMENTS) return NVFP4_ERR_INVALID_ARG;
 
-  nvfp4::GemmProblem p{};
+  nvfp4::GemmProblem& p = *out;
+  p = nvfp4::GemmProblem{};
   p.a_codes = A->codes;
   p.a_sf = A->sf;
   p.w_codes = W->codes;
@@ -201,9 +206,68 @@ int nvfp4_fused_proj(const nvfp4_operand* A, const float* g_a, const nvfp4_opera
   if (workspace_bytes < nvfp4::gemm_workspace_bytes(p.M, p.N, p.K) ||
       (nvfp4::gemm_workspace_bytes(p.M, p.N, p.K) > 0 && workspace == nullptr))
     return NVFP4_ERR_WORKSPACE;
-  st = check_device();
+  return check_device();
+}
+
+// [p, p + n) and [q, q + m) share a byte.
+bool overlap(const void* p, size_t n, const void* q, size_t m) {
+  const uintptr_t a = reinterpret_cast<uintptr_t>(p), b = reinterpret_cast<uintptr_t>(q);
+  return n != 0 && m != 0 && a < b + m && b < a + n;
+}
+
+}  // namespace
+
+extern "C" {
+
+int nvfp4_fused_proj(const nvfp4_operand* A, const float* g_a, const nvfp4_operand* W,
+                     const float* seg_global_scale, const nvfp4_segment* segs, int nseg,
+                     void* workspace, size_t workspace_bytes, void* stream) {
+  nvfp4::GemmProblem p;
+  int st = build_problem(A, g_a, W, seg_global_scale, segs, nseg, workspace, workspace_bytes, &p);
   if (st != NVFP4_OK) return st;
   cudaError_t e = nvfp4::launch_gemm(p, workspace, workspace_bytes, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e);
+  return NVFP4_OK;
+}
+
+int nvfp4_linear(const void* x, int x_dtype, int64_t M, int64_t K, int64_t ld_x, const float* g_in,
+                 uint8_t* a_codes, uint8_t* a_sf, float* g_a, const nvfp4_operand* W,
+                 const float* seg_global_scale, const nvfp4_segment* segs, int nseg, void* workspace,
+                 size_t workspace_bytes, void* stream) {
+  int st = check_quant_args(x, x_dtype, M, K, ld_x, g_a, a_codes, a_sf);
+  if (st != NVFP4_OK) return st;
+  st = check_operand(W);
+  if (st != NVFP4_OK) return st;
+  if (W->K != K) return NVFP4_ERR_INVALID_ARG;
+  if (M == 0) return NVFP4_OK;
+  if (g_in == nullptr && (workspace == nullptr || workspace_bytes < nvfp4_quantize_workspace_bytes(1) ||
+                          !aligned16(workspace)))
+    return NVFP4_ERR_WORKSPACE;
+  // The GEMM may read W while the quantiser still runs: nothing the quantiser
+  // writes may share memory with W or the segment scales.
+  const size_t wc = static_cast<size_t>(W->rows) * static_cast<size_t>(K / 2);
+  const size_t ws = nvfp4::sf_bytes(W->rows, K);
+  const size_t nsc = seg_global_scale ? sizeof(float) * static_cast<size_t>(nseg > 0 ? nseg : 0) : 0;
+  const size_t ac = static_cast<size_t>(M) * static_cast<size_t>(K / 2), as = nvfp4::sf_bytes(M, K);
+  const size_t wsb = g_in == nullptr ? nvfp4_quantize_workspace_bytes(1) : 0;
+  const void* written[4] = {a_codes, a_sf, g_a, workspace};
+  const size_t wbytes[4] = {ac, as, sizeof(float), wsb};
+  for (int i = 0; i < 4; ++i)
+    if (overlap(written[i], wbytes[i], W->codes, wc) || overlap(written[i], wbytes[i], W->sf, ws) ||
+        overlap(written[i], wbytes[i], seg_global_scale, nsc))
+      return NVFP4_ERR_INVALID_ARG;
+  nvfp4_operand A{a_codes, a_sf, M, K};
+  nvfp4::GemmProblem p;
+  st = build_problem(&A, g_a, W, seg_global_scale, segs, nseg, nullptr, 0, &p);
+  if (st != NVFP4_OK) return st;
+  nvfp4::RowSegments one{};
+  one.n = 1;
+  one.begin[0] = 0;
+  one.begin[1] = M;
+  st = quantize_impl(x, x_dtype, M, K, ld_x, one, g_in, g_a, a_codes, a_sf, workspace, workspace_bytes, stream);
+  if (st != NVFP4_OK) return st;
+  p.w_prefetch = true;  // the kernel before the GEMM is the quantiser, which leaves W alone
+  cudaError_t e = nvfp4::launch_gemm(p, nullptr, 0, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e);
   return NVFP4_OK;
 }

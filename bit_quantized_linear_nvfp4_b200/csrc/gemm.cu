@@ -256,6 +256,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = tail->tmem_base;
+  // Everything above may overlap the previous kernel on the stream; operands,
+  // scales and outputs are touched only after the wait (the MMA warp reads
+  // shared memory and TMEM only).
+  if (warp != 1) grid_dependency_wait();
+  if (threadIdx.x == 0) grid_launch_dependents();
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -493,6 +498,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   cluster_sync_all();  // both CTAs' barriers exist before any cross-CTA signal
   tc_fence_after();
   const uint32_t tmem = tail->tmem_base;
+  // Everything above may overlap the previous kernel on the stream; operands,
+  // scales and outputs are touched only after the wait (the MMA warp reads
+  // shared memory and TMEM only).
+  if (warp != 1) grid_dependency_wait();
+  if (threadIdx.x == 0) grid_launch_dependents();
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer (both CTAs)
@@ -769,6 +779,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   cluster_sync_all();
   tc_fence_after();
   const uint32_t tmem = tail->tmem_base;
+  // Everything above may overlap the previous kernel on the stream; operands,
+  // scales and outputs are touched only after the wait (the MMA warp reads
+  // shared memory and TMEM only).
+  if (warp != 1) grid_dependency_wait();
+  if (threadIdx.x == 0) grid_launch_dependents();
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer (both CTAs)
@@ -998,9 +1013,17 @@ cudaError_t launch_gemm(const GemmProblem& p, void*, size_t, cudaStream_t stream
       if (e != cudaSuccess) return e;
       attr_set = true;
     }
-    const int grid = tiles < sms ? tiles : sms;
-    gemm_kernel<<<grid, kThreads, kSmemBytes, stream>>>(tm_a, tm_b, tm_sfa, tm_sfb, a);
-    return cudaGetLastError();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(tiles < sms ? tiles : sms);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = kSmemBytes;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, gemm_kernel, tm_a, tm_b, tm_sfa, tm_sfb, a);
   }
   // Non-SwiGLU projections run either 192-wide double-buffered tiles or
   // 256-wide tiles with overlapping accumulators.  The 256-wide tile moves
@@ -1033,13 +1056,15 @@ cudaError_t launch_gemm(const GemmProblem& p, void*, size_t, cudaStream_t stream
     cfg.blockDim = dim3(kThreads);
     cfg.dynamicSmemBytes = kSmemBytes3;
     cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = 2;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = 2;
     return cudaLaunchKernelEx(&cfg, gemm_pair_db_kernel, tm_a, tm_b3, tm_sfa, tm_sfb3, b);
   }
   CUtensorMap tm_sfa4, tm_sfb4, tm_sfb8;
@@ -1058,13 +1083,15 @@ cudaError_t launch_gemm(const GemmProblem& p, void*, size_t, cudaStream_t stream
   cfg.blockDim = dim3(kThreads);
   cfg.dynamicSmemBytes = kSmemBytes2;
   cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 2;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   return cudaLaunchKernelEx(&cfg, gemm_pair_kernel, tm_a, tm_b, tm_sfa4, tm_sfb4, tm_sfb8, a);
 }
 

@@ -57,7 +57,11 @@ struct DCfg {
   static constexpr int kStageBytes = (kStageRaw + 1023) / 1024 * 1024;
   static constexpr int kStages = kSmemBudget / kStageBytes;
   static constexpr uint32_t kColAcc = 0, kColSFW = 64, kColSFX = 64 + 16 * CH;
-  static constexpr int kPartialBytes = BN * BM * 4;  // staged over the first stages
+  // FP32 partial staged row-major over the first stages: row r's BN tokens at
+  // r * kPartLd floats; the 4-float pad spreads a quarter-warp's 128-bit
+  // accesses over all 32 banks.
+  static constexpr int kPartLd = BN + 4;
+  static constexpr int kPartialBytes = kPartLd * BM * 4;
   static constexpr int kSmemBytes = kStages * kStageBytes + 1024 + 512;
   static_assert(kPartialBytes <= kStages * kStageBytes, "partial fits in the stage buffers");
   static_assert(kColSFX + 16 * CH <= kTmemCols, "scales fit in TMEM");
@@ -68,6 +72,7 @@ constexpr int kMaxStages = 12;
 struct DecodeArgs {
   int64_t M, N, K;
   int num_k_stages, split;
+  int w_prefetch;  // W is not written by the kernel before this one on the stream
   const float* g_a;
   const float* seg_scale;
   int nseg;
@@ -143,24 +148,45 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == 0) {
     if (elect_one()) {
+      // W codes + scales, then X codes + scales, of K-stage ks into stage st;
+      // one full barrier completes on the bytes of all four copies.
+      auto load_w = [&](int stage, int ks) {
+        uint8_t* st = smem + stage * kStageBytes;
+        if constexpr (CH == 1)
+          tma_load_2d(st, &tm_w, &tail->full[stage], ks * (BK / 2), rb * BM);
+        else
+          tma_load_3d(st, &tm_w, &tail->full[stage], 0, rb * BM, ks * CH);
+        tma_load_3d(st + kWBytes + kXBytes, &tm_sfw, &tail->full[stage], 0, ks * 4 * CH, rb);
+      };
+      auto load_x = [&](int stage, int ks) {
+        uint8_t* st = smem + stage * kStageBytes;
+        if constexpr (CH == 1)
+          tma_load_2d(st + kWBytes, &tm_x, &tail->full[stage], ks * (BK / 2), 0);
+        else
+          tma_load_3d(st + kWBytes, &tm_x, &tail->full[stage], 0, 0, ks * CH);
+        tma_load_3d(st + kWBytes + kXBytes + kSFWBytes, &tm_sfx, &tail->full[stage], 0, ks * 4 * CH, 0);
+      };
       int stage = 0;
       uint32_t phase = 0;
       bool issued[kStages] = {};
       uint32_t issued_phase[kStages] = {};
+      // Weights may stream before the previous kernel (the activation
+      // quantiser) has finished: fill the first stages with W only.
+      const int npre = args.w_prefetch ? min(kStages, ks1 - ks0) : 0;
+      for (int i = 0; i < npre; ++i) {
+        mbar_arrive_expect_tx(&tail->full[i], C::kStageRaw);
+        load_w(i, ks0 + i);
+        issued[i] = true;
+      }
+      grid_dependency_wait();
+      grid_launch_dependents();
       for (int ks = ks0; ks < ks1; ++ks) {
-        if (!mbar_wait_bounded(&tail->empty[stage], phase ^ 1u, abort_flag)) break;
-        uint8_t* st = smem + stage * kStageBytes;
-        mbar_arrive_expect_tx(&tail->full[stage], C::kStageRaw);
-        if constexpr (CH == 1) {
-          const int32_t kx = ks * (BK / 2);
-          tma_load_2d(st, &tm_w, &tail->full[stage], kx, rb * BM);
-          tma_load_2d(st + kWBytes, &tm_x, &tail->full[stage], kx, 0);
-        } else {
-          tma_load_3d(st, &tm_w, &tail->full[stage], 0, rb * BM, ks * CH);
-          tma_load_3d(st + kWBytes, &tm_x, &tail->full[stage], 0, 0, ks * CH);
+        if (ks - ks0 >= npre) {
+          if (!mbar_wait_bounded(&tail->empty[stage], phase ^ 1u, abort_flag)) break;
+          mbar_arrive_expect_tx(&tail->full[stage], C::kStageRaw);
+          load_w(stage, ks);
         }
-        tma_load_3d(st + kWBytes + kXBytes, &tm_sfw, &tail->full[stage], 0, ks * 4 * CH, rb);
-        tma_load_3d(st + kWBytes + kXBytes + kSFWBytes, &tm_sfx, &tail->full[stage], 0, ks * 4 * CH, 0);
+        load_x(stage, ks);
         issued[stage] = true;
         issued_phase[stage] = phase;
         if (++stage == kStages) { stage = 0; phase ^= 1u; }
@@ -207,6 +233,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // ------------------------------------------------------------ epilogue
+    grid_dependency_wait();  // g_a, the segment scales and the outputs
     const int q = warp & 3;
     const int row_local = q * 32 + lane;
     const int64_t n = static_cast<int64_t>(rb) * BM + row_local;
@@ -243,25 +270,31 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int t = 0; t < BN; ++t) acc[t] = 0.0f;
     }
     tc_fence_before();
-    float* partial = reinterpret_cast<float*>(smem);  // [token][row], reuses stage buffers
+    // [row][token] with row stride kPartLd, reusing the stage buffers
+    float* partial = reinterpret_cast<float*>(smem) + row_local * C::kPartLd;
     const uint32_t ready_local = smem_u32(&tail->ready);
     if (rank != 0) {
 #pragma unroll
-      for (int t = 0; t < BN; ++t)
-        if (t < args.M) partial[t * BM + row_local] = acc[t];
+      for (int t = 0; t < BN; t += 4)
+        *reinterpret_cast<float4*>(partial + t) = make_float4(acc[t], acc[t + 1], acc[t + 2], acc[t + 3]);
       mbar_arrive_remote(map_to_rank(ready_local, 0));
       mbar_wait_cluster_bounded(&tail->done, 0);
     } else {
       const bool ok = S == 1 || mbar_wait_cluster_bounded(&tail->ready, 0);
       if (ok) {
         for (int p = 1; p < S; ++p) {
-          const uint32_t peer = map_to_rank(smem_u32(partial), p) + 4u * row_local;
-          // issue every remote load of this peer before the first add
+          const uint32_t peer = map_to_rank(smem_u32(partial), p);
+          // every load of this peer is issued before the first add; groups of
+          // 16 tokens, tokens >= M are zero rows of X and never stored
           float v[BN];
 #pragma unroll
-          for (int t = 0; t < BN; ++t) v[t] = t < args.M ? ld_shared_cluster_f32(peer + 4u * (t * BM)) : 0.0f;
+          for (int t0 = 0; t0 < BN; t0 += 16)
+            if (t0 < args.M) ld_shared_cluster_f32x16(peer + 4u * t0, v + t0);
 #pragma unroll
-          for (int t = 0; t < BN; ++t) acc[t] += v[t];
+          for (int t0 = 0; t0 < BN; t0 += 16)
+            if (t0 < args.M)
+#pragma unroll
+              for (int t = 0; t < 16; ++t) acc[t0 + t] += v[t0 + t];
         }
       }
       if (ok && n < args.N) {
@@ -269,26 +302,34 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int i = 1; i < kMaxSeg; ++i)
           if (i < args.nseg && n >= args.seg[i].n_begin) s = i;
-        const EpiSegment& sg = args.seg[s];
+        // the segment's parameters, loaded once; one tight loop per kind
+        const int kind = args.seg[s].kind;
+        const int64_t ld = args.seg[s].ld_out;
+        const int64_t j = n - args.seg[s].n_begin;
         const float scale = __ldg(args.g_a) * __ldg(args.seg_scale + s);
-        const int64_t j = n - sg.n_begin;
-        float a_log = 0.0f, dt = 0.0f;
-        if (sg.kind == NVFP4_EPI_GDN_DECAY_F32) {
-          a_log = -expf(__ldg(sg.a_log + j));
-          dt = __ldg(sg.dt_bias + j);
-        }
+        const int mt = args.M < BN ? static_cast<int>(args.M) : BN;
+        if (kind == NVFP4_EPI_IDENTITY_BF16) {
+          __nv_bfloat16* o = static_cast<__nv_bfloat16*>(args.seg[s].out) + j;
 #pragma unroll
-        for (int t = 0; t < BN; ++t) {
-          if (t >= args.M) break;
-          const float y = acc[t] * scale;
-          if (sg.kind == NVFP4_EPI_IDENTITY_BF16) {
-            static_cast<__nv_bfloat16*>(sg.out)[t * sg.ld_out + j] = __float2bfloat16_rn(y);
-          } else {
-            float o = y;
-            if (sg.kind == NVFP4_EPI_SIGMOID_F32) o = sigmoid_f(y);
-            else if (sg.kind == NVFP4_EPI_GDN_DECAY_F32) o = a_log * softplus_f(y + dt);
-            static_cast<float*>(sg.out)[t * sg.ld_out + j] = o;
-          }
+          for (int t = 0; t < BN; ++t)
+            if (t < mt) o[t * ld] = __float2bfloat16_rn(acc[t] * scale);
+        } else if (kind == NVFP4_EPI_IDENTITY_F32) {
+          float* o = static_cast<float*>(args.seg[s].out) + j;
+#pragma unroll
+          for (int t = 0; t < BN; ++t)
+            if (t < mt) o[t * ld] = acc[t] * scale;
+        } else if (kind == NVFP4_EPI_SIGMOID_F32) {
+          float* o = static_cast<float*>(args.seg[s].out) + j;
+#pragma unroll
+          for (int t = 0; t < BN; ++t)
+            if (t < mt) o[t * ld] = sigmoid_f(acc[t] * scale);
+        } else {
+          float* o = static_cast<float*>(args.seg[s].out) + j;
+          const float a_log = -expf(__ldg(args.seg[s].a_log + j));
+          const float dt = __ldg(args.seg[s].dt_bias + j);
+#pragma unroll
+          for (int t = 0; t < BN; ++t)
+            if (t < mt) o[t * ld] = a_log * softplus_f(acc[t] * scale + dt);
         }
       }
       // every epilogue thread of the leader has finished reading the peers
@@ -339,6 +380,7 @@ cudaError_t launch_bn(const GemmProblem& p, cudaStream_t stream) {
   a.M = p.M;
   a.N = p.N;
   a.K = p.K;
+  a.w_prefetch = p.w_prefetch ? 1 : 0;
   a.num_k_stages = static_cast<int>(ceil_div(ceil_div(p.K, BK), CH));
   a.g_a = p.g_a;
   a.seg_scale = p.seg_scale;
@@ -364,13 +406,15 @@ cudaError_t launch_bn(const GemmProblem& p, cudaStream_t stream) {
   cfg.blockDim = dim3(kThreads);
   cfg.dynamicSmemBytes = C::kSmemBytes;
   cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = S;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   return cudaLaunchKernelEx(&cfg, decode_kernel<BN, CH>, tm_w, tm_x, tm_sfw, tm_sfx, a);
 }
 }  // namespace dk

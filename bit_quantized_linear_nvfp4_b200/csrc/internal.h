@@ -22,16 +22,20 @@ inline size_t sf_bytes(int64_t rows, int64_t K) {
   return static_cast<size_t>(ceil_div(rows, 128) * 128) * static_cast<size_t>(ceil_div(K, 64) * 4);
 }
 
-// Scratch words a device-computed scale needs: one amax word per segment and
-// one grid-barrier counter.
-size_t quantize_scratch_words(int nseg);
+// Most blocks the amax kernel launches (one per SM, at most this many).
+constexpr int kMaxAmaxBlocks = 256;
+
+// Scratch bytes a device-computed scale needs: one maximum per amax block and
+// segment.  Every call overwrites what it reads, so the scratch needs no
+// clearing.
+size_t quantize_scratch_bytes(int nseg);
 
 // Quantise rows [0, M) (scale layout padded to 128 rows).  Global scale of
 // segment s: g_in[s] if g_in, else amax over the segment's rows / 2688,
-// computed in the same launch with `ws` (quantize_scratch_words(segs.n) words,
-// cleared here) as scratch.  Writes g_out[s].
+// computed by a first launch into `ws` (quantize_scratch_bytes(segs.n)
+// bytes).  Writes g_out[s].
 cudaError_t launch_quantize(const void* x, int dtype, int64_t M, int64_t K, int64_t ld,
-                            const RowSegments& segs, const float* g_in, unsigned int* ws,
+                            const RowSegments& segs, const float* g_in, void* ws,
                             float* g_out, uint8_t* codes, uint8_t* sf, cudaStream_t stream);
 
 // GEMM epilogue description handed to the kernels.
@@ -56,6 +60,10 @@ struct GemmProblem {
   int nseg;
   EpiSegment seg[kMaxSeg];
   bool swiglu;             // two segments: gate [0, N/2), up [N/2, N)
+  // W and its scales are not written by the kernel launched just before the
+  // GEMM on the stream, so the weight-streaming kernel may start reading them
+  // before that kernel completes.
+  bool w_prefetch;
 };
 
 size_t gemm_workspace_bytes(int64_t M, int64_t N, int64_t K);

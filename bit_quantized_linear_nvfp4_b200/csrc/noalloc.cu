@@ -1,11 +1,11 @@
 // nvfp4_quantize_noalloc: the activation quantiser with a device-computed
 // global scale for callers that cannot allocate device memory.
 //
-// The dynamic global scale needs a few bytes of device scratch (the amax
-// reduction word) between its two passes.  nvfp4_quantize takes that scratch
-// from the caller's workspace; this entry point keeps it in a file-scope
-// __device__ array of the library instead, so the caller passes only its
-// inputs and outputs.
+// The dynamic global scale needs a little device scratch (one amax partial
+// per block of the first launch) between its two launches.  nvfp4_quantize
+// takes that scratch from the caller's workspace; this entry point keeps it in
+// a file-scope __device__ array of the library instead, so the caller passes
+// only its inputs and outputs.
 #include <cstdint>
 #include <mutex>
 
@@ -19,23 +19,23 @@ namespace na {
 // Capacity of the static scratch (bytes).  One call needs
 // nvfp4_quantize_workspace_bytes(1) bytes of it.
 constexpr size_t kScratchBytes = NVFP4_NOALLOC_SCRATCH_BYTES;
-static __device__ __align__(256) unsigned int g_scratch[kScratchBytes / sizeof(unsigned int)];
+static __device__ __align__(256) float g_scratch[kScratchBytes / sizeof(float)];
 
 constexpr int kMaxDevices = 64;
 std::mutex g_mutex;
-unsigned int* g_scratch_ptr[kMaxDevices] = {};
+float* g_scratch_ptr[kMaxDevices] = {};
 
 // Device address of g_scratch on the current device.  In host code the name
 // g_scratch is only a host-side stand-in, so the address is looked up once per
 // device (with that device current) and cached.
-cudaError_t scratch_address(int dev, unsigned int** out) {
+cudaError_t scratch_address(int dev, float** out) {
   if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
   std::lock_guard<std::mutex> lock(g_mutex);
   if (g_scratch_ptr[dev] == nullptr) {
     void* p = nullptr;
     cudaError_t e = cudaGetSymbolAddress(&p, g_scratch);
     if (e != cudaSuccess) return e;
-    g_scratch_ptr[dev] = static_cast<unsigned int*>(p);
+    g_scratch_ptr[dev] = static_cast<float*>(p);
   }
   *out = g_scratch_ptr[dev];
   return cudaSuccess;
@@ -54,7 +54,7 @@ extern "C" int nvfp4_quantize_noalloc(const void* x, int x_dtype, int64_t M, int
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return cuda_fail(e);
-  unsigned int* scratch = nullptr;
+  float* scratch = nullptr;
   e = nvfp4::na::scratch_address(dev, &scratch);
   if (e != cudaSuccess) return cuda_fail(e);
   nvfp4::RowSegments segs{};
@@ -62,7 +62,7 @@ extern "C" int nvfp4_quantize_noalloc(const void* x, int x_dtype, int64_t M, int
   segs.begin[0] = 0;
   segs.begin[1] = M;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  // launch_quantize clears the scratch words before accumulating into them
+  // the amax launch overwrites every scratch word the quantise launch reads
   e = nvfp4::launch_quantize(x, x_dtype, M, K, ld_x, segs, nullptr, scratch, g_out, codes, sf, s);
   if (e != cudaSuccess) return cuda_fail(e);
   return NVFP4_OK;

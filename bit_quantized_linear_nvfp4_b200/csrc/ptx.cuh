@@ -51,6 +51,12 @@ __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
       : "memory");
 }
 
+// Raise the expected transaction bytes of the current phase without arriving.
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.expect_tx.relaxed.cta.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+               : "memory");
+}
+
 __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
   asm volatile(
       "{\n\t.reg .b64 st;\n\t"
@@ -92,10 +98,27 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity
   }
 }
 
+// ------------------------------------------- programmatic dependent launch
+// A kernel launched with programmatic stream serialization may start while the
+// kernel before it on the stream is still running.  griddepcontrol.wait blocks
+// the calling thread until that kernel has completed and its memory writes are
+// visible (it returns at once when there is no such dependency);
+// launch_dependents lets the next such kernel start launching.
+__device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void grid_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // ---------------------------------------------------------------- TMA
 
 __device__ __forceinline__ void prefetch_tmap(const CUtensorMap* m) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(m)) : "memory");
+}
+
+// Contiguous global -> shared copy (no tensor map): both addresses 16-byte
+// aligned, bytes a multiple of 16; completes `bytes` on the mbarrier.
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile("cp.async.bulk.shared::cta.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+               ::"r"(smem_u32(dst)), "l"(src), "r"(bytes), "r"(smem_u32(bar))
+               : "memory");
 }
 
 __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* m, uint64_t* bar,
@@ -266,12 +289,26 @@ __device__ __forceinline__ bool mbar_wait_cluster_bounded(uint64_t* bar, uint32_
   }
 }
 
-// Ordered after the preceding acquire by the volatile asm sequence; no memory
-// clobber, so consecutive loads issue back to back.
+// One float of another CTA's shared memory (after a cluster barrier).
 __device__ __forceinline__ float ld_shared_cluster_f32(uint32_t cluster_saddr) {
   float v;
-  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(cluster_saddr));
+  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(cluster_saddr) : "memory");
   return v;
+}
+
+// Sixteen consecutive floats of another CTA's shared memory (16-byte aligned
+// address) as four 128-bit loads in one statement, so that all four are in
+// flight before the first result is used.  Ordered after the preceding
+// acquire by the volatile asm sequence.
+__device__ __forceinline__ void ld_shared_cluster_f32x16(uint32_t cluster_saddr, float* v) {
+  asm volatile(
+      "ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%16];\n\t"
+      "ld.shared::cluster.v4.f32 {%4, %5, %6, %7}, [%16+16];\n\t"
+      "ld.shared::cluster.v4.f32 {%8, %9, %10, %11}, [%16+32];\n\t"
+      "ld.shared::cluster.v4.f32 {%12, %13, %14, %15}, [%16+48];"
+      : "=f"(v[0]), "=f"(v[1]), "=f"(v[2]), "=f"(v[3]), "=f"(v[4]), "=f"(v[5]), "=f"(v[6]), "=f"(v[7]),
+        "=f"(v[8]), "=f"(v[9]), "=f"(v[10]), "=f"(v[11]), "=f"(v[12]), "=f"(v[13]), "=f"(v[14]), "=f"(v[15])
+      : "r"(cluster_saddr));
 }
 
 __device__ __forceinline__ void named_barrier_sync(uint32_t id, uint32_t threads) {

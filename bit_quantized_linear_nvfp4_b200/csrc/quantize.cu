@@ -8,17 +8,30 @@
 //   inv = S*g > 0 ? 1/(S*g) : 0, at most FLT_MAX;  code = E2M1_rn_satfinite(x*inv)
 // with g = amax|x| / (6 * 448) per tensor (or per row range) when not given.
 //
-// HBM-bound design.  A warp takes a chunk of 512 consecutive elements of one
-// row; lane l owns the 16-block l of the chunk (one 256-bit load for BF16),
-// so the block amax, scale and codes need no cross-lane traffic.  Each lane
-// stores its 16 codes as 8 contiguous bytes (a warp writes 256 bytes), and
-// four lanes' scale bytes are gathered by shuffles into one 32-bit word
-// stored at its place in the tcgen05 block-scale layout; layout padding
-// (rows up to 128, K/16 up to 4) is written with zeros.
+// HBM-bound design.  The work item is a chunk of 512 consecutive elements of
+// one row; lane l of a warp owns 16-element block l of a chunk (one 256-bit
+// load for BF16), so the block amax, scale and codes need no cross-lane
+// traffic.  Each lane stores its 16 codes as 8 contiguous bytes (a warp writes
+// 256 bytes), and four lanes' scale bytes are gathered by shuffles into one
+// 32-bit word of the tcgen05 block-scale layout; layout padding (rows up to
+// 128, K/16 up to a multiple of 4) is written with zeros.
 //
-// With a device-computed scale the kernel runs two passes in one cooperative
-// launch: amax over the rows, a grid barrier (bounded wait), then the
-// quantisation pass, which re-reads x from L2 when x fits there.
+// Large inputs: one block per SM owns a contiguous, balanced range of chunks;
+// its 32 warps read it with 256-bit loads straight into registers (several
+// chunks in flight per warp; at each step the block's warps cover 32
+// consecutive chunks).  A device-computed scale takes two launches: the amax
+// kernel stores one maximum per block and segment (plain stores, so no
+// scratch clearing) and the quantise kernel reduces them first.  Both are
+// launched with programmatic stream serialization and wait
+// (griddepcontrol.wait) before they touch global memory, so launch and
+// prologue overlap the kernel before.  The quantise kernel walks its range
+// backwards, so that when x is larger than L2 it starts on the chunks the
+// amax kernel read last.
+//
+// Small inputs with a device-computed scale (up to 8 blocks' worth): one
+// launch of a thread-block cluster; each block copies its share of x into
+// shared memory once, the blocks exchange their maxima through distributed
+// shared memory, and quantise from shared memory.
 #include <cfloat>
 #include <cstdint>
 
@@ -31,30 +44,39 @@
 namespace nvfp4 {
 namespace qk {
 
-constexpr int kChunk = 512;  // elements per warp per chunk (32 lanes x 16)
-// Large blocks keep the number of blocks (and so of same-address atomics in
-// the amax reduction and the grid barrier) near the SM count; FP32 input
-// needs more registers per lane and uses smaller blocks.
+constexpr int kChunk = 512;  // elements per chunk (32 lanes x 16)
+constexpr int kWarps = 32;   // warps per block
+constexpr int kThreads = kWarps * 32;
+constexpr int kUnrollQ = 2;  // chunks in flight per warp, quantise kernel
+
 template <int DTYPE>
 struct Cfg {
-  static constexpr int kThreads = DTYPE == NVFP4_DTYPE_BF16 ? 1024 : 256;
-  static constexpr int kWarps = kThreads / 32;
+  static constexpr int kEsz = DTYPE == NVFP4_DTYPE_BF16 ? 2 : 4;
+  static constexpr int kChunkBytes = kChunk * kEsz;
+  static constexpr int kWords = DTYPE == NVFP4_DTYPE_BF16 ? 8 : 16;  // per lane
+  static constexpr int kUnrollA = DTYPE == NVFP4_DTYPE_BF16 ? 4 : 2;  // chunks in flight per warp, amax
 };
-constexpr int kUnrollQ = 2;  // chunks per warp iteration, quantisation pass
-constexpr int kUnrollA = 4;  // chunks per warp iteration, amax pass
 
 struct QuantArgs {
   const uint8_t* x;
   int64_t ld_bytes;
   int32_t M, K, rows_pad, cpr;  // cpr: chunks per row
-  int32_t items_q, items_a;     // rows_pad * cpr, M * cpr
+  int64_t items;                // M * cpr (< 2^30)
+  uint64_t cpr_inv;             // ceil(2^64 / cpr) (0 when cpr == 1): row = mulhi(item, cpr_inv)
   int nseg;
   int32_t seg_begin[kMaxSeg + 1];
-  const float* g_in;
-  unsigned int* ws;  // [nseg] amax bits, [nseg] grid-barrier counter (dynamic only)
+  const float* g_in;    // given scales, or nullptr
+  float* partial;       // [amax_blocks][nseg] per-block maxima (device-computed scale)
+  int amax_blocks;
   float* g_out;
   uint8_t* codes;
   uint8_t* sf;
+};
+
+// The raw 16 elements of one lane: 8 words (BF16) or 16 words (F32).
+template <int DTYPE>
+struct Blk {
+  uint32_t w[Cfg<DTYPE>::kWords];
 };
 
 __device__ __forceinline__ void ld_v8(const void* p, uint32_t* r) {
@@ -64,40 +86,65 @@ __device__ __forceinline__ void ld_v8(const void* p, uint32_t* r) {
                : "l"(p));
 }
 __device__ __forceinline__ void ld_v4(const void* p, uint32_t* r) {
-  asm volatile("ld.global.nc.v4.u32 {%0, %1, %2, %3}, [%4];"
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
                : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
                : "l"(p));
 }
 
-// Raw 16-element block of one lane: 8 words (BF16) or 16 words (F32).
-template <int DTYPE>
-struct Block {
-  static constexpr int kWords = DTYPE == NVFP4_DTYPE_BF16 ? 8 : 16;
-  uint32_t w[kWords];
-};
-
+// From global memory; WIDE: 32-byte aligned, so 256-bit loads.
 template <int DTYPE, bool WIDE>
-__device__ __forceinline__ void load_block(const uint8_t* p, Block<DTYPE>& b) {
-  if constexpr (DTYPE == NVFP4_DTYPE_BF16) {
-    if constexpr (WIDE) {
-      ld_v8(p, b.w);
-    } else {
-      ld_v4(p, b.w);
-      ld_v4(p + 16, b.w + 4);
-    }
-  } else {
-    if constexpr (WIDE) {
-      ld_v8(p, b.w);
-      ld_v8(p + 32, b.w + 8);
-    } else {
+__device__ __forceinline__ void load_global(const uint8_t* p, Blk<DTYPE>& b) {
+  constexpr int kW = Cfg<DTYPE>::kWords;
 #pragma unroll
-      for (int i = 0; i < 4; ++i) ld_v4(p + 16 * i, b.w + 4 * i);
+  for (int i = 0; i < kW; i += 8) {
+    if constexpr (WIDE) {
+      ld_v8(p + 4 * i, b.w + i);
+    } else {
+      ld_v4(p + 4 * i, b.w + i);
+      ld_v4(p + 4 * i + 16, b.w + i + 4);
     }
   }
 }
 
+// From shared memory (16-byte aligned).
 template <int DTYPE>
-__device__ __forceinline__ void unpack(const Block<DTYPE>& b, float (&v)[16]) {
+__device__ __forceinline__ void load_shared(const uint8_t* p, Blk<DTYPE>& b) {
+  constexpr int kW = Cfg<DTYPE>::kWords;
+#pragma unroll
+  for (int i = 0; i < kW; i += 4) {
+    const uint4 v = *reinterpret_cast<const uint4*>(p + 4 * i);
+    b.w[i] = v.x;
+    b.w[i + 1] = v.y;
+    b.w[i + 2] = v.z;
+    b.w[i + 3] = v.w;
+  }
+}
+
+// max |x| of the block.  BF16: the magnitudes' bit patterns order like their
+// values (finite inputs), so a packed 16-bit integer max gives the exact
+// maximum.
+template <int DTYPE>
+__device__ __forceinline__ float block_amax(const Blk<DTYPE>& b) {
+  if constexpr (DTYPE == NVFP4_DTYPE_BF16) {
+    uint32_t m = 0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      uint32_t r;
+      asm("max.u16x2 %0, %1, %2;" : "=r"(r) : "r"(m), "r"(b.w[i] & 0x7FFF7FFFu));
+      m = r;
+    }
+    const uint32_t hi = m >> 16, lo = m & 0xFFFFu;
+    return __uint_as_float((hi > lo ? hi : lo) << 16);
+  } else {
+    float m = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) m = fmaxf(m, fabsf(__uint_as_float(b.w[i])));
+    return m;
+  }
+}
+
+template <int DTYPE>
+__device__ __forceinline__ void to_float(const Blk<DTYPE>& b, float (&v)[16]) {
   if constexpr (DTYPE == NVFP4_DTYPE_BF16) {
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
@@ -108,6 +155,16 @@ __device__ __forceinline__ void unpack(const Block<DTYPE>& b, float (&v)[16]) {
 #pragma unroll
     for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(b.w[i]);
   }
+}
+
+// Packed FP32 multiply of a pair by s (sm_100 f32x2; each lane rounds to
+// nearest even exactly as a scalar multiply does).
+__device__ __forceinline__ void mul_f32x2(float& a0, float& a1, float s) {
+  uint64_t x, y, k;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(x) : "f"(a0), "f"(a1));
+  asm("mov.b64 %0, {%1, %1};" : "=l"(k) : "f"(s));
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(y) : "l"(x), "l"(k));
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(a0), "=f"(a1) : "l"(y));
 }
 
 // E4M3 (satfinite, round to nearest even) of a non-negative float: low byte.
@@ -138,6 +195,16 @@ __device__ __forceinline__ uint32_t to_e2m1x8(const float* q) {
   return out;
 }
 
+// Row and first column of chunk `item` without a division: for 32-bit n and
+// d, floor(n / d) is the high word of n * ceil(2^64 / d) (Lemire, Kaser and
+// Kurz, "Faster remainder by direct computation", 2019).
+__device__ __forceinline__ void chunk_pos(const QuantArgs& a, int64_t item, int32_t& row, int32_t& col0) {
+  const uint64_t n = static_cast<uint64_t>(item);
+  const uint32_t r = a.cpr == 1 ? static_cast<uint32_t>(n) : static_cast<uint32_t>(__umul64hi(a.cpr_inv, n));
+  row = static_cast<int32_t>(r);
+  col0 = (static_cast<int32_t>(n) - static_cast<int32_t>(r) * a.cpr) * kChunk;
+}
+
 __device__ __forceinline__ int find_segment(const QuantArgs& a, int32_t row) {
   int s = 0;
 #pragma unroll
@@ -146,173 +213,324 @@ __device__ __forceinline__ int find_segment(const QuantArgs& a, int32_t row) {
   return s;
 }
 
-__device__ __forceinline__ unsigned int ld_acquire_u32(const unsigned int* p) {
-  unsigned int v;
-  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-  return v;
+__device__ __forceinline__ void block_range(int64_t items, int64_t& lo, int64_t& hi) {
+  lo = items * blockIdx.x / gridDim.x;
+  hi = items * (blockIdx.x + 1) / gridDim.x;
 }
 
-// Pass 1: per-segment amax of rows [0, M), one atomicMax per block and segment.
-template <int DTYPE, bool WIDE>
-__device__ __forceinline__ void amax_pass(const QuantArgs& a) {
-  constexpr int kWarps = Cfg<DTYPE>::kWarps;
-  const int lane = threadIdx.x & 31;
-  const int warp = threadIdx.x >> 5;
-  const int32_t gwarp = blockIdx.x * kWarps + warp;
-  const int32_t nwarps = gridDim.x * kWarps;
-  constexpr int kEsz = DTYPE == NVFP4_DTYPE_BF16 ? 2 : 4;
-  float lm[kMaxSeg];
+// Running per-segment maxima of one lane, kept in registers.
+struct SegMax {
+  float m[kMaxSeg];
+  __device__ __forceinline__ SegMax() {
 #pragma unroll
-  for (int s = 0; s < kMaxSeg; ++s) lm[s] = 0.0f;
-  for (int32_t base = gwarp * kUnrollA; base < a.items_a; base += nwarps * kUnrollA) {
-    Block<DTYPE> blk[kUnrollA];
+    for (int s = 0; s < kMaxSeg; ++s) m[s] = 0.0f;
+  }
+  __device__ __forceinline__ void add(int seg, float v) {
+#pragma unroll
+    for (int s = 0; s < kMaxSeg; ++s)
+      if (s == seg) m[s] = fmaxf(m[s], v);
+  }
+  // Block-wide maxima of segments [0, nseg): warp s returns segment s's
+  // maximum in every lane (red: kWarps x kMaxSeg shared floats).
+  __device__ __forceinline__ float reduce(int nseg, float (*red)[kMaxSeg]) const {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+#pragma unroll
+    for (int s = 0; s < kMaxSeg; ++s) {
+      if (s >= nseg) break;  // uniform
+      float v = m[s];
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, off));
+      if (lane == 0) red[warp][s] = v;
+    }
+    __syncthreads();
+    float v = 0.0f;
+    if (warp < nseg) {
+      v = red[lane][warp];
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, off));
+    }
+    return v;
+  }
+};
+
+// Codes and scale bytes of one lane's block of chunk `item` (all 32 lanes of
+// a warp call it for the same chunk; `have` is false past K).
+template <int DTYPE>
+__device__ __forceinline__ void quantize_block(const QuantArgs& a, const float* g_sh, const Blk<DTYPE>& b,
+                                               bool have, int32_t row, int32_t col) {
+  const int lane = threadIdx.x & 31;
+  const int32_t KA = (a.K + 63) / 64;
+  const float g = g_sh[find_segment(a, row)];
+  uint32_t sfb = 0;
+  uint2 word = make_uint2(0u, 0u);
+  if (have && g > 0.0f) {
+    const float m = block_amax<DTYPE>(b);
+    const float s = (m / 6.0f) / g;
+    sfb = to_e4m3(s);
+    const float denom = e4m3_value(sfb) * g;
+    float inv = denom > 0.0f ? 1.0f / denom : 0.0f;
+    inv = fminf(inv, FLT_MAX);
+    float q[16];
+    to_float<DTYPE>(b, q);
+#pragma unroll
+    for (int i = 0; i < 16; i += 2) mul_f32x2(q[i], q[i + 1], inv);
+    word.x = to_e2m1x8(q);
+    word.y = to_e2m1x8(q + 8);
+  }
+  if (have) *reinterpret_cast<uint2*>(a.codes + static_cast<int64_t>(row) * (a.K / 2) + col / 2) = word;
+  // four lanes' scale bytes -> one 32-bit word of the block-scale layout
+  const uint32_t s1 = __shfl_down_sync(0xffffffffu, sfb, 1);
+  const uint32_t s2 = __shfl_down_sync(0xffffffffu, sfb, 2);
+  const uint32_t s3 = __shfl_down_sync(0xffffffffu, sfb, 3);
+  const int32_t kb = col / 64;
+  if ((lane & 3) == 0 && kb < KA) {
+    const int64_t off = (static_cast<int64_t>(row >> 7) * KA + kb) * 512 + (row & 31) * 16 + ((row >> 5) & 3) * 4;
+    *reinterpret_cast<uint32_t*>(a.sf + off) = sfb | (s1 << 8) | (s2 << 16) | (s3 << 24);
+  }
+}
+
+// Zero scale words of the layout's padding rows [M, rows_pad).  They all lie
+// in the last 128-row block; word w (4 bytes) of a 512-byte atom holds row
+// (w / 4) + 32 * (w % 4) of the block, so a warp walks an atom's 128 words in
+// order (coalesced 128-byte stores) and writes those of padding rows.  Warps
+// of the whole grid take atoms.
+__device__ __forceinline__ void zero_padding_rows(const QuantArgs& a) {
+  if (a.rows_pad == a.M) return;
+  const int32_t KA = (a.K + 63) / 64;
+  const int32_t rb = a.M >> 7;
+  const int lane = threadIdx.x & 31;
+  const int32_t gw = blockIdx.x * kWarps + (threadIdx.x >> 5), nw = gridDim.x * kWarps;
+  for (int32_t kb = gw; kb < KA; kb += nw) {
+    uint32_t* atom = reinterpret_cast<uint32_t*>(a.sf + (static_cast<int64_t>(rb) * KA + kb) * 512);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int w = lane + 32 * i;
+      if (rb * 128 + (w >> 2) + 32 * (w & 3) >= a.M) atom[w] = 0u;
+    }
+  }
+}
+
+// Pass 1 (device-computed scale): per-segment amax of the block's chunks,
+// stored to partial[block][segment].
+template <int DTYPE, bool WIDE>
+__global__ void __launch_bounds__(kThreads, 1) amax_kernel(const __grid_constant__ QuantArgs a) {
+  using C = Cfg<DTYPE>;
+  __shared__ float red[kWarps][kMaxSeg];
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  grid_dependency_wait();  // x may come from the kernel before this one
+  if (threadIdx.x == 0) grid_launch_dependents();
+  int64_t lo, hi;
+  block_range(a.items, lo, hi);
+  SegMax sm;
+  constexpr int kUnrollA = C::kUnrollA;
+  for (int64_t base = lo; base < hi; base += kWarps * kUnrollA) {
+    Blk<DTYPE> b[kUnrollA];
     int32_t rows[kUnrollA];
     bool act[kUnrollA];
 #pragma unroll
     for (int u = 0; u < kUnrollA; ++u) {
-      const int32_t item = base + u;
-      const int32_t row = item / a.cpr;
-      const int32_t col = (item - row * a.cpr) * kChunk + lane * 16;
-      rows[u] = row;
-      act[u] = item < a.items_a && col < a.K;
-      if (act[u]) load_block<DTYPE, WIDE>(a.x + row * a.ld_bytes + static_cast<int64_t>(col) * kEsz, blk[u]);
+      const int64_t item = base + u * kWarps + warp;
+      act[u] = false;
+      rows[u] = 0;
+      if (item < hi) {
+        int32_t col;
+        chunk_pos(a, item, rows[u], col);
+        col += lane * 16;
+        act[u] = col < a.K;
+        if (act[u]) load_global<DTYPE, WIDE>(a.x + rows[u] * a.ld_bytes + static_cast<int64_t>(col) * C::kEsz, b[u]);
+      }
     }
 #pragma unroll
-    for (int u = 0; u < kUnrollA; ++u) {
-      if (!act[u]) continue;
-      float v[16];
-      unpack<DTYPE>(blk[u], v);
-      float m = 0.0f;
-#pragma unroll
-      for (int i = 0; i < 16; ++i) m = fmaxf(m, fabsf(v[i]));
-      const int s = find_segment(a, rows[u]);
-#pragma unroll
-      for (int i = 0; i < kMaxSeg; ++i)
-        if (i == s) lm[i] = fmaxf(lm[i], m);
-    }
+    for (int u = 0; u < kUnrollA; ++u)
+      if (act[u]) sm.add(find_segment(a, rows[u]), block_amax<DTYPE>(b[u]));
   }
-  __shared__ float red[kWarps][kMaxSeg];
-#pragma unroll
-  for (int s = 0; s < kMaxSeg; ++s) {
-    float m = lm[s];
+  const float m = sm.reduce(a.nseg, red);
+  if (warp < a.nseg && lane == 0) a.partial[blockIdx.x * a.nseg + warp] = m;
+}
+
+// Pass 2: global scale per segment (given, or the maximum of the amax
+// kernel's partials / 2688), then the codes and scale bytes of rows [0, M)
+// and zero scale words for the layout's padding rows [M, rows_pad).
+template <int DTYPE, bool WIDE>
+__global__ void __launch_bounds__(kThreads, 1) quant_kernel(const __grid_constant__ QuantArgs a) {
+  using C = Cfg<DTYPE>;
+  __shared__ float g_sh[kMaxSeg];
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  // Once every block of this grid has passed this point all of them are
+  // resident, so a dependent kernel may start launching (it waits for this
+  // grid's completion before touching what it writes).
+  if (threadIdx.x == 0) grid_launch_dependents();
+  grid_dependency_wait();
+  if (a.g_in != nullptr) {
+    if (threadIdx.x < a.nseg) g_sh[threadIdx.x] = a.g_in[threadIdx.x];
+  } else if (warp < a.nseg) {
+    float m = 0.0f;
+    for (int b = lane; b < a.amax_blocks; b += 32) m = fmaxf(m, a.partial[b * a.nseg + warp]);
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
-    if (lane == 0) red[warp][s] = m;
+    if (lane == 0) g_sh[warp] = m / 2688.0f;
   }
   __syncthreads();
-  if (threadIdx.x < a.nseg) {
-    float m = 0.0f;
-#pragma unroll
-    for (int w = 0; w < kWarps; ++w) m = fmaxf(m, red[w][threadIdx.x]);
-    if (m > 0.0f) atomicMax(a.ws + threadIdx.x, __float_as_uint(m));  // non-negative floats order as integers
-  }
-}
+  if (blockIdx.x == 0 && threadIdx.x < a.nseg) a.g_out[threadIdx.x] = g_sh[threadIdx.x];
 
-// Pass 2: quantise rows [0, rows_pad) (rows >= M only zero their scale words).
-template <int DTYPE, bool WIDE>
-__device__ __forceinline__ void quant_pass(const QuantArgs& a, const float* g_sh) {
-  constexpr int kWarps = Cfg<DTYPE>::kWarps;
-  const int lane = threadIdx.x & 31;
-  const int32_t gwarp = blockIdx.x * kWarps + (threadIdx.x >> 5);
-  const int32_t nwarps = gridDim.x * kWarps;
-  constexpr int kEsz = DTYPE == NVFP4_DTYPE_BF16 ? 2 : 4;
-  const int32_t KA = (a.K + 63) / 64;
-  const int64_t code_ld = a.K / 2;
-  for (int32_t base = gwarp * kUnrollQ; base < a.items_q; base += nwarps * kUnrollQ) {
-    Block<DTYPE> blk[kUnrollQ];
+  int64_t lo, hi;
+  block_range(a.items, lo, hi);
+  // backwards over the range, kWarps * kUnrollQ chunks per step
+  for (int64_t end = hi; end > lo; end -= kWarps * kUnrollQ) {
+    const int64_t base = end - kWarps * kUnrollQ > lo ? end - kWarps * kUnrollQ : lo;
+    Blk<DTYPE> b[kUnrollQ];
     int32_t rows[kUnrollQ], cols[kUnrollQ];
-    bool act[kUnrollQ];
-    float gs[kUnrollQ];
+    bool inr[kUnrollQ], act[kUnrollQ];
 #pragma unroll
     for (int u = 0; u < kUnrollQ; ++u) {
-      const int32_t item = base + u;
-      const int32_t row = item / a.cpr;
-      const int32_t col = (item - row * a.cpr) * kChunk + lane * 16;
-      rows[u] = row;
-      cols[u] = col;
-      gs[u] = row < a.M ? g_sh[find_segment(a, row)] : 0.0f;
-      act[u] = item < a.items_q && row < a.M && col < a.K && gs[u] > 0.0f;
-      if (act[u]) load_block<DTYPE, WIDE>(a.x + row * a.ld_bytes + static_cast<int64_t>(col) * kEsz, blk[u]);
-    }
-#pragma unroll
-    for (int u = 0; u < kUnrollQ; ++u) {
-      const int32_t item = base + u;
-      if (item >= a.items_q) break;  // uniform across the warp
-      const int32_t row = rows[u], col = cols[u];
-      uint32_t sfb = 0;
-      uint2 word = make_uint2(0u, 0u);
-      if (act[u]) {
-        const float g = gs[u];
-        float v[16];
-        unpack<DTYPE>(blk[u], v);
-        float m = 0.0f;
-#pragma unroll
-        for (int i = 0; i < 16; ++i) m = fmaxf(m, fabsf(v[i]));
-        const float s = (m / 6.0f) / g;
-        sfb = to_e4m3(s);
-        const float denom = e4m3_value(sfb) * g;
-        float inv = denom > 0.0f ? 1.0f / denom : 0.0f;
-        inv = fminf(inv, FLT_MAX);
-        float q[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i) q[i] = v[i] * inv;
-        word.x = to_e2m1x8(q);
-        word.y = to_e2m1x8(q + 8);
-      }
-      if (row < a.M && col < a.K)
-        *reinterpret_cast<uint2*>(a.codes + row * code_ld + col / 2) = word;
-      // four lanes' scale bytes -> one 32-bit word of the block-scale layout
-      const uint32_t s1 = __shfl_down_sync(0xffffffffu, sfb, 1);
-      const uint32_t s2 = __shfl_down_sync(0xffffffffu, sfb, 2);
-      const uint32_t s3 = __shfl_down_sync(0xffffffffu, sfb, 3);
-      const int32_t kb = col / 64;
-      if ((lane & 3) == 0 && kb < KA) {
-        const int64_t off = (static_cast<int64_t>(row >> 7) * KA + kb) * 512 + (row & 31) * 16 + ((row >> 5) & 3) * 4;
-        *reinterpret_cast<uint32_t*>(a.sf + off) = sfb | (s1 << 8) | (s2 << 16) | (s3 << 24);
+      const int64_t item = base + u * kWarps + warp;
+      inr[u] = item < end;
+      act[u] = false;
+      rows[u] = cols[u] = 0;
+      if (inr[u]) {
+        chunk_pos(a, item, rows[u], cols[u]);
+        cols[u] += lane * 16;
+        act[u] = cols[u] < a.K;
+        if (act[u]) load_global<DTYPE, WIDE>(a.x + rows[u] * a.ld_bytes + static_cast<int64_t>(cols[u]) * C::kEsz, b[u]);
       }
     }
+#pragma unroll
+    for (int u = 0; u < kUnrollQ; ++u)
+      if (inr[u]) quantize_block<DTYPE>(a, g_sh, b[u], act[u], rows[u], cols[u]);  // uniform across the warp
   }
+  zero_padding_rows(a);
 }
 
-template <int DTYPE, bool WIDE, bool DYNAMIC>
-__global__ void __launch_bounds__(Cfg<DTYPE>::kThreads) quantize_kernel(const __grid_constant__ QuantArgs a) {
+// Copies of up to 32 consecutive chunks [i0, i1) (lane j: chunk i0 + j) into
+// dst + j * kChunkBytes.  Chunks that follow one another both in x and in dst
+// (full chunks of one row, or of consecutive rows when rows are packed) are
+// merged into one copy, because a bulk copy costs about the same whatever its
+// size up to several KB.  plan() is warp-collective; issue() then starts the
+// copies on `bar`, after the caller has raised the barrier's expected bytes by
+// `total`.
+template <int DTYPE>
+struct ChunkCopies {
+  using C = Cfg<DTYPE>;
+  const uint8_t* src = nullptr;
+  uint32_t run = 0;    // bytes of the copy this lane starts (0: none)
+  uint32_t total = 0;  // bytes of all the chunks
+
+  __device__ __forceinline__ void plan(const QuantArgs& a, int64_t i0, int64_t i1) {
+    const int lane = threadIdx.x & 31;
+    const int64_t item = i0 + lane;
+    uint32_t bytes = 0;
+    if (item < i1) {
+      int32_t row, col;
+      chunk_pos(a, item, row, col);
+      const int32_t n = a.K - col < kChunk ? a.K - col : kChunk;
+      bytes = static_cast<uint32_t>(n) * C::kEsz;
+      src = a.x + row * a.ld_bytes + static_cast<int64_t>(col) * C::kEsz;
+    }
+    // a copy starts at every chunk that does not continue the previous one
+    const uint32_t prev_bytes = __shfl_up_sync(0xffffffffu, bytes, 1);
+    const uint64_t prev_src = __shfl_up_sync(0xffffffffu, reinterpret_cast<uint64_t>(src), 1);
+    const bool continues = lane > 0 && prev_bytes == static_cast<uint32_t>(C::kChunkBytes) &&
+                           reinterpret_cast<uint64_t>(src) == prev_src + C::kChunkBytes;
+    const uint32_t starts = __ballot_sync(0xffffffffu, bytes != 0 && !continues);
+    // exclusive prefix sum of the chunk sizes
+    uint32_t incl = bytes;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const uint32_t v = __shfl_up_sync(0xffffffffu, incl, off);
+      if (lane >= off) incl += v;
+    }
+    total = __shfl_sync(0xffffffffu, incl, 31);
+    const uint32_t excl = incl - bytes;
+    const uint32_t later = lane < 31 ? starts & (0xfffffffeu << lane) : 0u;
+    const int next = later ? __ffs(later) - 1 : 32;
+    const uint32_t end = __shfl_sync(0xffffffffu, excl, next & 31);
+    run = ((starts >> lane) & 1u) ? (next < 32 ? end : total) - excl : 0u;
+  }
+
+  __device__ __forceinline__ void issue(uint8_t* dst, uint64_t* bar) const {
+    if (run != 0) bulk_load(dst + (threadIdx.x & 31) * C::kChunkBytes, src, run, bar);
+  }
+};
+
+// Small inputs with a device-computed scale, in one launch: a cluster of C
+// blocks (C <= 8) each copies its whole share of x into shared memory, takes
+// the block amax, reads the other blocks' maxima through distributed shared
+// memory, and quantises from shared memory; x is read once.
+constexpr int kSmallSmem = 200 * 1024;
+constexpr int kMaxSmallBlocks = 8;
+
+template <int DTYPE>
+__global__ void __launch_bounds__(kThreads, 1) small_kernel(const __grid_constant__ QuantArgs a) {
+  using C = Cfg<DTYPE>;
+  extern __shared__ __align__(1024) uint8_t buf[];
+  __shared__ uint64_t full;
+  __shared__ float red[kWarps][kMaxSeg];
+  __shared__ float blk_amax[kMaxSeg];
   __shared__ float g_sh[kMaxSeg];
-  __shared__ int abort_sh;
-  if constexpr (DYNAMIC) {
-    amax_pass<DTYPE, WIDE>(a);
-    // grid barrier: every block's amax is published before any block reads it
-    __syncthreads();
-    if (threadIdx.x == 0) {
-      abort_sh = 0;
-      unsigned int* counter = a.ws + a.nseg;
-      __threadfence();
-      atomicAdd(counter, 1u);
-      const uint64_t t0 = global_timer_ns();
-      while (ld_acquire_u32(counter) < gridDim.x) {
-        if (global_timer_ns() - t0 > 2000000000ull) {
-          atomicOr(&g_device_error, kErrTimeout);
-          abort_sh = 1;
-          break;
-        }
-        __nanosleep(64);
-      }
-    }
-    __syncthreads();
-    if (abort_sh) return;
-    if (threadIdx.x < a.nseg) {
-      const float g = __uint_as_float(ld_acquire_u32(a.ws + threadIdx.x)) / 2688.0f;
-      g_sh[threadIdx.x] = g;
-      if (blockIdx.x == 0) a.g_out[threadIdx.x] = g;
-    }
-  } else {
-    if (threadIdx.x < a.nseg) {
-      const float g = a.g_in[threadIdx.x];
-      g_sh[threadIdx.x] = g;
-      if (blockIdx.x == 0) a.g_out[threadIdx.x] = g;
-    }
+  __shared__ int abort_flag;
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    mbar_init(&full, 1);
+    abort_flag = 0;
+    fence_mbarrier_init();
   }
   __syncthreads();
-  quant_pass<DTYPE, WIDE>(a, g_sh);
+  if (threadIdx.x == 0) grid_launch_dependents();
+  grid_dependency_wait();
+  int64_t lo, hi;
+  block_range(a.items, lo, hi);
+  if (warp == 0) {
+    for (int64_t i0 = lo; i0 < hi; i0 += 32) {
+      ChunkCopies<DTYPE> cc;
+      cc.plan(a, i0, hi < i0 + 32 ? hi : i0 + 32);
+      if (lane == 0) mbar_expect_tx(&full, cc.total);
+      __syncwarp();
+      cc.issue(buf + (i0 - lo) * C::kChunkBytes, &full);
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&full);
+  }
+  const bool ok = mbar_wait_bounded(&full, 0, &abort_flag);
+
+  SegMax sm;
+  if (ok)
+    for (int64_t i = lo + warp; i < hi; i += kWarps) {
+      int32_t row, col;
+      chunk_pos(a, i, row, col);
+      if (col + lane * 16 < a.K) {
+        Blk<DTYPE> b;
+        load_shared<DTYPE>(buf + (i - lo) * C::kChunkBytes + lane * 16 * C::kEsz, b);
+        sm.add(find_segment(a, row), block_amax<DTYPE>(b));
+      }
+    }
+  const float m = sm.reduce(a.nseg, red);
+  if (warp < a.nseg && lane == 0) blk_amax[warp] = m;
+  cluster_sync_all();  // every block's maxima are visible to the cluster
+  if (threadIdx.x < a.nseg) {
+    float v = 0.0f;
+    for (uint32_t rk = 0; rk < gridDim.x; ++rk)
+      v = fmaxf(v, ld_shared_cluster_f32(map_to_rank(smem_u32(&blk_amax[threadIdx.x]), rk)));
+    g_sh[threadIdx.x] = v / 2688.0f;
+  }
+  __syncthreads();
+  if (blockIdx.x == 0 && threadIdx.x < a.nseg) a.g_out[threadIdx.x] = g_sh[threadIdx.x];
+  if (ok)
+    for (int64_t i = lo + warp; i < hi; i += kWarps) {
+      int32_t row, col;
+      chunk_pos(a, i, row, col);
+      col += lane * 16;
+      Blk<DTYPE> b;
+      const bool have = col < a.K;
+      if (have) load_shared<DTYPE>(buf + (i - lo) * C::kChunkBytes + lane * 16 * C::kEsz, b);
+      quantize_block<DTYPE>(a, g_sh, b, have, row, col);
+    }
+  zero_padding_rows(a);
+  if (!ok && threadIdx.x == 0)  // let copies still in flight land (bounded)
+    mbar_wait_bounded(&full, 0, nullptr, 200000000ull);
+  cluster_sync_all();  // no block leaves while another may read its maxima
 }
 
 int num_sms() {
@@ -322,38 +540,64 @@ int num_sms() {
   return sms;
 }
 
-template <int DTYPE, bool WIDE, bool DYNAMIC>
-cudaError_t launch_t(const QuantArgs& a, cudaStream_t stream) {
-  constexpr int kThreads = Cfg<DTYPE>::kThreads;
-  constexpr int kWarps = Cfg<DTYPE>::kWarps;
-  auto kern = quantize_kernel<DTYPE, WIDE, DYNAMIC>;
-  int per_sm = 0;
-  cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kThreads, 0);
-  if (e != cudaSuccess) return e;
-  if (per_sm < 1) per_sm = 1;
-  const int64_t cap = static_cast<int64_t>(num_sms()) * per_sm;
-  const int64_t want = (static_cast<int64_t>(a.items_q) + kWarps * kUnrollQ - 1) / (kWarps * kUnrollQ);
-  int grid = static_cast<int>(want < cap ? want : cap);
-  if (grid < 1) grid = 1;
+// One block per SM (at most kMaxAmaxBlocks), at least 32 chunks per block.
+int grid_for(int64_t items) {
+  int64_t g = (items + kWarps - 1) / kWarps;
+  const int sms = num_sms();
+  const int64_t cap = sms < kMaxAmaxBlocks ? sms : kMaxAmaxBlocks;
+  if (g > cap) g = cap;
+  return g < 1 ? 1 : static_cast<int>(g);
+}
+
+template <class Kern>
+cudaError_t launch_pdl(Kern kern, int grid, int cluster, int smem, const QuantArgs& a, cudaStream_t stream) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
   cfg.blockDim = dim3(kThreads);
-  cfg.dynamicSmemBytes = 0;
+  cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeCooperative;
-  attr[0].val.cooperative = DYNAMIC ? 1 : 0;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = cluster;
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = cluster > 1 ? 2 : 1;
   return cudaLaunchKernelEx(&cfg, kern, a);
+}
+
+template <int DTYPE, bool WIDE>
+cudaError_t launch_t(QuantArgs a, bool dynamic, cudaStream_t stream) {
+  using C = Cfg<DTYPE>;
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(small_kernel<DTYPE>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmallSmem);
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  constexpr int64_t kSmallChunks = kSmallSmem / C::kChunkBytes;  // per block
+  const int64_t nsmall = (a.items + kSmallChunks - 1) / kSmallChunks;
+  if (dynamic && nsmall <= kMaxSmallBlocks) {
+    const int blocks = nsmall < 1 ? 1 : static_cast<int>(nsmall);
+    return launch_pdl(small_kernel<DTYPE>, blocks, blocks, kSmallSmem, a, stream);
+  }
+  const int grid = grid_for(a.items);
+  if (dynamic) {
+    a.amax_blocks = grid;
+    cudaError_t e = launch_pdl(amax_kernel<DTYPE, WIDE>, grid, 1, 0, a, stream);
+    if (e != cudaSuccess) return e;
+  }
+  return launch_pdl(quant_kernel<DTYPE, WIDE>, grid, 1, 0, a, stream);
 }
 
 }  // namespace qk
 
-size_t quantize_scratch_words(int nseg) { return static_cast<size_t>(nseg) + 1; }
+size_t quantize_scratch_bytes(int nseg) { return static_cast<size_t>(kMaxAmaxBlocks) * nseg * sizeof(float); }
 
 cudaError_t launch_quantize(const void* x, int dtype, int64_t M, int64_t K, int64_t ld,
-                            const RowSegments& segs, const float* g_in, unsigned int* ws,
+                            const RowSegments& segs, const float* g_in, void* ws,
                             float* g_out, uint8_t* codes, uint8_t* sf, cudaStream_t stream) {
   using namespace qk;
   QuantArgs a{};
@@ -364,32 +608,21 @@ cudaError_t launch_quantize(const void* x, int dtype, int64_t M, int64_t K, int6
   a.K = static_cast<int32_t>(K);
   a.rows_pad = static_cast<int32_t>(ceil_div(M, 128) * 128);
   a.cpr = static_cast<int32_t>(ceil_div(K, kChunk));
-  a.items_q = a.rows_pad * a.cpr;
-  a.items_a = a.M * a.cpr;
+  a.items = static_cast<int64_t>(a.M) * a.cpr;
+  a.cpr_inv = a.cpr == 1 ? 0 : ~0ull / static_cast<uint64_t>(a.cpr) + 1;
   a.nseg = segs.n;
   for (int i = 0; i <= kMaxSeg; ++i)
     a.seg_begin[i] = static_cast<int32_t>(i <= segs.n ? segs.begin[i] : segs.begin[segs.n]);
   a.g_in = g_in;
-  a.ws = ws;
+  a.partial = static_cast<float*>(ws);
   a.g_out = g_out;
   a.codes = codes;
   a.sf = sf;
   const bool dynamic = g_in == nullptr;
-  if (dynamic) {
-    cudaError_t e = cudaMemsetAsync(ws, 0, sizeof(unsigned int) * quantize_scratch_words(segs.n), stream);
-    if (e != cudaSuccess) return e;
-  }
   const bool wide = (reinterpret_cast<uintptr_t>(x) % 32 == 0) && (a.ld_bytes % 32 == 0);
-  if (dtype == NVFP4_DTYPE_BF16) {
-    if (dynamic) return wide ? launch_t<NVFP4_DTYPE_BF16, true, true>(a, stream)
-                             : launch_t<NVFP4_DTYPE_BF16, false, true>(a, stream);
-    return wide ? launch_t<NVFP4_DTYPE_BF16, true, false>(a, stream)
-                : launch_t<NVFP4_DTYPE_BF16, false, false>(a, stream);
-  }
-  if (dynamic) return wide ? launch_t<NVFP4_DTYPE_F32, true, true>(a, stream)
-                           : launch_t<NVFP4_DTYPE_F32, false, true>(a, stream);
-  return wide ? launch_t<NVFP4_DTYPE_F32, true, false>(a, stream)
-              : launch_t<NVFP4_DTYPE_F32, false, false>(a, stream);
+  if (dtype == NVFP4_DTYPE_BF16)
+    return wide ? launch_t<NVFP4_DTYPE_BF16, true>(a, dynamic, stream) : launch_t<NVFP4_DTYPE_BF16, false>(a, dynamic, stream);
+  return wide ? launch_t<NVFP4_DTYPE_F32, true>(a, dynamic, stream) : launch_t<NVFP4_DTYPE_F32, false>(a, dynamic, stream);
 }
 
 }  // namespace nvfp4

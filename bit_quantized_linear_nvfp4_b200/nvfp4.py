@@ -43,7 +43,7 @@ EXPORTED = (
     "nvfp4_status_string", "nvfp4_last_cuda_error", "nvfp4_sf_bytes",
     "nvfp4_quantize_workspace_bytes", "nvfp4_quantize", "nvfp4_quantize_segments",
     "nvfp4_gemm_workspace_bytes", "nvfp4_gemm", "nvfp4_fused_proj", "nvfp4_check",
-    "nvfp4_quantize_noalloc",
+    "nvfp4_quantize_noalloc", "nvfp4_linear",
 )
 
 
@@ -106,6 +106,10 @@ def _lib():
         lib.nvfp4_quantize_noalloc.restype = c.c_int
         lib.nvfp4_quantize_noalloc.argtypes = [c.c_void_p, c.c_int, c.c_int64, c.c_int64, c.c_int64,
                                                c.c_void_p, c.c_void_p, c.c_void_p, c.c_void_p]
+        lib.nvfp4_linear.restype = c.c_int
+        lib.nvfp4_linear.argtypes = [c.c_void_p, c.c_int, c.c_int64, c.c_int64, c.c_int64, c.c_void_p,
+                                     c.c_void_p, c.c_void_p, c.c_void_p, c.POINTER(_Operand), c.c_void_p,
+                                     c.POINTER(_Segment), c.c_int, c.c_void_p, c.c_size_t, c.c_void_p]
         lib.nvfp4_check.restype = c.c_int
         lib.nvfp4_check.argtypes = [c.c_void_p]
         _LIB = lib
@@ -235,10 +239,7 @@ class Segment:
     dt_bias: Optional[torch.Tensor] = None
 
 
-def nvfp4_fused_proj(A: Operand, g_a: torch.Tensor, W: Operand, seg_global_scale: torch.Tensor,
-                     segments: Sequence[Segment], workspace=None, stream=None):
-    """One GEMM over the segments, each with its own global scale and epilogue;
-    results go to each segment's `out` tensor."""
+def _segment_array(segments: Sequence[Segment]):
     n = len(segments)
     arr = (_Segment * n)()
     for i, s in enumerate(segments):
@@ -250,6 +251,14 @@ def nvfp4_fused_proj(A: Operand, g_a: torch.Tensor, W: Operand, seg_global_scale
         arr[i].ld_out = 0 if s.out is None else s.out.stride(0)
         arr[i].A_log = None if s.A_log is None else s.A_log.data_ptr()
         arr[i].dt_bias = None if s.dt_bias is None else s.dt_bias.data_ptr()
+    return arr, n
+
+
+def nvfp4_fused_proj(A: Operand, g_a: torch.Tensor, W: Operand, seg_global_scale: torch.Tensor,
+                     segments: Sequence[Segment], workspace=None, stream=None):
+    """One GEMM over the segments, each with its own global scale and epilogue;
+    results go to each segment's `out` tensor."""
+    arr, n = _segment_array(segments)
     need = nvfp4_gemm_workspace_bytes(A.rows, W.rows, A.K)
     if workspace is None and need > 0:
         workspace = torch.empty(need, dtype=torch.uint8, device=A.codes.device)
@@ -257,6 +266,29 @@ def nvfp4_fused_proj(A: Operand, g_a: torch.Tensor, W: Operand, seg_global_scale
     a, w = A._c(), W._c()
     _call("nvfp4_fused_proj", ctypes.byref(a), _ptr(g_a), ctypes.byref(w), _ptr(seg_global_scale),
           arr, n, _ptr(workspace), ws_bytes, _stream(stream))
+
+
+def nvfp4_linear(x: torch.Tensor, W: Operand, seg_global_scale: torch.Tensor, segments: Sequence[Segment],
+                 g_in: Optional[torch.Tensor] = None, *, a_codes=None, a_sf=None, g_a=None, workspace=None,
+                 stream=None):
+    """Quantise x[M, K] and run the fused projection on it in one call (the GEMM
+    may start streaming W while the quantiser runs).  Returns (A, g_a): the
+    quantised activation left in a_codes / a_sf / g_a."""
+    _check_2d(x)
+    M, K = x.shape
+    dev = x.device
+    a_codes = torch.empty((M, K // 2), dtype=torch.uint8, device=dev) if a_codes is None else a_codes
+    a_sf = torch.empty(nvfp4_sf_bytes(max(M, 1), K), dtype=torch.uint8, device=dev) if a_sf is None else a_sf
+    g_a = torch.empty(1, dtype=torch.float32, device=dev) if g_a is None else g_a
+    if g_in is None and workspace is None:
+        workspace = torch.empty(nvfp4_quantize_workspace_bytes(1), dtype=torch.uint8, device=dev)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    arr, n = _segment_array(segments)
+    w = W._c()
+    _call("nvfp4_linear", _ptr(x), _dtype_code(x), M, K, x.stride(0), _ptr(g_in), _ptr(a_codes), _ptr(a_sf),
+          _ptr(g_a), ctypes.byref(w), _ptr(seg_global_scale), arr, n, _ptr(workspace), ws_bytes,
+          _stream(stream))
+    return Operand(a_codes, a_sf, M, K), g_a
 
 
 def nvfp4_check(stream=None):

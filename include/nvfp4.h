@@ -28,6 +28,11 @@
  *     128 rows x 4 scales, scale (r, j) at byte
  *       ((r/128) * KA + j/4) * 512 + (r%32)*16 + ((r/32)%4)*4 + j%4,
  *     KA = ceil(K/64).  Padding bytes are zero (nvfp4_quantize writes them).
+ *   - Every kernel is launched with programmatic stream serialization: it
+ *     may start while the kernel before it on the stream is finishing, and
+ *     waits for that kernel to complete before it reads or writes any
+ *     argument buffer.  Only nvfp4_linear reads a buffer (the weights) before
+ *     that point, and only while its own quantiser runs.
  *   - Devices: compute capability 10.0 (B200) only.
  */
 #ifndef NVFP4_H
@@ -113,7 +118,8 @@ size_t nvfp4_quantize_workspace_bytes(int nseg);
  *           Values must be finite.
  *   K       multiple of 16.  M >= 0 (M == 0 writes only g_out).
  *   g_in    device float, a calibrated (static) global scale, or NULL to use
- *           g = amax|x| / 2688 computed on the device (two passes over x).
+ *           g = amax|x| / 2688 computed on the device (two launches, two passes
+ *           over x; the second re-reads x from L2 when it fits there).
  *   g_out   device float, receives the global scale used (may equal g_in).
  *   codes   device, [M, K/2] bytes, 16-byte aligned.
  *   sf      device, nvfp4_sf_bytes(M, K) bytes, 16-byte aligned; padding zeroed.
@@ -151,7 +157,7 @@ int nvfp4_quantize_segments(const void* w, int w_dtype, int64_t N, int64_t K, in
  * quantise activations: a plugin enqueued by an inference runtime that owns
  * all memory, code running under a fixed memory plan, or a C caller that only
  * holds the tensors it was given.  The dynamic scale needs a few bytes of
- * device scratch between its two passes; this entry point keeps that scratch
+ * device scratch between its two launches; this entry point keeps that scratch
  * in a static array inside the library (NVFP4_NOALLOC_SCRATCH_BYTES bytes,
  * held on every GPU that loads the library until the process exits), so the
  * caller passes only inputs and outputs and nothing is allocated.
@@ -161,16 +167,18 @@ int nvfp4_quantize_segments(const void* w, int w_dtype, int64_t N, int64_t K, in
  *   NVFP4_ERR_UNSUPPORTED_SHAPE.
  *   The first call on a device looks up the scratch address on that device;
  *   make that first call before any stream capture on the device.
- *   Every call shares the one scratch array (each call clears it before use):
+ *   Every call shares the one scratch array (each call writes the scratch it
+ *   later reads, so it needs no clearing):
  *   calls whose work overlaps on the GPU, on different streams, race and must
  *   be serialised by the caller.
  */
-#define NVFP4_NOALLOC_SCRATCH_BYTES 256
+#define NVFP4_NOALLOC_SCRATCH_BYTES 1024
 int nvfp4_quantize_noalloc(const void* x, int x_dtype, int64_t M, int64_t K, int64_t ld_x,
                            float* g_out, uint8_t* codes, uint8_t* sf, void* stream);
 
 /* Workspace bytes nvfp4_gemm / nvfp4_fused_proj need for an [M, N, K]
- * problem (non-zero for the small-M weight-streaming path only). */
+ * problem (currently 0 for every shape; the argument is kept so that a
+ * future path may use scratch). */
 size_t nvfp4_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K);
 
 /*
@@ -204,6 +212,29 @@ int nvfp4_gemm(const nvfp4_operand* A, const float* g_a, const nvfp4_operand* W,
 int nvfp4_fused_proj(const nvfp4_operand* A, const float* g_a, const nvfp4_operand* W,
                      const float* seg_global_scale, const nvfp4_segment* segs, int nseg,
                      void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * nvfp4_linear — the W4A4 linear layer in one call: quantise the activation x
+ * (as nvfp4_quantize) into the caller's buffers, then run nvfp4_fused_proj on
+ * the result ("Methodology in Plain English": activations are quantised on
+ * the fly, weights offline; "Main Findings", fused-GEMM bullets for the
+ * segments).  Because the library launches both kernels, the GEMM may start
+ * streaming W while the quantiser is still running; for few tokens (the
+ * weight-streaming, decode-shaped GEMM) that hides the quantiser.
+ *   x, x_dtype, M, K, ld_x, g_in   as nvfp4_quantize (K a multiple of 32).
+ *   a_codes, a_sf, g_a   device outputs of the quantiser (as codes, sf, g_out
+ *                        of nvfp4_quantize); afterwards they hold the
+ *                        quantised activation.  They and the workspace must
+ *                        not overlap W's buffers or seg_global_scale.
+ *   W, seg_global_scale, segs, nseg   as nvfp4_fused_proj (W->K == K).
+ *   workspace / workspace_bytes   as nvfp4_quantize (the GEMM needs none).
+ * M == 0 enqueues nothing.  All arguments are checked before either launch.
+ */
+int nvfp4_linear(const void* x, int x_dtype, int64_t M, int64_t K, int64_t ld_x,
+                 const float* g_in, uint8_t* a_codes, uint8_t* a_sf, float* g_a,
+                 const nvfp4_operand* W, const float* seg_global_scale,
+                 const nvfp4_segment* segs, int nseg, void* workspace,
+                 size_t workspace_bytes, void* stream);
 
 /*
  * nvfp4_check — synchronise `stream`, then report (and clear) the library's

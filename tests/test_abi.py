@@ -122,3 +122,31 @@ def test_segmented_quantize_rejects_bad_bounds(lib):
     assert call([1, 256]) == 1
     assert call([0, 200]) == 1
     assert call([0] + list(range(10, 256, 30)) + [256]) == 1   # more than 8 segments
+
+
+def _lin(lib, x=FAKE, M=4, K=256, ld=256, g_in=FAKE, ac=FAKE, asf=FAKE, ga=FAKE, W=None, sc=FAKE,
+         segs=None, ws=None, wsb=0):
+    v = ctypes.c_void_p
+    W = W or _op(codes=0x400000, sf=0x800000, rows=256)
+    if segs is None:
+        segs = [nv._Segment(0, 256, 0, 0, 0x900000, 256, None, None)]
+    arr = (nv._Segment * len(segs))(*segs)
+    return lib.nvfp4_linear(v(x) if x else None, 0, M, K, ld, v(g_in) if g_in else None,
+                            v(ac) if ac else None, v(asf) if asf else None, v(ga) if ga else None,
+                            ctypes.byref(W), v(sc) if sc else None, arr, len(segs), v(ws) if ws else None,
+                            wsb, None)
+
+
+def test_linear_rejects_bad_arguments(lib):
+    assert _lin(lib, K=24, ld=32) == 2                        # K % 16
+    assert _lin(lib, x=0) == 1
+    assert _lin(lib, ga=0) == 1                               # g_a receives the scale
+    assert _lin(lib, W=_op(codes=0x400000, sf=0x800000, rows=256, K=512)) == 1   # K mismatch
+    assert _lin(lib, g_in=0) == 6                             # dynamic scale without workspace
+    # nothing the quantiser writes may overlap W (the GEMM streams W early)
+    assert _lin(lib, ac=0x400000 + 64) == 1
+    assert _lin(lib, asf=0x800000) == 1
+    assert _lin(lib, ga=0x400010) == 1
+    assert _lin(lib, g_in=0, ws=0x800000 + 1024, wsb=4096) == 1
+    assert _lin(lib, segs=[nv._Segment(0, 100, 0, 0, 0x900000, 256, None, None)]) == 1   # segments
+    assert _lin(lib, M=0) == 0                                # empty: nothing enqueued
