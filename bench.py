@@ -140,7 +140,7 @@ def workload_spec(name: str):
 class ProductStep:
     """Device buffers for ROTATE input sets and CUDA graphs of the two stages."""
 
-    def __init__(self, name: str, device):
+    def __init__(self, name: str, device, rows=None):
         import torch
         from bit_quantized_linear_nvfp4_b200 import nvfp4 as nv
         from bit_quantized_linear_nvfp4_b200 import workloads as wl
@@ -150,7 +150,8 @@ class ProductStep:
         self.w = workload_spec(name)
         if self.w is None:
             M, K = wl.QUANT_SHAPE
-            x_np = wl.make_quant_input()
+            M = M if rows is None else rows  # a smaller case of the same kernels (profiling)
+            x_np = wl.make_quant_input(rows=M)
             self.M, self.K, self.N = M, K, 0
             self.flops = 0.0
             self.sets = [self._act_set(x_np)]  # 1.14 GB input, larger than L2
@@ -289,7 +290,7 @@ def run_product(args):
     dist = dist_init(world)
     peaks, peak_src = load_peaks()
 
-    step = ProductStep(args.workload, device)
+    step = ProductStep(args.workload, device, rows=args.rows)
     step.capture()
     stream = torch.cuda.current_stream()
     K, Wm = args.steps, args.warmup
@@ -532,6 +533,8 @@ def main():
     ap.add_argument("--impl", default="product", choices=["product", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--rows", type=int, default=None,
+                    help="quant workload only: quantise [rows, 17408] instead of the full tensor (for profiler captures)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

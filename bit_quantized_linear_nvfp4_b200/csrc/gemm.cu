@@ -193,12 +193,16 @@ __device__ __forceinline__ void store_swiglu(const KernelArgs& a, int64_t row, i
   const float ga = __ldg(a.g_a);
   const float sgate = ga * __ldg(a.seg_scale + 0);
   const float sup = ga * __ldg(a.seg_scale + 1);
+  // silu(g) * u = g * sigmoid(g) * u.  The result is rounded to BF16 (8-bit
+  // mantissa), so the fast exponential (a few FP32 ulp) and a correctly
+  // rounded reciprocal are ample; 1 / (1 + e^-g) stays correct at both ends
+  // (e^-g overflowing to inf gives 0).
   float v[32];
 #pragma unroll
   for (int j = 0; j < 32; ++j) {
     const float gv = __uint_as_float(rg[j]) * sgate;
     const float uv = __uint_as_float(ru[j]) * sup;
-    v[j] = gv / (1.0f + expf(-gv)) * uv;
+    v[j] = gv * __frcp_rn(1.0f + __expf(-gv)) * uv;
   }
   __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(sg.out) + row * sg.ld_out + o0;
   if (o0 + 31 < a.n_out && (o0 % 8) == 0) {
@@ -996,6 +1000,18 @@ cudaError_t launch_gemm(const GemmProblem& p, void*, size_t, cudaStream_t stream
   a.num_n_blocks = static_cast<int>(p.swiglu ? ceil_div(p.N / 2, 128) : ceil_div(p.N, BN));
   a.num_k_stages = static_cast<int>(ceil_div(p.K, BK));
   a.group_m = pair_kernel ? 8 : 16;
+  if (pair_kernel) {
+    // Tiles are walked m-fastest inside groups of group_m row blocks: the
+    // group's A panels stay in L2 while W streams through once per group.
+    // When all of A fits in L2 with room for the output stream, one group
+    // covers every row block, so W is read from DRAM once.  (Keeping W
+    // resident instead, one row block per group, cut DRAM reads for the GDN
+    // shape but ran slower: every pair then starts the same new A panel at
+    // once.)
+    const double a_bytes = static_cast<double>(p.M) * static_cast<double>(p.K) * (0.5 + 1.0 / 16);
+    constexpr double kResident = 48.0 * 1024 * 1024;
+    if (a_bytes <= kResident) a.group_m = a.num_m_blocks;
+  }
   a.g_a = p.g_a;
   a.seg_scale = p.seg_scale;
   a.nseg = p.nseg;
