@@ -13,10 +13,12 @@
 //    128-row block of W and each streams 1/S of K, so about S * N/128 CTAs
 //    stream W at once.
 //  * The S partial accumulators are summed through distributed shared memory:
-//    peers stage their FP32 partial in their own shared memory and arrive on
-//    the leader's mbarrier; the leader adds them in rank order (deterministic),
-//    applies the global scales and the segment's epilogue, stores, and then
-//    releases the peers.  No workspace, no atomics.  All waits are bounded.
+//    every CTA stages its FP32 partial in its own shared memory; after a
+//    cluster barrier each CTA finalises a share of the tokens, adding the
+//    ranks' partials in rank order (deterministic), applying the global
+//    scales and the segment's epilogue and storing.  A second cluster barrier
+//    keeps every CTA alive until the others have read it.  No workspace, no
+//    atomics; all mbarrier waits are bounded.
 //
 // Warps: 0 TMA producer, 1 TMEM owner + MMA issuer, 2..5 epilogue (one TMEM
 // lane quadrant each).
@@ -72,7 +74,8 @@ constexpr int kMaxStages = 12;
 struct DecodeArgs {
   int64_t M, N, K;
   int num_k_stages, split;
-  int w_prefetch;  // W is not written by the kernel before this one on the stream
+  int w_prefetch;   // W is not written by the kernel before this one on the stream
+  int l2_prefetch;  // W fits in L2: request a CTA's whole W range up front
   const float* g_a;
   const float* seg_scale;
   int nseg;
@@ -83,8 +86,6 @@ struct Tail {
   uint64_t full[kMaxStages];
   uint64_t empty[kMaxStages];
   uint64_t tmem_full;
-  uint64_t ready;  // leader: peers' partials staged
-  uint64_t done;   // peer: leader finished reading
   uint64_t drain;
   uint32_t tmem_base;
   int abort_flag;
@@ -126,8 +127,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&tail->empty[s], 1);
     }
     mbar_init(&tail->tmem_full, 1);
-    mbar_init(&tail->ready, S > 1 ? kEpiWarps * 32 * (S - 1) : 1);
-    mbar_init(&tail->done, 1);
     mbar_init(&tail->drain, 1);
     tail->abort_flag = 0;
     fence_mbarrier_init();
@@ -171,13 +170,25 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool issued[kStages] = {};
       uint32_t issued_phase[kStages] = {};
       // Weights may stream before the previous kernel (the activation
-      // quantiser) has finished: fill the first stages with W only.
+      // quantiser) has finished: fill the first stages with W only, and
+      // request the rest of this CTA's W range into L2 (when W fits there),
+      // so that HBM streams W while the quantiser runs.  (Issued after the
+      // wait instead, with nothing to overlap, the L2 requests only compete
+      // with the stage loads; standalone calls skip them.)
       const int npre = args.w_prefetch ? min(kStages, ks1 - ks0) : 0;
       for (int i = 0; i < npre; ++i) {
         mbar_arrive_expect_tx(&tail->full[i], C::kStageRaw);
         load_w(i, ks0 + i);
         issued[i] = true;
       }
+      if (args.w_prefetch && args.l2_prefetch)
+        for (int ks = ks0 + npre; ks < ks1; ++ks) {
+          if constexpr (CH == 1)
+            tma_prefetch_l2_2d(&tm_w, ks * (BK / 2), rb * BM);
+          else
+            tma_prefetch_l2_3d(&tm_w, 0, rb * BM, ks * CH);
+          tma_prefetch_l2_3d(&tm_sfw, 0, ks * 4 * CH, rb);
+        }
       grid_dependency_wait();
       grid_launch_dependents();
       for (int ks = ks0; ks < ks1; ++ks) {
@@ -270,77 +281,95 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int t = 0; t < BN; ++t) acc[t] = 0.0f;
     }
     tc_fence_before();
-    // [row][token] with row stride kPartLd, reusing the stage buffers
+    // this CTA's FP32 partial, row-major ([row][token], row stride kPartLd),
+    // staged in its stage buffers for the whole cluster to read
     float* partial = reinterpret_cast<float*>(smem) + row_local * C::kPartLd;
-    const uint32_t ready_local = smem_u32(&tail->ready);
-    if (rank != 0) {
 #pragma unroll
-      for (int t = 0; t < BN; t += 4)
-        *reinterpret_cast<float4*>(partial + t) = make_float4(acc[t], acc[t + 1], acc[t + 2], acc[t + 3]);
-      mbar_arrive_remote(map_to_rank(ready_local, 0));
-      mbar_wait_cluster_bounded(&tail->done, 0);
-    } else {
-      const bool ok = S == 1 || mbar_wait_cluster_bounded(&tail->ready, 0);
-      if (ok) {
-        for (int p = 1; p < S; ++p) {
-          const uint32_t peer = map_to_rank(smem_u32(partial), p);
-          // every load of this peer is issued before the first add; groups of
-          // 16 tokens, tokens >= M are zero rows of X and never stored
-          float v[BN];
+    for (int t = 0; t < BN; t += 4)
+      *reinterpret_cast<float4*>(partial + t) = make_float4(acc[t], acc[t + 1], acc[t + 2], acc[t + 3]);
+  }
+  // every CTA of the cluster has staged its partial
+  cluster_sync_all();
+  if (warp >= 2) {
+    // This CTA finalises token groups [g0, g1) of 4 tokens: the sum of the
+    // ranks' partials in rank order (the same arithmetic whichever CTA does
+    // it), then the segment's epilogue.  Tokens >= M are zero rows of X and
+    // are never stored.
+    const int q = warp & 3;
+    const int row_local = q * 32 + lane;
+    const int64_t n = static_cast<int64_t>(rb) * BM + row_local;
+    constexpr int kG = BN / 4;
+    const int G = (static_cast<int>(args.M) + 3) / 4;
+    const int g0 = static_cast<int>(rank) * G / S, g1 = (static_cast<int>(rank) + 1) * G / S;
+    float4 sum[kG];
 #pragma unroll
-          for (int t0 = 0; t0 < BN; t0 += 16)
-            if (t0 < args.M) ld_shared_cluster_f32x16(peer + 4u * t0, v + t0);
+    for (int i = 0; i < kG; ++i) sum[i] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+    const uint32_t mine = smem_u32(reinterpret_cast<float*>(smem) + row_local * C::kPartLd);
+    for (int p = 0; p < S; ++p) {
+      const uint32_t src = map_to_rank(mine, static_cast<uint32_t>(p));
+      float4 v[kG];
+      // every load of this rank is issued before the first add
 #pragma unroll
-          for (int t0 = 0; t0 < BN; t0 += 16)
-            if (t0 < args.M)
+      for (int i = 0; i < kG; ++i)
+        if (g0 + i < g1) v[i] = ld_shared_cluster_f32x4(src + 16u * static_cast<uint32_t>(g0 + i));
 #pragma unroll
-              for (int t = 0; t < 16; ++t) acc[t0 + t] += v[t0 + t];
+      for (int i = 0; i < kG; ++i)
+        if (g0 + i < g1) {
+          sum[i].x += v[i].x;
+          sum[i].y += v[i].y;
+          sum[i].z += v[i].z;
+          sum[i].w += v[i].w;
         }
-      }
-      if (ok && n < args.N) {
-        int s = 0;
+    }
+    if (g1 > g0 && n < args.N) {
+      int s = 0;
 #pragma unroll
-        for (int i = 1; i < kMaxSeg; ++i)
-          if (i < args.nseg && n >= args.seg[i].n_begin) s = i;
-        // the segment's parameters, loaded once; one tight loop per kind
-        const int kind = args.seg[s].kind;
-        const int64_t ld = args.seg[s].ld_out;
-        const int64_t j = n - args.seg[s].n_begin;
-        const float scale = __ldg(args.g_a) * __ldg(args.seg_scale + s);
-        const int mt = args.M < BN ? static_cast<int>(args.M) : BN;
+      for (int i = 1; i < kMaxSeg; ++i)
+        if (i < args.nseg && n >= args.seg[i].n_begin) s = i;
+      // the segment's parameters, loaded once; one tight loop per kind
+      const int kind = args.seg[s].kind;
+      const int64_t ld = args.seg[s].ld_out;
+      const int64_t j = n - args.seg[s].n_begin;
+      const float scale = __ldg(args.g_a) * __ldg(args.seg_scale + s);
+      const int mt = static_cast<int>(args.M);
+      float a_log = 0.0f, dt = 0.0f;
+      if (kind == NVFP4_EPI_GDN_DECAY_F32) {
+        a_log = -expf(__ldg(args.seg[s].a_log + j));
+        dt = __ldg(args.seg[s].dt_bias + j);
+      }
+#pragma unroll
+      for (int i = 0; i < kG; ++i) {
+        if (g0 + i >= g1) break;
+        const int t0 = 4 * (g0 + i);
+        const float y[4] = {sum[i].x * scale, sum[i].y * scale, sum[i].z * scale, sum[i].w * scale};
         if (kind == NVFP4_EPI_IDENTITY_BF16) {
           __nv_bfloat16* o = static_cast<__nv_bfloat16*>(args.seg[s].out) + j;
 #pragma unroll
-          for (int t = 0; t < BN; ++t)
-            if (t < mt) o[t * ld] = __float2bfloat16_rn(acc[t] * scale);
+          for (int c = 0; c < 4; ++c)
+            if (t0 + c < mt) o[(t0 + c) * ld] = __float2bfloat16_rn(y[c]);
         } else if (kind == NVFP4_EPI_IDENTITY_F32) {
           float* o = static_cast<float*>(args.seg[s].out) + j;
 #pragma unroll
-          for (int t = 0; t < BN; ++t)
-            if (t < mt) o[t * ld] = acc[t] * scale;
+          for (int c = 0; c < 4; ++c)
+            if (t0 + c < mt) o[(t0 + c) * ld] = y[c];
         } else if (kind == NVFP4_EPI_SIGMOID_F32) {
           float* o = static_cast<float*>(args.seg[s].out) + j;
 #pragma unroll
-          for (int t = 0; t < BN; ++t)
-            if (t < mt) o[t * ld] = sigmoid_f(acc[t] * scale);
+          for (int c = 0; c < 4; ++c)
+            if (t0 + c < mt) o[(t0 + c) * ld] = sigmoid_f(y[c]);
         } else {
           float* o = static_cast<float*>(args.seg[s].out) + j;
-          const float a_log = -expf(__ldg(args.seg[s].a_log + j));
-          const float dt = __ldg(args.seg[s].dt_bias + j);
 #pragma unroll
-          for (int t = 0; t < BN; ++t)
-            if (t < mt) o[t * ld] = a_log * softplus_f(acc[t] * scale + dt);
+          for (int c = 0; c < 4; ++c)
+            if (t0 + c < mt) o[(t0 + c) * ld] = a_log * softplus_f(y[c] + dt);
         }
       }
-      // every epilogue thread of the leader has finished reading the peers
-      named_barrier_sync(1, kEpiWarps * 32);
-      if (threadIdx.x == 64)
-        for (int p = 1; p < S; ++p) mbar_arrive_remote(map_to_rank(smem_u32(&tail->done), p));
     }
   }
 
+  // no CTA leaves (or reuses its shared memory) while another may read it
   tc_fence_before();
-  __syncthreads();
+  cluster_sync_all();
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
@@ -381,6 +410,7 @@ cudaError_t launch_bn(const GemmProblem& p, cudaStream_t stream) {
   a.N = p.N;
   a.K = p.K;
   a.w_prefetch = p.w_prefetch ? 1 : 0;
+  a.l2_prefetch = static_cast<double>(p.N) * static_cast<double>(p.K) * (0.5 + 1.0 / 16) <= 64.0 * 1024 * 1024;
   a.num_k_stages = static_cast<int>(ceil_div(ceil_div(p.K, BK), CH));
   a.g_a = p.g_a;
   a.seg_scale = p.seg_scale;

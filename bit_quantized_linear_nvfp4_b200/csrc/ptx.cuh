@@ -121,6 +121,18 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t b
                : "memory");
 }
 
+// Prefetch a tensor-map box into L2 (no shared memory, no barrier).
+__device__ __forceinline__ void tma_prefetch_l2_2d(const CUtensorMap* m, int32_t x, int32_t y) {
+  asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];"
+               ::"l"(reinterpret_cast<uint64_t>(m)), "r"(x), "r"(y)
+               : "memory");
+}
+__device__ __forceinline__ void tma_prefetch_l2_3d(const CUtensorMap* m, int32_t x, int32_t y, int32_t z) {
+  asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global.tile [%0, {%1, %2, %3}];"
+               ::"l"(reinterpret_cast<uint64_t>(m)), "r"(x), "r"(y), "r"(z)
+               : "memory");
+}
+
 __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* m, uint64_t* bar,
                                             int32_t x, int32_t y) {
   asm volatile(
@@ -296,19 +308,15 @@ __device__ __forceinline__ float ld_shared_cluster_f32(uint32_t cluster_saddr) {
   return v;
 }
 
-// Sixteen consecutive floats of another CTA's shared memory (16-byte aligned
-// address) as four 128-bit loads in one statement, so that all four are in
-// flight before the first result is used.  Ordered after the preceding
-// acquire by the volatile asm sequence.
-__device__ __forceinline__ void ld_shared_cluster_f32x16(uint32_t cluster_saddr, float* v) {
-  asm volatile(
-      "ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%16];\n\t"
-      "ld.shared::cluster.v4.f32 {%4, %5, %6, %7}, [%16+16];\n\t"
-      "ld.shared::cluster.v4.f32 {%8, %9, %10, %11}, [%16+32];\n\t"
-      "ld.shared::cluster.v4.f32 {%12, %13, %14, %15}, [%16+48];"
-      : "=f"(v[0]), "=f"(v[1]), "=f"(v[2]), "=f"(v[3]), "=f"(v[4]), "=f"(v[5]), "=f"(v[6]), "=f"(v[7]),
-        "=f"(v[8]), "=f"(v[9]), "=f"(v[10]), "=f"(v[11]), "=f"(v[12]), "=f"(v[13]), "=f"(v[14]), "=f"(v[15])
-      : "r"(cluster_saddr));
+// Four consecutive floats of another CTA's shared memory (16-byte aligned
+// address), ordered after the preceding cluster barrier by the volatile asm
+// sequence; no memory clobber, so consecutive loads issue back to back.
+__device__ __forceinline__ float4 ld_shared_cluster_f32x4(uint32_t cluster_saddr) {
+  float4 v;
+  asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
+               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+               : "r"(cluster_saddr));
+  return v;
 }
 
 __device__ __forceinline__ void named_barrier_sync(uint32_t id, uint32_t threads) {
