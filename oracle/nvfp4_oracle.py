@@ -288,6 +288,30 @@ def common_global_scale(seg_scales) -> np.float32:
     return np.float32(np.min(np.asarray(seg_scales, np.float32)))
 
 
+def requantize(codes: np.ndarray, sf: np.ndarray, g_rows, g_new):
+    """Checkpoint-side harmonisation of fused modules' scales (Paper summary
+    page (ai.info), "Methodology in Plain English": the fused modules' global
+    scales are made to agree on the checkpoint side, so that a kernel applying
+    one scale to the fused GEMM is correct).  Reading: every element is
+    dequantised with its own module's scale, rounded once to FP32
+    (x_hat = e2m1 * S * g_old; e2m1 * S is exact), and the result is quantised
+    again with the common scale g_new exactly as quantize() does.  The common
+    scale that clips nothing is the largest module scale, which is the scale
+    of the fused (concatenated) weight; a smaller one makes the larger
+    modules' block scales saturate.
+
+    g_rows: the old global scale of each row (float32[M]) or one scalar.
+    Returns (codes, sf, g_new) like quantize().
+    """
+    codes = np.asarray(codes, np.uint8)
+    M, K = codes.shape
+    g_rows = np.broadcast_to(np.asarray(g_rows, np.float64).reshape(-1, 1) if np.ndim(g_rows) else
+                             np.float64(g_rows), (M, 1))
+    vals = e2m1_decode(codes).reshape(M, K // BLOCK, BLOCK) * e4m3_decode(sf)[:, :, None]  # exact
+    x_hat = (vals.reshape(M, K) * g_rows).astype(np.float32)  # one rounding to FP32
+    return quantize(x_hat, np.float32(g_new))
+
+
 def bf16_round(y) -> np.ndarray:
     """Round FP64 values to BF16 (8 significant bits, nearest, ties to even);
     returned as FP64.  y = m * 2^e with 0.5 <= |m| < 1, so y / 2^(e-8) has its

@@ -1,0 +1,105 @@
+"""Pins for the oracle's checkpoint-side harmonisation (requantize), CPU only.
+
+requantize() re-encodes NVFP4 data quantised with one global scale under
+another.  What fixes it, independently of its own code:
+  * idempotence: re-encoding under the same scale returns the same codes and
+    scale bytes (the block maximum decodes to +-6 * S, so the re-derived block
+    scale is S again and every element lands back on its own code);
+  * a power-of-two change of scale, g_new = 2 g, halves every block scale that
+    stays a normal E4M3 value and leaves every code alone;
+  * per-row scales: rows of different modules use their own old scale (each
+    module's rows alone give the same result);
+  * re-encoding under a larger scale (block scales shrink, nothing clips)
+    keeps every value within the quantiser's half-step bound of the value it
+    started from; the largest module scale (the scale of the fused tensor,
+    amax over all modules / 2688) is therefore safe for every module;
+  * re-encoding under a smaller scale makes block scales grow: a module's
+    top block saturates at 448 and its largest elements clip.
+"""
+import numpy as np
+
+from oracle import nvfp4_oracle as o
+
+
+def _w(M, K, seed, scale=0.02):
+    rng = np.random.default_rng(seed)
+    return (scale * rng.standard_normal((M, K))).astype(np.float32)
+
+
+def test_idempotent_under_the_same_scale():
+    for seed in range(4):
+        x = _w(48, 256, seed, scale=1.0 + seed)
+        x[3, 17] *= 40  # an outlier block
+        c, s, g = o.quantize(x)
+        c2, s2, g2 = o.requantize(c, s, g, g)
+        assert g2 == g
+        assert np.array_equal(c2, c) and np.array_equal(s2, s)
+
+
+def test_power_of_two_scale_change_halves_block_scales():
+    x = _w(32, 512, 7)
+    c, s, g = o.quantize(x)
+    c2, s2, _ = o.requantize(c, s, g, np.float32(2) * g)
+    S, S2 = o.e4m3_decode(s), o.e4m3_decode(s2)
+    normal = S >= 2.0 ** -5  # S / 2 still a normal E4M3 value
+    assert normal.mean() > 0.9
+    assert np.all(S2[normal] == S[normal] / 2)
+    nb = np.repeat(normal, 16, axis=1)
+    assert np.array_equal(c2[nb], c[nb])
+
+
+def test_rows_use_their_own_module_scale():
+    a, b = _w(40, 128, 1, 0.02), _w(24, 128, 2, 0.05)
+    ca, sa, ga = o.quantize(a)
+    cb, sb, gb = o.quantize(b)
+    gc = o.common_global_scale([ga, gb])
+    g_rows = np.concatenate([np.full(40, ga, np.float32), np.full(24, gb, np.float32)])
+    c, s, g = o.requantize(np.concatenate([ca, cb]), np.concatenate([sa, sb]), g_rows, gc)
+    c1, s1, _ = o.requantize(ca, sa, ga, gc)
+    c2, s2, _ = o.requantize(cb, sb, gb, gc)
+    assert g == gc
+    assert np.array_equal(c, np.concatenate([c1, c2])) and np.array_equal(s, np.concatenate([s1, s2]))
+
+
+def _half_step_ok(c_old, s_old, g_old, c, s, g):
+    x_hat = o.dequantize(c_old, s_old, g_old)
+    y_hat = o.dequantize(c, s, g)
+    S = np.repeat(o.e4m3_decode(s), 16, axis=1).astype(np.float64)
+    v = np.abs(o.e2m1_decode(c))
+    step = np.where(v < 2, 0.5, np.where(v < 4, 1.0, 2.0))  # E2M1 grid step at the result
+    return np.all(np.abs(y_hat - x_hat) <= 0.5 * step * S * np.float64(g) * (1 + 1e-6) + 1e-30)
+
+
+def test_reencoded_values_within_half_step_under_a_larger_scale():
+    a = _w(64, 256, 3, 0.02)
+    ca, sa, ga = o.quantize(a)
+    for f in (1.3, 1.8, 2.75):
+        gc = np.float32(ga * f)
+        c, s, g = o.requantize(ca, sa, ga, gc)
+        assert np.all(o.e4m3_decode(s) <= o.e4m3_decode(sa))  # block scales shrink
+        assert _half_step_ok(ca, sa, ga, c, s, g)
+
+
+def test_harmonising_to_the_fused_tensor_scale():
+    """The largest module scale equals the scale of the concatenated weight."""
+    mods = [_w(32, 256, 10 + i, 0.02 * (1 + 2 * i)) for i in range(3)]
+    qs = [o.quantize(m) for m in mods]
+    g_fused = o.global_scale(np.concatenate(mods))
+    assert g_fused == max(g for _, _, g in qs)
+    for c, s, g in qs:
+        c2, s2, g2 = o.requantize(c, s, g, g_fused)
+        assert _half_step_ok(c, s, g, c2, s2, g2)
+
+
+def test_harmonising_to_a_smaller_scale_clips_the_top_block():
+    a = _w(32, 256, 4, 0.05)
+    ca, sa, ga = o.quantize(a)
+    gc = np.float32(ga / 2)  # the smaller scale of another module
+    c, s, g = o.requantize(ca, sa, ga, gc)
+    top = np.unravel_index(np.argmax(o.e4m3_decode(sa)), sa.shape)
+    assert sa[top] == 0x7E and s[top] == 0x7E  # 448 before and after: saturated
+    r, b = top
+    x_hat = o.dequantize(ca, sa, ga)[r, 16 * b:16 * b + 16]
+    y_hat = o.dequantize(c, s, g)[r, 16 * b:16 * b + 16]
+    assert np.abs(y_hat).max() == 6 * 448 * np.float64(gc)  # the largest value clips to 6 * 448 * gc
+    assert np.abs(x_hat).max() > 1.9 * np.abs(y_hat).max()
