@@ -272,6 +272,35 @@ int nvfp4_linear(const void* x, int x_dtype, int64_t M, int64_t K, int64_t ld_x,
   return NVFP4_OK;
 }
 
+int nvfp4_requantize_segments(const nvfp4_operand* W, const int64_t* row_bounds, int nseg,
+                              const float* g_old, const float* g_new, uint8_t* codes_out, uint8_t* sf_out,
+                              float* g_out, void* stream) {
+  int st = check_operand(W);
+  if (st != NVFP4_OK) return st;
+  if (row_bounds == nullptr || nseg < 1 || nseg > NVFP4_MAX_SEGMENTS) return NVFP4_ERR_INVALID_ARG;
+  if (row_bounds[0] != 0 || row_bounds[nseg] != W->rows) return NVFP4_ERR_INVALID_ARG;
+  nvfp4::RowSegments segs{};
+  segs.n = nseg;
+  for (int i = 0; i <= nseg; ++i) {
+    if (i > 0 && row_bounds[i] <= row_bounds[i - 1]) return NVFP4_ERR_INVALID_ARG;
+    segs.begin[i] = row_bounds[i];
+  }
+  if (g_old == nullptr || codes_out == nullptr || sf_out == nullptr || g_out == nullptr) return NVFP4_ERR_INVALID_ARG;
+  if (!aligned16(codes_out) || !aligned16(sf_out) || (reinterpret_cast<uintptr_t>(g_out) & 3u) != 0)
+    return NVFP4_ERR_MISALIGNED;
+  // in place, or into separate buffers: no partial overlap
+  const size_t nc = static_cast<size_t>(W->rows) * static_cast<size_t>(W->K / 2), ns = nvfp4::sf_bytes(W->rows, W->K);
+  if ((codes_out != W->codes && overlap(codes_out, nc, W->codes, nc)) || (sf_out != W->sf && overlap(sf_out, ns, W->sf, ns)) ||
+      overlap(codes_out, nc, sf_out, ns) || overlap(codes_out, nc, W->sf, ns) || overlap(sf_out, ns, W->codes, nc))
+    return NVFP4_ERR_INVALID_ARG;
+  st = check_device();
+  if (st != NVFP4_OK) return st;
+  cudaError_t e = nvfp4::launch_requantize(W->codes, W->sf, W->rows, W->K, segs, g_old, g_new, codes_out, sf_out, g_out,
+                                           static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e);
+  return NVFP4_OK;
+}
+
 int nvfp4_gemm(const nvfp4_operand* A, const float* g_a, const nvfp4_operand* W, const float* g_w,
                void* out, int out_dtype, int64_t ld_out, void* workspace, size_t workspace_bytes,
                void* stream) {

@@ -38,6 +38,13 @@ cudaError_t launch_quantize(const void* x, int dtype, int64_t M, int64_t K, int6
                             const RowSegments& segs, const float* g_in, void* ws,
                             float* g_out, uint8_t* codes, uint8_t* sf, cudaStream_t stream);
 
+// Re-encode codes/sf of [N, K] (row ranges `segs` quantised with g_old[s])
+// under one common scale (*g_new, or the largest g_old when g_new is null);
+// writes codes_out / sf_out (may equal the inputs) and g_out[s] = common scale.
+cudaError_t launch_requantize(const uint8_t* codes, const uint8_t* sf, int64_t N, int64_t K,
+                              const RowSegments& segs, const float* g_old, const float* g_new,
+                              uint8_t* codes_out, uint8_t* sf_out, float* g_out, cudaStream_t stream);
+
 // GEMM epilogue description handed to the kernels.
 struct EpiSegment {
   int64_t n_begin, n_end;

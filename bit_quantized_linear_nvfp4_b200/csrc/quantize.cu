@@ -533,6 +533,81 @@ __global__ void __launch_bounds__(kThreads, 1) small_kernel(const __grid_constan
   cluster_sync_all();  // no block leaves while another may read its maxima
 }
 
+// Checkpoint-side harmonisation: re-encode an NVFP4 operand whose row ranges
+// (modules) carry their own global scales under one common scale.  Each
+// element is dequantised with its module's scale and rounded once to FP32
+// (x_hat = e2m1 * S * g_old; e2m1 * S is exact), then quantised exactly as
+// the quantiser does.  The common scale is given, or the largest module
+// scale (the fused tensor's scale, which clips no block).  Works in place:
+// a lane reads its 8 code bytes and its scale byte before the warp writes.
+struct RequantArgs {
+  QuantArgs q;                 // output side: one segment, the common scale
+  const uint8_t* in_codes;
+  const uint8_t* in_sf;
+  const float* g_old;          // device [nseg_old]
+  const float* g_new;          // device [1] or nullptr
+  int nseg_old;
+  int32_t old_begin[kMaxSeg + 1];
+};
+
+__device__ __forceinline__ float e2m1_value(uint32_t c) {
+  // twice the magnitudes 0, .5, 1, 1.5, 2, 3, 4, 6 as nibbles
+  const float v = static_cast<float>((0xC8643210u >> (4 * (c & 7u))) & 15u) * 0.5f;
+  return (c & 8u) ? -v : v;
+}
+
+__global__ void __launch_bounds__(kThreads, 1) requant_kernel(const __grid_constant__ RequantArgs r) {
+  const QuantArgs& a = r.q;
+  __shared__ float g_sh[kMaxSeg];
+  __shared__ float g_old_sh[kMaxSeg];
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) grid_launch_dependents();
+  grid_dependency_wait();
+  if (threadIdx.x < r.nseg_old) g_old_sh[threadIdx.x] = r.g_old[threadIdx.x];
+  if (threadIdx.x == 0) {
+    float g = 0.0f;
+    if (r.g_new != nullptr) {
+      g = *r.g_new;
+    } else {
+      for (int i = 0; i < r.nseg_old; ++i) g = fmaxf(g, r.g_old[i]);
+    }
+    g_sh[0] = g;
+  }
+  __syncthreads();
+  if (blockIdx.x == 0 && threadIdx.x < r.nseg_old) a.g_out[threadIdx.x] = g_sh[0];
+  const int32_t KA = (a.K + 63) / 64;
+  int64_t lo, hi;
+  block_range(a.items, lo, hi);
+  for (int64_t i = lo + warp; i < hi; i += kWarps) {
+    int32_t row, col;
+    chunk_pos(a, i, row, col);
+    col += lane * 16;
+    const bool have = col < a.K;
+    Blk<NVFP4_DTYPE_F32> b;
+    if (have) {
+      const uint2 c = *reinterpret_cast<const uint2*>(r.in_codes + static_cast<int64_t>(row) * (a.K / 2) + col / 2);
+      const int32_t j = col / 16;
+      const uint32_t sfb = r.in_sf[(static_cast<int64_t>(row >> 7) * KA + (j >> 2)) * 512 + (row & 31) * 16 +
+                                   ((row >> 5) & 3) * 4 + (j & 3)];
+      int s = 0;
+#pragma unroll
+      for (int k = 1; k < kMaxSeg; ++k)
+        if (k < r.nseg_old && row >= r.old_begin[k]) s = k;
+      const float S = e4m3_value(sfb), g = g_old_sh[s];
+#pragma unroll
+      for (int e = 0; e < 16; ++e) {
+        const uint32_t word = e < 8 ? c.x : c.y;
+        const uint32_t code = (word >> (4 * (e & 7))) & 15u;
+        b.w[e] = __float_as_uint((e2m1_value(code) * S) * g);  // e2m1 * S exact, one rounding
+      }
+    }
+    __syncwarp();  // in place: every lane has read before any lane writes
+    quantize_block<NVFP4_DTYPE_F32>(a, g_sh, b, have, row, col);
+  }
+  zero_padding_rows(a);
+}
+
 int num_sms() {
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
@@ -595,6 +670,42 @@ cudaError_t launch_t(QuantArgs a, bool dynamic, cudaStream_t stream) {
 }  // namespace qk
 
 size_t quantize_scratch_bytes(int nseg) { return static_cast<size_t>(kMaxAmaxBlocks) * nseg * sizeof(float); }
+
+cudaError_t launch_requantize(const uint8_t* codes, const uint8_t* sf, int64_t N, int64_t K,
+                              const RowSegments& segs, const float* g_old, const float* g_new,
+                              uint8_t* codes_out, uint8_t* sf_out, float* g_out, cudaStream_t stream) {
+  using namespace qk;
+  RequantArgs r{};
+  QuantArgs& a = r.q;
+  a.M = static_cast<int32_t>(N);
+  a.K = static_cast<int32_t>(K);
+  a.rows_pad = static_cast<int32_t>(ceil_div(N, 128) * 128);
+  a.cpr = static_cast<int32_t>(ceil_div(K, kChunk));
+  a.items = static_cast<int64_t>(a.M) * a.cpr;
+  a.cpr_inv = a.cpr == 1 ? 0 : ~0ull / static_cast<uint64_t>(a.cpr) + 1;
+  a.nseg = 1;
+  for (int i = 0; i <= kMaxSeg; ++i) a.seg_begin[i] = i == 0 ? 0 : a.M;
+  a.g_out = g_out;
+  a.codes = codes_out;
+  a.sf = sf_out;
+  r.in_codes = codes;
+  r.in_sf = sf;
+  r.g_old = g_old;
+  r.g_new = g_new;
+  r.nseg_old = segs.n;
+  for (int i = 0; i <= kMaxSeg; ++i)
+    r.old_begin[i] = static_cast<int32_t>(i <= segs.n ? segs.begin[i] : segs.begin[segs.n]);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid_for(a.items));
+  cfg.blockDim = dim3(kThreads);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, requant_kernel, r);
+}
 
 cudaError_t launch_quantize(const void* x, int dtype, int64_t M, int64_t K, int64_t ld,
                             const RowSegments& segs, const float* g_in, void* ws,

@@ -43,7 +43,7 @@ EXPORTED = (
     "nvfp4_status_string", "nvfp4_last_cuda_error", "nvfp4_sf_bytes",
     "nvfp4_quantize_workspace_bytes", "nvfp4_quantize", "nvfp4_quantize_segments",
     "nvfp4_gemm_workspace_bytes", "nvfp4_gemm", "nvfp4_fused_proj", "nvfp4_check",
-    "nvfp4_quantize_noalloc", "nvfp4_linear",
+    "nvfp4_quantize_noalloc", "nvfp4_linear", "nvfp4_requantize_segments",
 )
 
 
@@ -110,6 +110,9 @@ def _lib():
         lib.nvfp4_linear.argtypes = [c.c_void_p, c.c_int, c.c_int64, c.c_int64, c.c_int64, c.c_void_p,
                                      c.c_void_p, c.c_void_p, c.c_void_p, c.POINTER(_Operand), c.c_void_p,
                                      c.POINTER(_Segment), c.c_int, c.c_void_p, c.c_size_t, c.c_void_p]
+        lib.nvfp4_requantize_segments.restype = c.c_int
+        lib.nvfp4_requantize_segments.argtypes = [c.POINTER(_Operand), c.c_void_p, c.c_int, c.c_void_p, c.c_void_p,
+                                                  c.c_void_p, c.c_void_p, c.c_void_p, c.c_void_p]
         lib.nvfp4_check.restype = c.c_int
         lib.nvfp4_check.argtypes = [c.c_void_p]
         _LIB = lib
@@ -289,6 +292,25 @@ def nvfp4_linear(x: torch.Tensor, W: Operand, seg_global_scale: torch.Tensor, se
           _ptr(g_a), ctypes.byref(w), _ptr(seg_global_scale), arr, n, _ptr(workspace), ws_bytes,
           _stream(stream))
     return Operand(a_codes, a_sf, M, K), g_a
+
+
+def nvfp4_requantize_segments(W: Operand, row_bounds: Sequence[int], g_old: torch.Tensor,
+                              g_new: Optional[torch.Tensor] = None, *, codes=None, sf=None, g_out=None,
+                              in_place: bool = False, stream=None):
+    """Re-encode W (modules = row ranges with scales g_old) under one common
+    global scale (g_new, or the largest of g_old) -> (Operand, g_out[nseg])."""
+    nseg = len(row_bounds) - 1
+    dev = W.codes.device
+    if in_place:
+        codes, sf = W.codes, W.sf
+    codes = torch.empty_like(W.codes) if codes is None else codes
+    sf = torch.empty_like(W.sf) if sf is None else sf
+    g_out = torch.empty(nseg, dtype=torch.float32, device=dev) if g_out is None else g_out
+    bounds = (ctypes.c_int64 * (nseg + 1))(*[int(b) for b in row_bounds])
+    w = W._c()
+    _call("nvfp4_requantize_segments", ctypes.byref(w), bounds, nseg, _ptr(g_old), _ptr(g_new), _ptr(codes),
+          _ptr(sf), _ptr(g_out), _stream(stream))
+    return Operand(codes, sf, W.rows, W.K), g_out
 
 
 def nvfp4_check(stream=None):

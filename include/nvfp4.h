@@ -237,6 +237,32 @@ int nvfp4_linear(const void* x, int x_dtype, int64_t M, int64_t K, int64_t ld_x,
                  size_t workspace_bytes, void* stream);
 
 /*
+ * nvfp4_requantize_segments — checkpoint-side harmonisation of fused modules'
+ * global scales ("Methodology in Plain English": the fused modules' scales
+ * are made to agree on the checkpoint side, so that a kernel that applies one
+ * global scale to the fused GEMM is correct).  Every element of the NVFP4
+ * operand W is dequantised with its module's scale (x = e2m1 * S * g_old[s],
+ * rounded once to FP32) and quantised again, exactly as nvfp4_quantize does,
+ * with one common scale.
+ *   W           host struct, device buffers: the operand [N, K] to re-encode.
+ *   row_bounds  host, nseg + 1 increasing row indices (as nvfp4_quantize_segments).
+ *   g_old       device float [nseg]: the modules' current global scales.
+ *   g_new       device float, the common scale, or NULL for the largest of
+ *               g_old, which is the scale of the fused (concatenated) weight
+ *               and the only choice that clips no block (a smaller common
+ *               scale makes the larger modules' top block scales saturate).
+ *   codes_out, sf_out  device, [N, K/2] and nvfp4_sf_bytes(N, K) bytes, 16-byte
+ *               aligned; either exactly W's buffers (in place) or disjoint
+ *               from them.
+ *   g_out       device float [nseg], receives the common scale for every
+ *               module, so (codes_out, sf_out, g_out) is again an operand with
+ *               its per-segment scale table.
+ */
+int nvfp4_requantize_segments(const nvfp4_operand* W, const int64_t* row_bounds, int nseg,
+                              const float* g_old, const float* g_new, uint8_t* codes_out,
+                              uint8_t* sf_out, float* g_out, void* stream);
+
+/*
  * nvfp4_check — synchronise `stream`, then report (and clear) the library's
  * device error word: NVFP4_ERR_DEVICE_TIMEOUT if a bounded wait inside a
  * kernel gave up since the last check, NVFP4_ERR_CUDA on a CUDA error.

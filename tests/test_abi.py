@@ -150,3 +150,23 @@ def test_linear_rejects_bad_arguments(lib):
     assert _lin(lib, g_in=0, ws=0x800000 + 1024, wsb=4096) == 1
     assert _lin(lib, segs=[nv._Segment(0, 100, 0, 0, 0x900000, 256, None, None)]) == 1   # segments
     assert _lin(lib, M=0) == 0                                # empty: nothing enqueued
+
+
+def test_requantize_rejects_bad_arguments(lib):
+    v = ctypes.c_void_p
+    W = _op(codes=0x400000, sf=0x800000, rows=256, K=256)
+
+    def call(bounds=(0, 100, 256), g_old=FAKE, codes=0x900000, sf=0xA00000, g_out=FAKE, W=W):
+        b = (ctypes.c_int64 * len(bounds))(*bounds)
+        return lib.nvfp4_requantize_segments(ctypes.byref(W), b, len(bounds) - 1, v(g_old) if g_old else None, None,
+                                             v(codes) if codes else None, v(sf) if sf else None,
+                                             v(g_out) if g_out else None, None)
+    assert call(bounds=(0, 100, 200)) == 1            # bounds must end at W->rows
+    assert call(bounds=(0, 120, 100, 256)) == 1       # increasing
+    assert call(g_old=0) == 1
+    assert call(codes=0) == 1
+    assert call(g_out=FAKE + 2) == 3
+    assert call(codes=0x900000 + 8) == 3
+    assert call(codes=0x400000 + 64) == 1             # partial overlap with W's codes
+    assert call(sf=0x800000 + 16) == 1                # partial overlap with W's scales
+    assert call(W=_op(codes=0x400000, sf=0x800000, rows=256, K=48)) == 2

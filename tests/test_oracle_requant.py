@@ -103,3 +103,37 @@ def test_harmonising_to_a_smaller_scale_clips_the_top_block():
     y_hat = o.dequantize(c, s, g)[r, 16 * b:16 * b + 16]
     assert np.abs(y_hat).max() == 6 * 448 * np.float64(gc)  # the largest value clips to 6 * 448 * gc
     assert np.abs(x_hat).max() > 1.9 * np.abs(y_hat).max()
+
+
+def test_harmonised_weights_match_the_scale_table_accuracy():
+    """The comparison NEXT-1 asks for, on a GDN-like fused weight whose gate
+    segments have a larger amax (x2.75, the pages' mismatch ratio): the fused
+    GEMM with per-module scales (the table), with one common scale after
+    checkpoint-side re-encoding, and with one common scale and no re-encoding
+    (the mismatch).  Errors against the product with the unquantised weights,
+    the activation quantised the same way in all three."""
+    rng = np.random.default_rng(17)
+    K, M = 512, 64
+    x = rng.standard_normal((M, K)).astype(np.float32)
+    widths, gains = [128, 128, 32, 32], [1.0, 1.0, 2.75, 2.75]
+    segs = [(0.02 * gain * rng.standard_normal((n, K))).astype(np.float32) for n, gain in zip(widths, gains)]
+    xq = o.quantize(x)
+    x_hat = o.dequantize(*xq)
+    qs = [o.quantize(s) for s in segs]
+    g = [q[2] for q in qs]
+    g_fused = max(g)
+    err = {"table": [], "harmonised": [], "mismatch": []}
+    for (c, s, gs), w in zip(qs, segs):
+        ref = x_hat @ w.astype(np.float64).T
+        c2, s2, g2 = o.requantize(c, s, gs, g_fused)
+        y = {"table": x_hat @ o.dequantize(c, s, gs).T,
+             "harmonised": x_hat @ o.dequantize(c2, s2, g2).T,
+             "mismatch": x_hat @ o.dequantize(c, s, o.common_global_scale(g)).T}
+        for k in err:
+            err[k].append(np.linalg.norm(y[k] - ref) / np.linalg.norm(ref))
+    for i in range(len(widths)):
+        # re-encoding costs little accuracy next to the exact per-module scales
+        assert err["harmonised"][i] <= 1.6 * err["table"][i] + 1e-3
+        assert err["table"][i] < 0.2
+    # the mismatch scales the larger-amax segments by g_c / g_s = 1 / 2.75
+    assert min(err["mismatch"][2:]) > 0.5 and max(err["mismatch"][:2]) < 0.2
