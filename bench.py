@@ -493,9 +493,161 @@ def cpu_baseline(name, target_s=12.0, steps=None):
             "host_cpus": os.cpu_count()}
 
 
+def run_requant(args):
+    """Checkpoint-side harmonisation of the GDN in-projection weight
+    [12352, 5120] (six modules): nvfp4_requantize_segments under the fused
+    tensor's scale, one call per step; HBM-bound (reads and writes codes and
+    scale bytes)."""
+    import torch
+    from bit_quantized_linear_nvfp4_b200 import nvfp4 as nv
+    from bit_quantized_linear_nvfp4_b200 import workloads as wl
+    world, rank, local = dist_env()
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    dist = dist_init(world)
+    peaks, peak_src = load_peaks()
+    w = wl.GDN
+    segs = wl.make_w_segments(w)
+    bounds = np.concatenate([[0], np.cumsum([sg.width for sg in w.segments])]).astype(np.int64)
+    N, K = int(bounds[-1]), w.K
+    wdev = torch.from_numpy(np.concatenate(segs)).to(device).to(torch.bfloat16)
+    sets = []
+    for _ in range(ROTATE):
+        W, gw = nv.nvfp4_quantize_segments(wdev, bounds)
+        out = (torch.empty_like(W.codes), torch.empty_like(W.sf), torch.empty_like(gw))
+        sets.append((W, gw, out))
+    del wdev
+    stream = torch.cuda.current_stream()
+
+    def call(i):
+        W, gw, (c, sf, g) = sets[i % ROTATE]
+        nv.nvfp4_requantize_segments(W, bounds, gw, codes=c, sf=sf, g_out=g)
+
+    for i in range(ROTATE):
+        call(i)
+    torch.cuda.synchronize()
+    graphs = []
+    for i in range(ROTATE):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            call(i)
+        graphs.append(g)
+    Kst, Wm = args.steps, args.warmup
+    for i in range(Wm):
+        graphs[i % ROTATE].replay()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    dist_barrier(dist)
+    torch.cuda.synchronize()
+    t0.record(stream)
+    for i in range(Kst):
+        graphs[i % ROTATE].replay()
+    t1.record(stream)
+    torch.cuda.synchronize()
+    dist_barrier(dist)
+    clk = clocks.stop()
+    ms = dist_max(dist, t0.elapsed_time(t1), device) / Kst
+    nv.nvfp4_check()
+    per_set = N * K // 2 + nv.nvfp4_sf_bytes(N, K)
+    bytes_step = 2 * per_set
+    hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    ach = bytes_step / (ms * 1e-3) / 1e9
+    # end to end: the checkpoint's codes and scales in from pinned host memory, the result out
+    W0, gw0, (c0, sf0, g0) = sets[0]
+    h_codes, h_sf = W0.codes.cpu().pin_memory(), W0.sf.cpu().pin_memory()
+    o_codes, o_sf = torch.empty_like(h_codes).pin_memory(), torch.empty_like(h_sf).pin_memory()
+
+    def e2e_one():
+        W0.codes.copy_(h_codes, non_blocking=True)
+        W0.sf.copy_(h_sf, non_blocking=True)
+        graphs[0].replay()
+        o_codes.copy_(c0, non_blocking=True)
+        o_sf.copy_(sf0, non_blocking=True)
+
+    for _ in range(Wm):
+        e2e_one()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(Kst):
+        e2e_one()
+    b.record(stream)
+    torch.cuda.synchronize()
+    ms_e2e = a.elapsed_time(b) / Kst
+    line = {
+        "metric": METRIC, "value": bytes_step * world / (ms * 1e-3) / 1e9, "unit": "GB/s", "n_gpus": world,
+        "steps": Kst, "warmup": Wm, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "nvfp4 (FP32 arithmetic)", "data": "synthetic (N(0,0.02) weights, six modules)",
+        "config": {"workload": "requant_gdn_weight_12352x5120", "N": N, "K": K, "segments": len(w.segments),
+                   "parallelism": "replicas" if world > 1 else "single",
+                   "l2": f"{ROTATE} rotating weight copies, working set above the 126 MB L2"},
+        "roofline": {"bound": "hbm", "achieved": ach, "peak": hbm, "unit": "GB/s", "frac": ach / hbm,
+                     "traffic": TRAFFIC_BYTES.get("requant"), "peak_source": f"{peak_src} copy bandwidth",
+                     "kernel": "nvfp4 requantize", "ms_per_launch": ms},
+        "clocks": clk,
+        "e2e": {"value": bytes_step / (ms_e2e * 1e-3) / 1e9, "unit": "GB/s", "h2d_bytes_per_step": per_set,
+                "d2h_bytes_per_step": per_set, "ms_per_step": ms_e2e},
+        "gpu_launches": Kst,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        from oracle import nvfp4_oracle as o
+        rows = 512
+        wq = [o.quantize(sg_w) for sg_w in segs]
+        c_all = np.concatenate([c for c, _, _ in wq])[:rows]
+        s_all = np.concatenate([sf for _, sf, _ in wq])[:rows]
+        g_rows = np.repeat(np.array([g for _, _, g in wq], np.float32), [sg.width for sg in w.segments])[:rows]
+        g_c = max(g for _, _, g in wq)
+        t = time.perf_counter()
+        n = 0
+        while time.perf_counter() - t < args.cpu_seconds / 2 or n == 0:
+            o.requantize(c_all, s_all, g_rows, g_c)
+            n += 1
+        per = (time.perf_counter() - t) / n
+        line["cpu_baseline"] = {"value": 2 * rows * K * 0.5625 / per / 1e9, "unit": "GB/s", "cores": _blas_threads(),
+                                "kind": "oracle", "sample": f"{rows} rows x {K} per pass ({n} passes)",
+                                "host_cpus": os.cpu_count()}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    for g in graphs:
+        del g
+    if dist is not None:
+        dist.destroy_process_group()
+
+
 def run_reference(args):
     world, rank, _ = dist_env()
     if rank != 0:
+        return
+    if args.workload == "requant":
+        from bit_quantized_linear_nvfp4_b200 import workloads as wl
+        from oracle import nvfp4_oracle as o
+        w = wl.GDN
+        rows = 256
+        wq = [o.quantize(sg) for sg in wl.make_w_segments(w)]
+        c_all = np.concatenate([c for c, _, _ in wq])[:rows]
+        s_all = np.concatenate([sf for _, sf, _ in wq])[:rows]
+        g_rows = np.repeat(np.array([g for _, _, g in wq], np.float32), [sg.width for sg in w.segments])[:rows]
+        g_c = max(g for _, _, g in wq)
+        for _ in range(args.warmup):
+            o.requantize(c_all, s_all, g_rows, g_c)
+        t = time.perf_counter()
+        for _ in range(args.steps):
+            o.requantize(c_all, s_all, g_rows, g_c)
+        per = (time.perf_counter() - t) / args.steps
+        val = 2 * rows * w.K * 0.5625 / per / 1e9
+        sample = f"{rows} rows x {w.K} of the GDN weight per step (oracle requantize)"
+        print(json.dumps({"impl": "reference", "metric": METRIC, "value": val, "unit": "GB/s", "n_gpus": world,
+                          "steps": args.steps, "warmup": args.warmup, "ms_per_step": per * 1e3,
+                          "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+                          "dtype": "f32 (oracle)", "data": "synthetic",
+                          "config": {"workload": "requant_gdn_weight_12352x5120", "N": 12352, "K": w.K},
+                          "cpu_baseline": {"value": val, "unit": "GB/s", "cores": _blas_threads(), "kind": "oracle",
+                                           "sample": sample},
+                          "e2e": {"value": val, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}),
+              flush=True)
         return
     w, x, wq, g_a, extra = _prepare_oracle(args.workload)
     K = x.shape[1]
@@ -529,7 +681,7 @@ def main():
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--workload", default="oproj",
-                    choices=["oproj", "mlp", "gdn", "tiny", "decode1", "decode8", "decode64", "quant"])
+                    choices=["oproj", "mlp", "gdn", "tiny", "decode1", "decode8", "decode64", "quant", "requant"])
     ap.add_argument("--impl", default="product", choices=["product", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
@@ -540,6 +692,8 @@ def main():
         args.warmup = 3
     if args.impl == "reference":
         run_reference(args)
+    elif args.workload == "requant":
+        run_requant(args)
     else:
         run_product(args)
 

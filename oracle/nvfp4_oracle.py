@@ -312,6 +312,31 @@ def requantize(codes: np.ndarray, sf: np.ndarray, g_rows, g_new):
     return quantize(x_hat, np.float32(g_new))
 
 
+def kv_fp8_quantize(x: np.ndarray, scale) -> np.ndarray:
+    """FP8 (E4M3) KV-cache codec with a calibrated static per-tensor scale
+    (Paper summary page (ai.info), "Main Findings", KV-cache bullet: an FP8
+    KV cache whose scales are calibrated, not left at 1.0).  Reading, in FP32:
+    inv = 1 / scale (once), y = x * inv, code = sign(y) | E4M3_rn_satfinite(|y|),
+    the sign of zero kept; scale <= 0 (or not finite) gives all-zero codes."""
+    x = np.asarray(x, dtype=np.float32)
+    s = np.float32(scale)
+    if not (np.isfinite(s) and s > 0):
+        return np.zeros(x.shape, np.uint8)
+    inv = np.float32(1) / s
+    with np.errstate(over="ignore"):
+        y = (x * inv).astype(np.float32)
+    mag = e4m3_encode_nonneg(np.abs(y))
+    return (mag | (np.signbit(y).astype(np.uint8) << 7)).astype(np.uint8)
+
+
+def kv_fp8_dequantize(codes: np.ndarray, scale, out_dtype: str = "bf16") -> np.ndarray:
+    """x_hat = e4m3(code) * scale rounded to FP32, then to BF16 when the output
+    is BF16 (returned as float64 holding the rounded values)."""
+    v = e4m3_decode(codes).astype(np.float32)
+    y = (v * np.float32(scale)).astype(np.float32).astype(np.float64)
+    return bf16_round(y) if out_dtype == "bf16" else y
+
+
 def bf16_round(y) -> np.ndarray:
     """Round FP64 values to BF16 (8 significant bits, nearest, ties to even);
     returned as FP64.  y = m * 2^e with 0.5 <= |m| < 1, so y / 2^(e-8) has its
