@@ -617,9 +617,148 @@ def run_requant(args):
         dist.destroy_process_group()
 
 
+def run_kvfp8(args):
+    """FP8 (E4M3) KV-cache codec: quantise the K and V of a 32768-token prefill
+    chunk (8 KV heads x 128, BF16) under calibrated static scales, two calls
+    per step; HBM-bound (2 B read + 1 B written per element)."""
+    import torch
+    from bit_quantized_linear_nvfp4_b200 import nvfp4 as nv
+    from bit_quantized_linear_nvfp4_b200 import workloads as wl
+    world, rank, local = dist_env()
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    dist = dist_init(world)
+    peaks, peak_src = load_peaks()
+    T, C = 32768, 1024
+    rng = np.random.default_rng(6)
+    kv_np = [wl.round_to_bf16(rng.standard_normal((T, C)).astype(np.float32)) for _ in range(2)]
+    scales = [np.float32(np.abs(a).max() / 448) for a in kv_np]
+    sets = []
+    for r in range(ROTATE):
+        srcs = [torch.from_numpy(a).to(device).to(torch.bfloat16) for a in kv_np]
+        outs = [torch.empty((T, C), dtype=torch.uint8, device=device) for _ in range(2)]
+        sc = [torch.tensor([v], dtype=torch.float32, device=device) for v in scales]
+        sets.append((srcs, outs, sc))
+    stream = torch.cuda.current_stream()
+
+    def call(i):
+        srcs, outs, sc = sets[i % ROTATE]
+        for x, o_, s_ in zip(srcs, outs, sc):
+            nv.nvfp4_kv_fp8_quantize(x, s_, out=o_)
+
+    for i in range(ROTATE):
+        call(i)
+    torch.cuda.synchronize()
+    graphs = []
+    for i in range(ROTATE):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            call(i)
+        graphs.append(g)
+    Kst, Wm = args.steps, args.warmup
+    for i in range(Wm):
+        graphs[i % ROTATE].replay()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    dist_barrier(dist)
+    torch.cuda.synchronize()
+    t0.record(stream)
+    for i in range(Kst):
+        graphs[i % ROTATE].replay()
+    t1.record(stream)
+    torch.cuda.synchronize()
+    dist_barrier(dist)
+    clk = clocks.stop()
+    ms = dist_max(dist, t0.elapsed_time(t1), device) / Kst
+    nv.nvfp4_check()
+    bytes_step = 2 * T * C * 3
+    hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    ach = bytes_step / (ms * 1e-3) / 1e9
+    srcs0, outs0, _ = sets[0]
+    h_in = [x.cpu().pin_memory() for x in srcs0]
+    h_out = [torch.empty((T, C), dtype=torch.uint8).pin_memory() for _ in range(2)]
+
+    def e2e_one():
+        for d, h in zip(srcs0, h_in):
+            d.copy_(h, non_blocking=True)
+        graphs[0].replay()
+        for h, d in zip(h_out, outs0):
+            h.copy_(d, non_blocking=True)
+
+    for _ in range(Wm):
+        e2e_one()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(Kst):
+        e2e_one()
+    b.record(stream)
+    torch.cuda.synchronize()
+    ms_e2e = a.elapsed_time(b) / Kst
+    line = {
+        "metric": METRIC, "value": bytes_step * world / (ms * 1e-3) / 1e9, "unit": "GB/s", "n_gpus": world,
+        "steps": Kst, "warmup": Wm, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "fp8 e4m3 (FP32 arithmetic)", "data": "synthetic (N(0,1) BF16 K and V)",
+        "config": {"workload": "kv_fp8_encode_2x32768x1024", "tokens": T, "cols": C, "tensors": 2,
+                   "parallelism": "replicas" if world > 1 else "single",
+                   "l2": f"{ROTATE} rotating K/V sets, working set above the 126 MB L2"},
+        "roofline": {"bound": "hbm", "achieved": ach, "peak": hbm, "unit": "GB/s", "frac": ach / hbm,
+                     "traffic": TRAFFIC_BYTES.get("kvfp8"), "peak_source": f"{peak_src} copy bandwidth",
+                     "kernel": "nvfp4 kv fp8 encode", "ms_per_launch": ms / 2},
+        "clocks": clk,
+        "e2e": {"value": bytes_step / (ms_e2e * 1e-3) / 1e9, "unit": "GB/s", "h2d_bytes_per_step": 2 * T * C * 2,
+                "d2h_bytes_per_step": 2 * T * C, "ms_per_step": ms_e2e},
+        "gpu_launches": 2 * Kst,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        from oracle import nvfp4_oracle as o
+        rows = 2048
+        t = time.perf_counter()
+        n = 0
+        while time.perf_counter() - t < args.cpu_seconds / 2 or n == 0:
+            o.kv_fp8_quantize(kv_np[0][:rows], scales[0])
+            n += 1
+        per = (time.perf_counter() - t) / n
+        line["cpu_baseline"] = {"value": rows * C * 3 / per / 1e9, "unit": "GB/s", "cores": _blas_threads(),
+                                "kind": "oracle", "sample": f"{rows} rows x {C} per pass ({n} passes)",
+                                "host_cpus": os.cpu_count()}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    for g in graphs:
+        del g
+    if dist is not None:
+        dist.destroy_process_group()
+
+
 def run_reference(args):
     world, rank, _ = dist_env()
     if rank != 0:
+        return
+    if args.workload == "kvfp8":
+        from oracle import nvfp4_oracle as o
+        rng = np.random.default_rng(6)
+        rows, C = 2048, 1024
+        x = rng.standard_normal((rows, C)).astype(np.float32)
+        s = np.float32(np.abs(x).max() / 448)
+        for _ in range(args.warmup):
+            o.kv_fp8_quantize(x, s)
+        t = time.perf_counter()
+        for _ in range(args.steps):
+            o.kv_fp8_quantize(x, s)
+        per = (time.perf_counter() - t) / args.steps
+        val = rows * C * 3 / per / 1e9
+        print(json.dumps({"impl": "reference", "metric": METRIC, "value": val, "unit": "GB/s", "n_gpus": world,
+                          "steps": args.steps, "warmup": args.warmup, "ms_per_step": per * 1e3,
+                          "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+                          "dtype": "f32 (oracle)", "data": "synthetic",
+                          "config": {"workload": "kv_fp8_encode_2x32768x1024", "tokens": 32768, "cols": C},
+                          "cpu_baseline": {"value": val, "unit": "GB/s", "cores": _blas_threads(), "kind": "oracle",
+                                           "sample": f"{rows} rows x {C} per step (oracle KV encode)"},
+                          "e2e": {"value": val, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}),
+              flush=True)
         return
     if args.workload == "requant":
         from bit_quantized_linear_nvfp4_b200 import workloads as wl
@@ -681,7 +820,8 @@ def main():
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--workload", default="oproj",
-                    choices=["oproj", "mlp", "gdn", "tiny", "decode1", "decode8", "decode64", "quant", "requant"])
+                    choices=["oproj", "mlp", "gdn", "tiny", "decode1", "decode8", "decode64", "quant", "requant",
+                             "kvfp8"])
     ap.add_argument("--impl", default="product", choices=["product", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
@@ -694,6 +834,8 @@ def main():
         run_reference(args)
     elif args.workload == "requant":
         run_requant(args)
+    elif args.workload == "kvfp8":
+        run_kvfp8(args)
     else:
         run_product(args)
 

@@ -8,7 +8,8 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libnvfp4.so")
-SOURCES = ["libnvfp4.cu", "quantize.cu", "gemm.cu", "gemm_decode.cu", "api.cu", "noalloc.cu", "ptx.cuh", "internal.h"]
+SOURCES = ["libnvfp4.cu", "quantize.cu", "gemm.cu", "gemm_decode.cu", "api.cu", "noalloc.cu", "kv_fp8.cu", "ptx.cuh",
+           "internal.h"]
 
 
 def nvcc_path() -> str:

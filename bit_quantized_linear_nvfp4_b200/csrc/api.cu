@@ -301,6 +301,44 @@ int nvfp4_requantize_segments(const nvfp4_operand* W, const int64_t* row_bounds,
   return NVFP4_OK;
 }
 
+int nvfp4_kv_fp8_quantize(const void* x, int x_dtype, int64_t rows, int64_t cols, int64_t ld_x,
+                          const float* scale, uint8_t* out, int64_t ld_out, void* stream) {
+  if (x_dtype != NVFP4_DTYPE_BF16 && x_dtype != NVFP4_DTYPE_F32) return NVFP4_ERR_INVALID_ARG;
+  if (rows < 0 || cols < 0 || scale == nullptr) return NVFP4_ERR_INVALID_ARG;
+  if (cols % 8 != 0) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+  if (rows == 0 || cols == 0) return NVFP4_OK;
+  if (x == nullptr || out == nullptr || ld_x < cols || ld_out < cols) return NVFP4_ERR_INVALID_ARG;
+  const int esz = x_dtype == NVFP4_DTYPE_BF16 ? 2 : 4;
+  if (!aligned16(x) || (ld_x * esz) % 16 != 0) return NVFP4_ERR_MISALIGNED;
+  if ((reinterpret_cast<uintptr_t>(out) & 7u) != 0 || ld_out % 8 != 0 || (reinterpret_cast<uintptr_t>(scale) & 3u) != 0)
+    return NVFP4_ERR_MISALIGNED;
+  int st = check_device();
+  if (st != NVFP4_OK) return st;
+  cudaError_t e = nvfp4::launch_kv_fp8(true, x_dtype, x, ld_x, out, ld_out, rows, cols, scale,
+                                       static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e);
+  return NVFP4_OK;
+}
+
+int nvfp4_kv_fp8_dequantize(const uint8_t* codes, int64_t rows, int64_t cols, int64_t ld_codes,
+                            const float* scale, void* out, int out_dtype, int64_t ld_out, void* stream) {
+  if (out_dtype != NVFP4_DTYPE_BF16 && out_dtype != NVFP4_DTYPE_F32) return NVFP4_ERR_INVALID_ARG;
+  if (rows < 0 || cols < 0 || scale == nullptr) return NVFP4_ERR_INVALID_ARG;
+  if (cols % 8 != 0) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+  if (rows == 0 || cols == 0) return NVFP4_OK;
+  if (codes == nullptr || out == nullptr || ld_codes < cols || ld_out < cols) return NVFP4_ERR_INVALID_ARG;
+  const int esz = out_dtype == NVFP4_DTYPE_BF16 ? 2 : 4;
+  if ((reinterpret_cast<uintptr_t>(codes) & 7u) != 0 || ld_codes % 8 != 0) return NVFP4_ERR_MISALIGNED;
+  if (!aligned16(out) || (ld_out * esz) % 16 != 0 || (reinterpret_cast<uintptr_t>(scale) & 3u) != 0)
+    return NVFP4_ERR_MISALIGNED;
+  int st = check_device();
+  if (st != NVFP4_OK) return st;
+  cudaError_t e = nvfp4::launch_kv_fp8(false, out_dtype, codes, ld_codes, out, ld_out, rows, cols, scale,
+                                       static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e);
+  return NVFP4_OK;
+}
+
 int nvfp4_gemm(const nvfp4_operand* A, const float* g_a, const nvfp4_operand* W, const float* g_w,
                void* out, int out_dtype, int64_t ld_out, void* workspace, size_t workspace_bytes,
                void* stream) {

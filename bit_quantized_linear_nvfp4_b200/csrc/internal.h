@@ -45,6 +45,12 @@ cudaError_t launch_requantize(const uint8_t* codes, const uint8_t* sf, int64_t N
                               const RowSegments& segs, const float* g_old, const float* g_new,
                               uint8_t* codes_out, uint8_t* sf_out, float* g_out, cudaStream_t stream);
 
+// FP8 (E4M3) KV codec with a static scale: encode x [rows, cols] (BF16/F32,
+// row stride ld_src elements) into codes (row stride ld_dst bytes), or decode
+// codes (row stride ld_src bytes) into BF16/F32 (row stride ld_dst elements).
+cudaError_t launch_kv_fp8(bool encode, int dtype, const void* src, int64_t ld_src, void* dst, int64_t ld_dst,
+                          int64_t rows, int64_t cols, const float* scale, cudaStream_t stream);
+
 // GEMM epilogue description handed to the kernels.
 struct EpiSegment {
   int64_t n_begin, n_end;

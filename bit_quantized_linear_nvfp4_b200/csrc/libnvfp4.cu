@@ -5,3 +5,4 @@
 #include "gemm_decode.cu"
 #include "api.cu"
 #include "noalloc.cu"
+#include "kv_fp8.cu"

@@ -577,33 +577,52 @@ __global__ void __launch_bounds__(kThreads, 1) requant_kernel(const __grid_const
   __syncthreads();
   if (blockIdx.x == 0 && threadIdx.x < r.nseg_old) a.g_out[threadIdx.x] = g_sh[0];
   const int32_t KA = (a.K + 63) / 64;
+  constexpr int U = 8;  // chunks in flight per warp (9 bytes per lane each)
   int64_t lo, hi;
   block_range(a.items, lo, hi);
-  for (int64_t i = lo + warp; i < hi; i += kWarps) {
-    int32_t row, col;
-    chunk_pos(a, i, row, col);
-    col += lane * 16;
-    const bool have = col < a.K;
-    Blk<NVFP4_DTYPE_F32> b;
-    if (have) {
-      const uint2 c = *reinterpret_cast<const uint2*>(r.in_codes + static_cast<int64_t>(row) * (a.K / 2) + col / 2);
-      const int32_t j = col / 16;
-      const uint32_t sfb = r.in_sf[(static_cast<int64_t>(row >> 7) * KA + (j >> 2)) * 512 + (row & 31) * 16 +
-                                   ((row >> 5) & 3) * 4 + (j & 3)];
-      int s = 0;
+  for (int64_t base = lo; base < hi; base += kWarps * U) {
+    uint2 c[U];
+    uint32_t sfb[U];
+    int32_t rows[U], cols[U];
+    bool inr[U], have[U];
 #pragma unroll
-      for (int k = 1; k < kMaxSeg; ++k)
-        if (k < r.nseg_old && row >= r.old_begin[k]) s = k;
-      const float S = e4m3_value(sfb), g = g_old_sh[s];
-#pragma unroll
-      for (int e = 0; e < 16; ++e) {
-        const uint32_t word = e < 8 ? c.x : c.y;
-        const uint32_t code = (word >> (4 * (e & 7))) & 15u;
-        b.w[e] = __float_as_uint((e2m1_value(code) * S) * g);  // e2m1 * S exact, one rounding
+    for (int u = 0; u < U; ++u) {
+      const int64_t i = base + u * kWarps + warp;
+      inr[u] = i < hi;
+      have[u] = false;
+      rows[u] = cols[u] = 0;
+      if (inr[u]) {
+        chunk_pos(a, i, rows[u], cols[u]);
+        cols[u] += lane * 16;
+        have[u] = cols[u] < a.K;
+        if (have[u]) {
+          const int32_t row = rows[u], col = cols[u], j = col / 16;
+          c[u] = *reinterpret_cast<const uint2*>(r.in_codes + static_cast<int64_t>(row) * (a.K / 2) + col / 2);
+          sfb[u] = r.in_sf[(static_cast<int64_t>(row >> 7) * KA + (j >> 2)) * 512 + (row & 31) * 16 +
+                           ((row >> 5) & 3) * 4 + (j & 3)];
+        }
       }
     }
-    __syncwarp();  // in place: every lane has read before any lane writes
-    quantize_block<NVFP4_DTYPE_F32>(a, g_sh, b, have, row, col);
+    __syncwarp();  // in place: every lane has read all U chunks before any lane writes
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      if (!inr[u]) continue;  // uniform across the warp
+      Blk<NVFP4_DTYPE_F32> b;
+      if (have[u]) {
+        int s = 0;
+#pragma unroll
+        for (int k = 1; k < kMaxSeg; ++k)
+          if (k < r.nseg_old && rows[u] >= r.old_begin[k]) s = k;
+        const float S = e4m3_value(sfb[u]), g = g_old_sh[s];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          const uint32_t word = e < 8 ? c[u].x : c[u].y;
+          const uint32_t code = (word >> (4 * (e & 7))) & 15u;
+          b.w[e] = __float_as_uint((e2m1_value(code) * S) * g);  // e2m1 * S exact, one rounding
+        }
+      }
+      quantize_block<NVFP4_DTYPE_F32>(a, g_sh, b, have[u], rows[u], cols[u]);
+    }
   }
   zero_padding_rows(a);
 }

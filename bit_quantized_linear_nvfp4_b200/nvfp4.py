@@ -44,6 +44,7 @@ EXPORTED = (
     "nvfp4_quantize_workspace_bytes", "nvfp4_quantize", "nvfp4_quantize_segments",
     "nvfp4_gemm_workspace_bytes", "nvfp4_gemm", "nvfp4_fused_proj", "nvfp4_check",
     "nvfp4_quantize_noalloc", "nvfp4_linear", "nvfp4_requantize_segments",
+    "nvfp4_kv_fp8_quantize", "nvfp4_kv_fp8_dequantize",
 )
 
 
@@ -113,6 +114,12 @@ def _lib():
         lib.nvfp4_requantize_segments.restype = c.c_int
         lib.nvfp4_requantize_segments.argtypes = [c.POINTER(_Operand), c.c_void_p, c.c_int, c.c_void_p, c.c_void_p,
                                                   c.c_void_p, c.c_void_p, c.c_void_p, c.c_void_p]
+        lib.nvfp4_kv_fp8_quantize.restype = c.c_int
+        lib.nvfp4_kv_fp8_quantize.argtypes = [c.c_void_p, c.c_int, c.c_int64, c.c_int64, c.c_int64, c.c_void_p,
+                                              c.c_void_p, c.c_int64, c.c_void_p]
+        lib.nvfp4_kv_fp8_dequantize.restype = c.c_int
+        lib.nvfp4_kv_fp8_dequantize.argtypes = [c.c_void_p, c.c_int64, c.c_int64, c.c_int64, c.c_void_p,
+                                                c.c_void_p, c.c_int, c.c_int64, c.c_void_p]
         lib.nvfp4_check.restype = c.c_int
         lib.nvfp4_check.argtypes = [c.c_void_p]
         _LIB = lib
@@ -311,6 +318,29 @@ def nvfp4_requantize_segments(W: Operand, row_bounds: Sequence[int], g_old: torc
     _call("nvfp4_requantize_segments", ctypes.byref(w), bounds, nseg, _ptr(g_old), _ptr(g_new), _ptr(codes),
           _ptr(sf), _ptr(g_out), _stream(stream))
     return Operand(codes, sf, W.rows, W.K), g_out
+
+
+def nvfp4_kv_fp8_quantize(x: torch.Tensor, scale: torch.Tensor, *, out=None, stream=None) -> torch.Tensor:
+    """FP8 (E4M3) codes of x[rows, cols] (BF16/F32) under the static scale (a
+    device float tensor); returns uint8 codes [rows, cols]."""
+    _check_2d(x)
+    rows, cols = x.shape
+    out = torch.empty((rows, cols), dtype=torch.uint8, device=x.device) if out is None else out
+    _call("nvfp4_kv_fp8_quantize", _ptr(x), _dtype_code(x), rows, cols, x.stride(0), _ptr(scale), _ptr(out),
+          out.stride(0), _stream(stream))
+    return out
+
+
+def nvfp4_kv_fp8_dequantize(codes: torch.Tensor, scale: torch.Tensor, out_dtype=torch.bfloat16, *, out=None,
+                            stream=None) -> torch.Tensor:
+    """Decode FP8 (E4M3) codes [rows, cols] with the static scale."""
+    _check_2d(codes)
+    rows, cols = codes.shape
+    out = torch.empty((rows, cols), dtype=out_dtype, device=codes.device) if out is None else out
+    code = DTYPE_BF16 if out.dtype == torch.bfloat16 else DTYPE_F32
+    _call("nvfp4_kv_fp8_dequantize", _ptr(codes), rows, cols, codes.stride(0), _ptr(scale), _ptr(out), code,
+          out.stride(0), _stream(stream))
+    return out
 
 
 def nvfp4_check(stream=None):

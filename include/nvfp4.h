@@ -263,6 +263,27 @@ int nvfp4_requantize_segments(const nvfp4_operand* W, const int64_t* row_bounds,
                               uint8_t* sf_out, float* g_out, void* stream);
 
 /*
+ * nvfp4_kv_fp8_quantize / nvfp4_kv_fp8_dequantize — FP8 (E4M3) KV-cache codec
+ * with a calibrated static per-tensor scale ("Main Findings", KV-cache
+ * bullet: FP8 KV with calibrated scales instead of 1.0).  The attention that
+ * consumes the cache is not part of this library.
+ *   Encode: code = E4M3_rn_satfinite(x * inv), inv = 1 / *scale in FP32 (once),
+ *     the sign kept (also for zero); *scale not a positive finite number gives
+ *     all-zero codes.  x: device [rows, cols] BF16 or F32 (x_dtype), row stride
+ *     ld_x elements, 16-byte aligned rows; out: device [rows, cols] bytes, row
+ *     stride ld_out, 8-byte aligned.
+ *   Decode: out = e4m3(code) * *scale rounded to FP32 (then to BF16 for a BF16
+ *     output).  codes: row stride ld_codes bytes, 8-byte aligned; out: device
+ *     BF16 or F32 (out_dtype), row stride ld_out elements, 16-byte aligned rows.
+ *   cols must be a multiple of 8; scale is a device float (the calibrated
+ *   value, typically amax / 448 over calibration data).
+ */
+int nvfp4_kv_fp8_quantize(const void* x, int x_dtype, int64_t rows, int64_t cols, int64_t ld_x,
+                          const float* scale, uint8_t* out, int64_t ld_out, void* stream);
+int nvfp4_kv_fp8_dequantize(const uint8_t* codes, int64_t rows, int64_t cols, int64_t ld_codes,
+                            const float* scale, void* out, int out_dtype, int64_t ld_out, void* stream);
+
+/*
  * nvfp4_check — synchronise `stream`, then report (and clear) the library's
  * device error word: NVFP4_ERR_DEVICE_TIMEOUT if a bounded wait inside a
  * kernel gave up since the last check, NVFP4_ERR_CUDA on a CUDA error.

@@ -170,3 +170,27 @@ def test_requantize_rejects_bad_arguments(lib):
     assert call(codes=0x400000 + 64) == 1             # partial overlap with W's codes
     assert call(sf=0x800000 + 16) == 1                # partial overlap with W's scales
     assert call(W=_op(codes=0x400000, sf=0x800000, rows=256, K=48)) == 2
+
+
+def test_kv_fp8_rejects_bad_arguments(lib):
+    v = ctypes.c_void_p
+
+    def enc(x=FAKE, dtype=0, rows=4, cols=64, ld_x=64, scale=FAKE, out=FAKE, ld_out=64):
+        return lib.nvfp4_kv_fp8_quantize(v(x) if x else None, dtype, rows, cols, ld_x, v(scale) if scale else None,
+                                         v(out) if out else None, ld_out, None)
+
+    def dec(c=FAKE, rows=4, cols=64, ld_c=64, scale=FAKE, out=FAKE, dtype=0, ld_out=64):
+        return lib.nvfp4_kv_fp8_dequantize(v(c) if c else None, rows, cols, ld_c, v(scale) if scale else None,
+                                           v(out) if out else None, dtype, ld_out, None)
+    assert enc(cols=60, ld_x=64, ld_out=64) == 2      # cols % 8
+    assert enc(dtype=3) == 1
+    assert enc(scale=0) == 1
+    assert enc(x=FAKE + 8) == 3                        # rows 16-byte aligned
+    assert enc(ld_x=68) == 3                           # BF16 row stride not a multiple of 16 bytes
+    assert enc(out=FAKE + 4) == 3
+    assert enc(ld_out=60) == 1                         # ld_out < cols
+    assert enc(rows=0) == 0 and enc(cols=0, ld_x=0, ld_out=0) == 0
+    assert dec(c=FAKE + 4) == 3
+    assert dec(out=FAKE + 8) == 3
+    assert dec(dtype=1, ld_out=66) == 3
+    assert dec(ld_c=32) == 1
