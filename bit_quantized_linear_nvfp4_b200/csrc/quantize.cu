@@ -577,7 +577,7 @@ __global__ void __launch_bounds__(kThreads, 1) requant_kernel(const __grid_const
   __syncthreads();
   if (blockIdx.x == 0 && threadIdx.x < r.nseg_old) a.g_out[threadIdx.x] = g_sh[0];
   const int32_t KA = (a.K + 63) / 64;
-  constexpr int U = 8;  // chunks in flight per warp (9 bytes per lane each)
+  constexpr int U = 4;  // chunks in flight per warp (9 bytes per lane each)
   int64_t lo, hi;
   block_range(a.items, lo, hi);
   for (int64_t base = lo; base < hi; base += kWarps * U) {
