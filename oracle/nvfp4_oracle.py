@@ -337,6 +337,55 @@ def kv_fp8_dequantize(codes: np.ndarray, scale, out_dtype: str = "bf16") -> np.n
     return bf16_round(y) if out_dtype == "bf16" else y
 
 
+def activation_stats(x: np.ndarray, g=None) -> dict:
+    """Activation statistics at NVFP4 granularity (Paper summary page
+    (ai.info), "Main Findings", activation bullet: max/RMS, kurtosis, hot
+    channels against the median channel, the share of 16-element blocks
+    dominated by a single value, and the per-token A4 quantisation error).
+    Readings: a block is dominated when its largest magnitude exceeds the sum
+    of the other fifteen; the A4 error of a token is ||x - x_hat|| / ||x||
+    with x_hat the NVFP4 dequantisation under the tensor's global scale g (the
+    quantiser's; computed from x when not given); moments in FP64."""
+    x = np.asarray(x, dtype=np.float32)
+    M, K = x.shape
+    x64 = x.astype(np.float64)
+    ab = np.abs(x64).reshape(M, K // BLOCK, BLOCK)
+    amax_b = ab.max(axis=2)
+    dominated = amax_b > (ab.sum(axis=2) - amax_b)
+    codes, sf, gq = quantize(x, g)
+    x_hat = dequantize(codes, sf, gq).astype(np.float32).astype(np.float64)
+    return {
+        "n": float(M * K), "sum": x64.sum(), "sum_sq": (x64 ** 2).sum(), "sum_cube": (x64 ** 3).sum(),
+        "sum_4th": (x64 ** 4).sum(), "amax": np.abs(x64).max() if x.size else 0.0,
+        "blocks": float(amax_b.size), "dominated": float(dominated.sum()),
+        "row_err2": ((x64 - x_hat) ** 2).sum(axis=1), "row_norm2": (x64 ** 2).sum(axis=1),
+        "col_sq": (x64 ** 2).sum(axis=0), "col_max": np.abs(x64).max(axis=0),
+    }
+
+
+def activation_summary(st: dict) -> dict:
+    """Derived figures of activation_stats(): max/RMS, kurtosis (fourth central
+    moment over the squared variance), dominated-block share, per-token A4
+    error (mean, min, max) and the hot-channel ratio (largest channel RMS over
+    the median channel RMS)."""
+    n = st["n"]
+    mean = st["sum"] / n
+    m2 = st["sum_sq"] / n
+    var = m2 - mean ** 2
+    m4c = st["sum_4th"] / n - 4 * mean * st["sum_cube"] / n + 6 * mean ** 2 * m2 - 3 * mean ** 4
+    norm = np.sqrt(st["row_norm2"])
+    err = np.sqrt(st["row_err2"]) / np.where(norm > 0, norm, 1.0)
+    col_rms = np.sqrt(np.asarray(st["col_sq"]) * (len(st["row_norm2"]) and 1.0 / len(st["row_norm2"])))
+    med = np.median(col_rms)
+    return {"max_over_rms": st["amax"] / np.sqrt(m2) if m2 > 0 else 0.0,
+            "kurtosis": m4c / var ** 2 if var > 0 else 0.0,
+            "dominated_share": st["dominated"] / st["blocks"] if st["blocks"] else 0.0,
+            "a4_err_mean": float(err.mean()) if err.size else 0.0,
+            "a4_err_min": float(err.min()) if err.size else 0.0,
+            "a4_err_max": float(err.max()) if err.size else 0.0,
+            "hot_channel_ratio": float(col_rms.max() / med) if med > 0 else 0.0}
+
+
 def bf16_round(y) -> np.ndarray:
     """Round FP64 values to BF16 (8 significant bits, nearest, ties to even);
     returned as FP64.  y = m * 2^e with 0.5 <= |m| < 1, so y / 2^(e-8) has its
