@@ -1,0 +1,288 @@
+// Activation statistics at NVFP4 granularity, sm_100a.
+//
+// "Why Gated DeltaNet Survives 4-Bit Quantization" (ai.info summary), "Main
+// Findings", activation bullet: the residual stream's max/RMS, kurtosis, hot
+// channels against the median channel, the share of 16-element blocks
+// dominated by a single value, and the per-token A4 quantisation error.  One
+// pass over X accumulates (the caller zeroes the outputs once; later calls
+// add, e.g. over calibration batches):
+//   moments[8] (FP64): sum x, sum x^2, sum x^3, sum x^4, max |x|, elements,
+//                      16-blocks, dominated 16-blocks (largest magnitude >
+//                      the sum of the other fifteen, decided in FP64);
+//   row_err2[M], row_norm2[M] (FP32): sum (x - x_hat)^2 and sum x^2 per row,
+//                      x_hat the NVFP4 dequantisation under the global scale g
+//                      with the quantiser's exact arithmetic;
+//   col_sq[K], col_max[K] (FP32): sum x^2 and max |x| per column.
+//
+// HBM-bound.  A warp owns a unit = (512-column strip, range of rows); lane l
+// reads block l of the strip in each row with one 256-bit load, several rows in
+// flight.  Per-column sums stay in the lane's registers for the whole unit,
+// so the column outputs take one atomic per column and unit; row sums are
+// warp-reduced, one atomic per row and strip; FP64 moments are block-reduced,
+// one atomic per block.
+#include <cfloat>
+#include <cstdint>
+
+#include <cuda_runtime.h>
+
+#include "internal.h"
+#include "ptx.cuh"
+
+namespace nvfp4 {
+namespace st {
+
+constexpr int kThreads = 256;
+constexpr int kWarps = kThreads / 32;
+
+struct StatsArgs {
+  const uint8_t* x;
+  int64_t ld_bytes;
+  int32_t M, K, cpr;  // cpr: 512-column strips
+  int32_t ranges;     // row ranges per strip
+  const float* g;
+  double* moments;
+  float* row_err2;
+  float* row_norm2;
+  float* col_sq;
+  float* col_max;
+};
+
+template <int DTYPE>
+struct Raw {
+  uint32_t w[DTYPE == NVFP4_DTYPE_BF16 ? 8 : 16];
+};
+
+__device__ __forceinline__ void ld_v8(const void* p, uint32_t* r) {
+  asm volatile("ld.global.nc.L1::no_allocate.v8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]),
+                 "=r"(r[6]), "=r"(r[7])
+               : "l"(p));
+}
+
+template <int DTYPE, bool WIDE>
+__device__ __forceinline__ void load(const uint8_t* p, Raw<DTYPE>& b) {
+  constexpr int kW = DTYPE == NVFP4_DTYPE_BF16 ? 8 : 16;
+#pragma unroll
+  for (int i = 0; i < kW; i += 8) {
+    if constexpr (WIDE) {
+      ld_v8(p + 4 * i, b.w + i);
+    } else {
+      const uint4 a = __ldg(reinterpret_cast<const uint4*>(p + 4 * i));
+      const uint4 c = __ldg(reinterpret_cast<const uint4*>(p + 4 * i + 16));
+      b.w[i] = a.x; b.w[i + 1] = a.y; b.w[i + 2] = a.z; b.w[i + 3] = a.w;
+      b.w[i + 4] = c.x; b.w[i + 5] = c.y; b.w[i + 6] = c.z; b.w[i + 7] = c.w;
+    }
+  }
+}
+
+template <int DTYPE>
+__device__ __forceinline__ void to_f32(const Raw<DTYPE>& b, float (&v)[16]) {
+  if constexpr (DTYPE == NVFP4_DTYPE_BF16) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      v[2 * i] = __uint_as_float(b.w[i] << 16);
+      v[2 * i + 1] = __uint_as_float(b.w[i] & 0xFFFF0000u);
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(b.w[i]);
+  }
+}
+
+__device__ __forceinline__ float e4m3_val(uint32_t b) {
+  const uint32_t e = (b >> 3) & 15u, m = b & 7u;
+  return e ? __uint_as_float(((e + 120u) << 23) | (m << 20)) : static_cast<float>(m) * 0.001953125f;
+}
+
+// E2M1 (satfinite, nearest even) of a float, as its value.
+__device__ __forceinline__ float e2m1_round(float q) {
+  uint16_t r;
+  asm("{\n\t.reg .b8 c;\n\tcvt.rn.satfinite.e2m1x2.f32 c, %1, %1;\n\tmov.b16 %0, {c, c};\n\t}" : "=h"(r) : "f"(q));
+  const uint32_t c = r & 15u;
+  const float v = static_cast<float>((0xC8643210u >> (4 * (c & 7u))) & 15u) * 0.5f;
+  return (c & 8u) ? -v : v;
+}
+
+__device__ __forceinline__ double warp_sum(double v) {
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+  return v;
+}
+__device__ __forceinline__ float warp_sumf(float v) {
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+  return v;
+}
+
+template <int DTYPE, bool WIDE>
+__global__ void __launch_bounds__(kThreads, 2) stats_kernel(const __grid_constant__ StatsArgs a) {
+  constexpr int kEsz = DTYPE == NVFP4_DTYPE_BF16 ? 2 : 4;
+  constexpr int kRows = DTYPE == NVFP4_DTYPE_BF16 ? 4 : 2;  // rows in flight per warp
+  __shared__ double red[kWarps][8];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  grid_dependency_wait();
+  if (threadIdx.x == 0) grid_launch_dependents();
+  const float g = a.g != nullptr ? __ldg(a.g) : 0.0f;
+  const bool quant = a.g != nullptr && g > 0.0f;
+  double s1 = 0, s2 = 0, s3 = 0, s4 = 0, blocks = 0, dom = 0;
+  float amax = 0.0f;
+  const int64_t units = static_cast<int64_t>(a.cpr) * a.ranges;
+  const int64_t nwarps = static_cast<int64_t>(gridDim.x) * kWarps;
+  for (int64_t u = static_cast<int64_t>(blockIdx.x) * kWarps + warp; u < units; u += nwarps) {
+    const int32_t strip = static_cast<int32_t>(u % a.cpr);
+    const int32_t rr = static_cast<int32_t>(u / a.cpr);
+    const int32_t r0 = static_cast<int32_t>(static_cast<int64_t>(a.M) * rr / a.ranges);
+    const int32_t r1 = static_cast<int32_t>(static_cast<int64_t>(a.M) * (rr + 1) / a.ranges);
+    const int32_t col = strip * 512 + lane * 16;
+    const bool have = col < a.K;
+    float csq[16], cmx[16];
+#pragma unroll
+    for (int e = 0; e < 16; ++e) csq[e] = cmx[e] = 0.0f;
+    for (int32_t row0 = r0; row0 < r1; row0 += kRows) {
+      Raw<DTYPE> raw[kRows];
+#pragma unroll
+      for (int k = 0; k < kRows; ++k)
+        if (have && row0 + k < r1)
+          load<DTYPE, WIDE>(a.x + static_cast<int64_t>(row0 + k) * a.ld_bytes + static_cast<int64_t>(col) * kEsz, raw[k]);
+#pragma unroll
+      for (int k = 0; k < kRows; ++k) {
+        if (row0 + k >= r1) break;  // uniform across the warp
+        float rn2 = 0.0f, re2 = 0.0f;
+        if (have) {
+          float v[16];
+          to_f32<DTYPE>(raw[k], v);
+          float am = 0.0f, b1 = 0.0f, b2 = 0.0f, b3 = 0.0f, b4 = 0.0f;
+          double asum = 0.0;
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const float x = v[e], ax = fabsf(x), x2 = x * x;
+            am = fmaxf(am, ax);
+            asum += static_cast<double>(ax);
+            b1 += x;
+            b2 += x2;
+            b3 += x2 * x;
+            b4 += x2 * x2;
+            csq[e] += x2;
+            cmx[e] = fmaxf(cmx[e], ax);
+          }
+          amax = fmaxf(amax, am);
+          s1 += b1; s2 += b2; s3 += b3; s4 += b4;
+          blocks += 1.0;
+          if (static_cast<double>(am) > asum - static_cast<double>(am)) dom += 1.0;
+          rn2 = b2;
+          if (quant) {
+            // the quantiser's arithmetic (block scale, reciprocal, codes)
+            const float s = (am / 6.0f) / g;
+            uint16_t sr;
+            asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(sr) : "f"(0.0f), "f"(s));
+            const float S = e4m3_val(sr & 0xFFu);
+            const float denom = S * g;
+            float inv = denom > 0.0f ? 1.0f / denom : 0.0f;
+            inv = fminf(inv, FLT_MAX);
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+              const float xh = (e2m1_round(v[e] * inv) * S) * g;
+              const float d = v[e] - xh;
+              re2 += d * d;
+            }
+          }
+        }
+        rn2 = warp_sumf(rn2);
+        re2 = warp_sumf(re2);
+        if (lane == 0) {
+          if (a.row_norm2 != nullptr) atomicAdd(a.row_norm2 + row0 + k, rn2);
+          if (a.row_err2 != nullptr && quant) atomicAdd(a.row_err2 + row0 + k, re2);
+        }
+      }
+    }
+    if (have) {
+#pragma unroll
+      for (int e = 0; e < 16; ++e) {
+        if (a.col_sq != nullptr) atomicAdd(a.col_sq + col + e, csq[e]);
+        if (a.col_max != nullptr) atomicMax(reinterpret_cast<unsigned int*>(a.col_max) + col + e, __float_as_uint(cmx[e]));
+      }
+    }
+  }
+  // block reduction of the moments, then one atomic each
+  double m[7] = {s1, s2, s3, s4, static_cast<double>(amax), blocks, dom};
+#pragma unroll
+  for (int i = 0; i < 7; ++i) {
+    if (i == 4) {
+      double v = m[i];
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) v = fmax(v, __shfl_xor_sync(0xffffffffu, v, off));
+      m[i] = v;
+    } else {
+      m[i] = warp_sum(m[i]);
+    }
+    if (lane == 0) red[warp][i] = m[i];
+  }
+  __syncthreads();
+  if (threadIdx.x < 7) {
+    const int i = threadIdx.x;
+    double v = red[0][i];
+    for (int w = 1; w < kWarps; ++w) v = i == 4 ? fmax(v, red[w][i]) : v + red[w][i];
+    if (i == 4) {
+      atomicMax(reinterpret_cast<unsigned long long*>(a.moments + 4), static_cast<unsigned long long>(__double_as_longlong(v)));
+    } else {
+      atomicAdd(a.moments + (i < 4 ? i : i + 1), v);
+    }
+  }
+  if (threadIdx.x == 0) {
+    double nb = 0.0;
+    for (int w = 0; w < kWarps; ++w) nb += red[w][5];
+    atomicAdd(a.moments + 5, 16.0 * nb);  // elements = 16 per block
+  }
+}
+
+int sm_count() {
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  return sms;
+}
+
+}  // namespace st
+
+cudaError_t launch_act_stats(const void* x, int dtype, int64_t M, int64_t K, int64_t ld, const float* g,
+                             double* moments, float* row_err2, float* row_norm2, float* col_sq, float* col_max,
+                             cudaStream_t stream) {
+  using namespace st;
+  if (M == 0) return cudaSuccess;
+  StatsArgs a{};
+  const int esz = dtype == NVFP4_DTYPE_BF16 ? 2 : 4;
+  a.x = static_cast<const uint8_t*>(x);
+  a.ld_bytes = ld * esz;
+  a.M = static_cast<int32_t>(M);
+  a.K = static_cast<int32_t>(K);
+  a.cpr = static_cast<int32_t>(ceil_div(K, 512));
+  const int64_t blocks = static_cast<int64_t>(sm_count()) * 2;
+  const int64_t warps = blocks * kWarps;
+  int64_t ranges = warps / a.cpr;
+  if (ranges < 1) ranges = 1;
+  if (ranges > M) ranges = M;
+  a.ranges = static_cast<int32_t>(ranges);
+  a.g = g;
+  a.moments = moments;
+  a.row_err2 = row_err2;
+  a.row_norm2 = row_norm2;
+  a.col_sq = col_sq;
+  a.col_max = col_max;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(blocks));
+  cfg.blockDim = dim3(kThreads);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const bool wide = (reinterpret_cast<uintptr_t>(x) % 32 == 0) && (a.ld_bytes % 32 == 0);
+  if (dtype == NVFP4_DTYPE_BF16)
+    return wide ? cudaLaunchKernelEx(&cfg, stats_kernel<NVFP4_DTYPE_BF16, true>, a)
+                : cudaLaunchKernelEx(&cfg, stats_kernel<NVFP4_DTYPE_BF16, false>, a);
+  return wide ? cudaLaunchKernelEx(&cfg, stats_kernel<NVFP4_DTYPE_F32, true>, a)
+              : cudaLaunchKernelEx(&cfg, stats_kernel<NVFP4_DTYPE_F32, false>, a);
+}
+
+}  // namespace nvfp4

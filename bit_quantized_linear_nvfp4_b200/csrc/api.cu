@@ -339,6 +339,30 @@ int nvfp4_kv_fp8_dequantize(const uint8_t* codes, int64_t rows, int64_t cols, in
   return NVFP4_OK;
 }
 
+int nvfp4_activation_stats(const void* x, int x_dtype, int64_t M, int64_t K, int64_t ld_x, const float* g,
+                           double* moments, float* row_err2, float* row_norm2, float* col_sq, float* col_max,
+                           void* stream) {
+  if (x_dtype != NVFP4_DTYPE_BF16 && x_dtype != NVFP4_DTYPE_F32) return NVFP4_ERR_INVALID_ARG;
+  if (M < 0 || K <= 0 || moments == nullptr) return NVFP4_ERR_INVALID_ARG;
+  if (K % 16 != 0) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+  if (M > (int64_t(1) << 31) - 1 || K > (int64_t(1) << 30)) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+  if (row_err2 != nullptr && g == nullptr) return NVFP4_ERR_INVALID_ARG;
+  if (M == 0) return NVFP4_OK;
+  if (x == nullptr || ld_x < K) return NVFP4_ERR_INVALID_ARG;
+  const int esz = x_dtype == NVFP4_DTYPE_BF16 ? 2 : 4;
+  if (!aligned16(x) || (ld_x * esz) % 16 != 0) return NVFP4_ERR_MISALIGNED;
+  if ((reinterpret_cast<uintptr_t>(moments) & 7u) != 0) return NVFP4_ERR_MISALIGNED;
+  const void* f32s[5] = {g, row_err2, row_norm2, col_sq, col_max};
+  for (const void* q : f32s)
+    if ((reinterpret_cast<uintptr_t>(q) & 3u) != 0) return NVFP4_ERR_MISALIGNED;
+  int st = check_device();
+  if (st != NVFP4_OK) return st;
+  cudaError_t e = nvfp4::launch_act_stats(x, x_dtype, M, K, ld_x, g, moments, row_err2, row_norm2, col_sq, col_max,
+                                          static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e);
+  return NVFP4_OK;
+}
+
 int nvfp4_gemm(const nvfp4_operand* A, const float* g_a, const nvfp4_operand* W, const float* g_w,
                void* out, int out_dtype, int64_t ld_out, void* workspace, size_t workspace_bytes,
                void* stream) {

@@ -51,6 +51,11 @@ cudaError_t launch_requantize(const uint8_t* codes, const uint8_t* sf, int64_t N
 cudaError_t launch_kv_fp8(bool encode, int dtype, const void* src, int64_t ld_src, void* dst, int64_t ld_dst,
                           int64_t rows, int64_t cols, const float* scale, cudaStream_t stream);
 
+// Activation statistics of x [M, K] (accumulating; see nvfp4_activation_stats).
+cudaError_t launch_act_stats(const void* x, int dtype, int64_t M, int64_t K, int64_t ld, const float* g,
+                             double* moments, float* row_err2, float* row_norm2, float* col_sq, float* col_max,
+                             cudaStream_t stream);
+
 // GEMM epilogue description handed to the kernels.
 struct EpiSegment {
   int64_t n_begin, n_end;

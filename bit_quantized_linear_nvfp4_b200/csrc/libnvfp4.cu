@@ -6,3 +6,4 @@
 #include "api.cu"
 #include "noalloc.cu"
 #include "kv_fp8.cu"
+#include "act_stats.cu"

@@ -44,7 +44,7 @@ EXPORTED = (
     "nvfp4_quantize_workspace_bytes", "nvfp4_quantize", "nvfp4_quantize_segments",
     "nvfp4_gemm_workspace_bytes", "nvfp4_gemm", "nvfp4_fused_proj", "nvfp4_check",
     "nvfp4_quantize_noalloc", "nvfp4_linear", "nvfp4_requantize_segments",
-    "nvfp4_kv_fp8_quantize", "nvfp4_kv_fp8_dequantize",
+    "nvfp4_kv_fp8_quantize", "nvfp4_kv_fp8_dequantize", "nvfp4_activation_stats",
 )
 
 
@@ -120,6 +120,10 @@ def _lib():
         lib.nvfp4_kv_fp8_dequantize.restype = c.c_int
         lib.nvfp4_kv_fp8_dequantize.argtypes = [c.c_void_p, c.c_int64, c.c_int64, c.c_int64, c.c_void_p,
                                                 c.c_void_p, c.c_int, c.c_int64, c.c_void_p]
+        lib.nvfp4_activation_stats.restype = c.c_int
+        lib.nvfp4_activation_stats.argtypes = [c.c_void_p, c.c_int, c.c_int64, c.c_int64, c.c_int64, c.c_void_p,
+                                               c.c_void_p, c.c_void_p, c.c_void_p, c.c_void_p, c.c_void_p,
+                                               c.c_void_p]
         lib.nvfp4_check.restype = c.c_int
         lib.nvfp4_check.argtypes = [c.c_void_p]
         _LIB = lib
@@ -340,6 +344,49 @@ def nvfp4_kv_fp8_dequantize(codes: torch.Tensor, scale: torch.Tensor, out_dtype=
     code = DTYPE_BF16 if out.dtype == torch.bfloat16 else DTYPE_F32
     _call("nvfp4_kv_fp8_dequantize", _ptr(codes), rows, cols, codes.stride(0), _ptr(scale), _ptr(out), code,
           out.stride(0), _stream(stream))
+    return out
+
+
+def nvfp4_activation_stats(x: torch.Tensor, g: Optional[torch.Tensor] = None, *, into: Optional[dict] = None,
+                           stream=None) -> dict:
+    """Accumulate NVFP4-granularity statistics of x[M, K] into `into` (a dict of
+    device tensors from a previous call, or fresh zeros): moments (float64[8]),
+    row_err2 / row_norm2 (float32[M], A4 error needs g), col_sq / col_max
+    (float32[K])."""
+    _check_2d(x)
+    M, K = x.shape
+    dev = x.device
+    if into is None:
+        into = {"moments": torch.zeros(8, dtype=torch.float64, device=dev),
+                "row_err2": torch.zeros(M, dtype=torch.float32, device=dev) if g is not None else None,
+                "row_norm2": torch.zeros(M, dtype=torch.float32, device=dev),
+                "col_sq": torch.zeros(K, dtype=torch.float32, device=dev),
+                "col_max": torch.zeros(K, dtype=torch.float32, device=dev)}
+    _call("nvfp4_activation_stats", _ptr(x), _dtype_code(x), M, K, x.stride(0), _ptr(g), _ptr(into["moments"]),
+          _ptr(into["row_err2"]), _ptr(into["row_norm2"]), _ptr(into["col_sq"]), _ptr(into["col_max"]),
+          _stream(stream))
+    return into
+
+
+def activation_summary(stats: dict) -> dict:
+    """Host-side figures from nvfp4_activation_stats' accumulators: max/RMS,
+    kurtosis (fourth central moment / variance^2), dominated-block share,
+    per-token A4 error (mean, min, max) and hot-channel ratio (largest channel
+    RMS over the median channel RMS)."""
+    m = stats["moments"].double().cpu().tolist()
+    n = m[5]
+    mean, m2 = m[0] / n, m[1] / n
+    var = m2 - mean * mean
+    m4c = m[3] / n - 4 * mean * m[2] / n + 6 * mean * mean * m2 - 3 * mean ** 4
+    out = {"max_over_rms": m[4] / m2 ** 0.5 if m2 > 0 else 0.0, "kurtosis": m4c / var ** 2 if var > 0 else 0.0,
+           "dominated_share": m[7] / m[6] if m[6] else 0.0}
+    rows = stats["row_norm2"].double()
+    if stats.get("row_err2") is not None:
+        err = (stats["row_err2"].double() / torch.where(rows > 0, rows, torch.ones_like(rows))).sqrt()
+        out.update(a4_err_mean=err.mean().item(), a4_err_min=err.min().item(), a4_err_max=err.max().item())
+    col_rms = (stats["col_sq"].double() / rows.numel()).sqrt()
+    med = col_rms.median().item()
+    out["hot_channel_ratio"] = col_rms.max().item() / med if med > 0 else 0.0
     return out
 
 

@@ -284,6 +284,32 @@ int nvfp4_kv_fp8_dequantize(const uint8_t* codes, int64_t rows, int64_t cols, in
                             const float* scale, void* out, int out_dtype, int64_t ld_out, void* stream);
 
 /*
+ * nvfp4_activation_stats — activation statistics at NVFP4 granularity, one
+ * pass over x ("Main Findings", activation bullet: max/RMS, kurtosis, hot
+ * channels against the median channel, the share of 16-element blocks
+ * dominated by one value, per-token A4 error).  Every output ACCUMULATES: the
+ * caller zeroes them once, and further calls add (statistics over several
+ * calibration batches).
+ *   x        device [M, K] BF16 or F32 (x_dtype), row stride ld_x elements,
+ *            16-byte aligned rows; K a multiple of 16.
+ *   g        device float, the global scale for the A4 error (nvfp4_quantize's
+ *            g_out), or NULL (then row_err2 must be NULL).
+ *   moments  device double[8]: sum x, sum x^2, sum x^3, sum x^4 (FP64
+ *            accumulation), max |x|, elements, 16-blocks, dominated 16-blocks
+ *            (largest magnitude > the sum of the other fifteen).
+ *   row_err2, row_norm2  device float[M] or NULL: per row, sum (x - x_hat)^2
+ *            with x_hat the NVFP4 dequantisation under g (the quantiser's
+ *            arithmetic), and sum x^2.
+ *   col_sq, col_max  device float[K] or NULL: per column, sum x^2 and max |x|.
+ * Derived figures: max/RMS = moments[4] / sqrt(moments[1] / moments[5]);
+ * kurtosis from the four moments; per-token A4 error sqrt(row_err2/row_norm2);
+ * hot-channel ratio from sqrt(col_sq / M) against its median.
+ */
+int nvfp4_activation_stats(const void* x, int x_dtype, int64_t M, int64_t K, int64_t ld_x, const float* g,
+                           double* moments, float* row_err2, float* row_norm2, float* col_sq, float* col_max,
+                           void* stream);
+
+/*
  * nvfp4_check — synchronise `stream`, then report (and clear) the library's
  * device error word: NVFP4_ERR_DEVICE_TIMEOUT if a bounded wait inside a
  * kernel gave up since the last check, NVFP4_ERR_CUDA on a CUDA error.

@@ -194,3 +194,20 @@ def test_kv_fp8_rejects_bad_arguments(lib):
     assert dec(out=FAKE + 8) == 3
     assert dec(dtype=1, ld_out=66) == 3
     assert dec(ld_c=32) == 1
+
+
+def test_activation_stats_rejects_bad_arguments(lib):
+    v = ctypes.c_void_p
+
+    def call(x=FAKE, dtype=0, M=4, K=64, ld=64, g=FAKE, mom=FAKE, re=FAKE, rn=FAKE, cs=FAKE, cm=FAKE):
+        p = lambda a: v(a) if a else None
+        return lib.nvfp4_activation_stats(p(x), dtype, M, K, ld, p(g), p(mom), p(re), p(rn), p(cs), p(cm), None)
+    assert call(K=40) == 2
+    assert call(dtype=5) == 1
+    assert call(mom=0) == 1
+    assert call(g=0) == 1                   # A4 error requested without a global scale
+    assert call(x=FAKE + 8) == 3
+    assert call(mom=FAKE + 4) == 3
+    assert call(cs=FAKE + 2) == 3
+    assert call(ld=32) == 1
+    assert call(M=0) == 0
