@@ -733,9 +733,139 @@ def run_kvfp8(args):
         dist.destroy_process_group()
 
 
+def run_actstats(args):
+    """Activation statistics of the GDN prefill activation X[32768, 5120] (BF16,
+    0.5% outlier channels x100): one nvfp4_activation_stats call per step, with
+    the global scale for the A4 error; HBM-bound (2 B read per element)."""
+    import torch
+    from bit_quantized_linear_nvfp4_b200 import nvfp4 as nv
+    from bit_quantized_linear_nvfp4_b200 import workloads as wl
+    world, rank, local = dist_env()
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    dist = dist_init(world)
+    peaks, peak_src = load_peaks()
+    w = wl.GDN
+    x_np = wl.make_x(w)
+    M, K = x_np.shape
+    sets = []
+    for _ in range(ROTATE):
+        x = torch.from_numpy(x_np).to(device).to(torch.bfloat16)
+        _, g = nv.nvfp4_quantize(x)
+        acc = nv.nvfp4_activation_stats(x, g)
+        sets.append((x, g, acc))
+    stream = torch.cuda.current_stream()
+    graphs = []
+    torch.cuda.synchronize()
+    for x, g, acc in sets:
+        gr = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gr):
+            nv.nvfp4_activation_stats(x, g, into=acc)
+        graphs.append(gr)
+    Kst, Wm = args.steps, args.warmup
+    for i in range(Wm):
+        graphs[i % ROTATE].replay()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    dist_barrier(dist)
+    torch.cuda.synchronize()
+    t0.record(stream)
+    for i in range(Kst):
+        graphs[i % ROTATE].replay()
+    t1.record(stream)
+    torch.cuda.synchronize()
+    dist_barrier(dist)
+    clk = clocks.stop()
+    ms = dist_max(dist, t0.elapsed_time(t1), device) / Kst
+    nv.nvfp4_check()
+    bytes_step = M * K * 2
+    hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    ach = bytes_step / (ms * 1e-3) / 1e9
+    x0, g0, acc0 = sets[0]
+    h_x = x0.cpu().pin_memory()
+    h_m = torch.empty(8, dtype=torch.float64).pin_memory()
+
+    def e2e_one():
+        x0.copy_(h_x, non_blocking=True)
+        graphs[0].replay()
+        h_m.copy_(acc0["moments"], non_blocking=True)
+
+    for _ in range(Wm):
+        e2e_one()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(Kst):
+        e2e_one()
+    b.record(stream)
+    torch.cuda.synchronize()
+    ms_e2e = a.elapsed_time(b) / Kst
+    line = {
+        "metric": METRIC, "value": bytes_step * world / (ms * 1e-3) / 1e9, "unit": "GB/s", "n_gpus": world,
+        "steps": Kst, "warmup": Wm, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16 in, fp64/fp32 accumulation", "data": "synthetic (GDN prefill activation)",
+        "config": {"workload": "activation_stats_32768x5120", "M": M, "K": K,
+                   "parallelism": "replicas" if world > 1 else "single",
+                   "l2": f"{ROTATE} rotating inputs, working set above the 126 MB L2"},
+        "roofline": {"bound": "hbm", "achieved": ach, "peak": hbm, "unit": "GB/s", "frac": ach / hbm,
+                     "traffic": TRAFFIC_BYTES.get("actstats"), "peak_source": f"{peak_src} copy bandwidth",
+                     "kernel": "nvfp4 activation stats", "ms_per_launch": ms},
+        "clocks": clk,
+        "e2e": {"value": bytes_step / (ms_e2e * 1e-3) / 1e9, "unit": "GB/s", "h2d_bytes_per_step": bytes_step,
+                "d2h_bytes_per_step": 64, "ms_per_step": ms_e2e},
+        "gpu_launches": Kst,
+        "summary": nv.activation_summary(acc0),
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        from oracle import nvfp4_oracle as o
+        rows = 512
+        g_np = np.float32(g0.item())
+        t = time.perf_counter()
+        n = 0
+        while time.perf_counter() - t < args.cpu_seconds / 2 or n == 0:
+            o.activation_stats(x_np[:rows], g_np)
+            n += 1
+        per = (time.perf_counter() - t) / n
+        line["cpu_baseline"] = {"value": rows * K * 2 / per / 1e9, "unit": "GB/s", "cores": _blas_threads(),
+                                "kind": "oracle", "sample": f"{rows} rows x {K} per pass ({n} passes)",
+                                "host_cpus": os.cpu_count()}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    for gr in graphs:
+        del gr
+    if dist is not None:
+        dist.destroy_process_group()
+
+
 def run_reference(args):
     world, rank, _ = dist_env()
     if rank != 0:
+        return
+    if args.workload == "actstats":
+        from bit_quantized_linear_nvfp4_b200 import workloads as wl
+        from oracle import nvfp4_oracle as o
+        rows = 256
+        x = wl.make_x(wl.GDN, rows=rows)
+        g = o.global_scale(x)
+        for _ in range(args.warmup):
+            o.activation_stats(x, g)
+        t = time.perf_counter()
+        for _ in range(args.steps):
+            o.activation_stats(x, g)
+        per = (time.perf_counter() - t) / args.steps
+        val = rows * x.shape[1] * 2 / per / 1e9
+        print(json.dumps({"impl": "reference", "metric": METRIC, "value": val, "unit": "GB/s", "n_gpus": world,
+                          "steps": args.steps, "warmup": args.warmup, "ms_per_step": per * 1e3,
+                          "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+                          "dtype": "f64 (oracle)", "data": "synthetic",
+                          "config": {"workload": "activation_stats_32768x5120", "M": 32768, "K": x.shape[1]},
+                          "cpu_baseline": {"value": val, "unit": "GB/s", "cores": _blas_threads(), "kind": "oracle",
+                                           "sample": f"{rows} rows x {x.shape[1]} per step (oracle statistics)"},
+                          "e2e": {"value": val, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}),
+              flush=True)
         return
     if args.workload == "kvfp8":
         from oracle import nvfp4_oracle as o
@@ -821,7 +951,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--workload", default="oproj",
                     choices=["oproj", "mlp", "gdn", "tiny", "decode1", "decode8", "decode64", "quant", "requant",
-                             "kvfp8"])
+                             "kvfp8", "actstats"])
     ap.add_argument("--impl", default="product", choices=["product", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
@@ -836,6 +966,8 @@ def main():
         run_requant(args)
     elif args.workload == "kvfp8":
         run_kvfp8(args)
+    elif args.workload == "actstats":
+        run_actstats(args)
     else:
         run_product(args)
 

@@ -181,7 +181,8 @@ __global__ void __launch_bounds__(kThreads, 2) stats_kernel(const __grid_constan
             inv = fminf(inv, FLT_MAX);
 #pragma unroll
             for (int e = 0; e < 16; ++e) {
-              const float xh = (e2m1_round(v[e] * inv) * S) * g;
+              // x_hat rounded to FP32 on its own (no contraction into the subtraction)
+              const float xh = __fmul_rn(__fmul_rn(e2m1_round(v[e] * inv), S), g);
               const float d = v[e] - xh;
               re2 += d * d;
             }

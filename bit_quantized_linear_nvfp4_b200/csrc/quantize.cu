@@ -618,7 +618,7 @@ __global__ void __launch_bounds__(kThreads, 1) requant_kernel(const __grid_const
         for (int e = 0; e < 16; ++e) {
           const uint32_t word = e < 8 ? c[u].x : c[u].y;
           const uint32_t code = (word >> (4 * (e & 7))) & 15u;
-          b.w[e] = __float_as_uint((e2m1_value(code) * S) * g);  // e2m1 * S exact, one rounding
+          b.w[e] = __float_as_uint(__fmul_rn(e2m1_value(code) * S, g));  // e2m1 * S exact, one rounding
         }
       }
       quantize_block<NVFP4_DTYPE_F32>(a, g_sh, b, have[u], rows[u], cols[u]);

@@ -385,7 +385,7 @@ def activation_summary(stats: dict) -> dict:
         err = (stats["row_err2"].double() / torch.where(rows > 0, rows, torch.ones_like(rows))).sqrt()
         out.update(a4_err_mean=err.mean().item(), a4_err_min=err.min().item(), a4_err_max=err.max().item())
     col_rms = (stats["col_sq"].double() / rows.numel()).sqrt()
-    med = col_rms.median().item()
+    med = torch.quantile(col_rms, 0.5).item()  # the mean of the two middle values for an even count
     out["hot_channel_ratio"] = col_rms.max().item() / med if med > 0 else 0.0
     return out
 
