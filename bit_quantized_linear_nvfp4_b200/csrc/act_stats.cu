@@ -23,6 +23,7 @@
 #include <cfloat>
 #include <cstdint>
 
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
 #include "internal.h"
@@ -94,13 +95,41 @@ __device__ __forceinline__ float e4m3_val(uint32_t b) {
   return e ? __uint_as_float(((e + 120u) << 23) | (m << 20)) : static_cast<float>(m) * 0.001953125f;
 }
 
-// E2M1 (satfinite, nearest even) of a float, as its value.
-__device__ __forceinline__ float e2m1_round(float q) {
-  uint16_t r;
-  asm("{\n\t.reg .b8 c;\n\tcvt.rn.satfinite.e2m1x2.f32 c, %1, %1;\n\tmov.b16 %0, {c, c};\n\t}" : "=h"(r) : "f"(q));
-  const uint32_t c = r & 15u;
-  const float v = static_cast<float>((0xC8643210u >> (4 * (c & 7u))) & 15u) * 0.5f;
-  return (c & 8u) ? -v : v;
+// Packed FP32 pairs (sm_100 f32x2 arithmetic; every lane rounds like the
+// scalar instruction).
+__device__ __forceinline__ uint64_t pk(float a, float b) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+  return r;
+}
+__device__ __forceinline__ float2 upk(uint64_t v) {
+  float2 f;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(f.x), "=f"(f.y) : "l"(v));
+  return f;
+}
+__device__ __forceinline__ uint64_t mul2(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+
+// E2M1 (satfinite, nearest even) of a pair of floats, returned as the pair of
+// code values (exact; element a in .x).
+__device__ __forceinline__ float2 e2m1_round2(float2 q) {
+  uint32_t h2;
+  asm("{\n\t.reg .b8 c;\n\tcvt.rn.satfinite.e2m1x2.f32 c, %2, %1;\n\tcvt.rn.f16x2.e2m1x2 %0, c;\n\t}"
+      : "=r"(h2) : "f"(q.x), "f"(q.y));
+  return __half22float2(*reinterpret_cast<const __half2*>(&h2));
 }
 
 __device__ __forceinline__ double warp_sum(double v) {
@@ -151,25 +180,32 @@ __global__ void __launch_bounds__(kThreads, 2) stats_kernel(const __grid_constan
         if (have) {
           float v[16];
           to_f32<DTYPE>(raw[k], v);
-          float am = 0.0f, b1 = 0.0f, b2 = 0.0f, b3 = 0.0f, b4 = 0.0f;
+          float am = 0.0f;
           double asum = 0.0;
+          uint64_t p1 = 0, p2 = 0, p3 = 0, p4 = 0;  // packed even/odd partial sums
 #pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            const float x = v[e], ax = fabsf(x), x2 = x * x;
-            am = fmaxf(am, ax);
-            asum += static_cast<double>(ax);
-            b1 += x;
-            b2 += x2;
-            b3 += x2 * x;
-            b4 += x2 * x2;
-            csq[e] += x2;
-            cmx[e] = fmaxf(cmx[e], ax);
+          for (int e = 0; e < 16; e += 2) {
+            const uint64_t xv = pk(v[e], v[e + 1]);
+            const uint64_t x2 = mul2(xv, xv);
+            p1 = add2(p1, xv);
+            p2 = add2(p2, x2);
+            p3 = fma2(x2, xv, p3);
+            p4 = fma2(x2, x2, p4);
+            const float2 sq = upk(x2);
+            csq[e] += sq.x;
+            csq[e + 1] += sq.y;
+            const float a0 = fabsf(v[e]), a1 = fabsf(v[e + 1]);
+            cmx[e] = fmaxf(cmx[e], a0);
+            cmx[e + 1] = fmaxf(cmx[e + 1], a1);
+            am = fmaxf(am, fmaxf(a0, a1));
+            asum += static_cast<double>(a0) + static_cast<double>(a1);
           }
+          const float2 f1 = upk(p1), f2 = upk(p2), f3 = upk(p3), f4 = upk(p4);
           amax = fmaxf(amax, am);
-          s1 += b1; s2 += b2; s3 += b3; s4 += b4;
+          s1 += f1.x + f1.y; s2 += f2.x + f2.y; s3 += f3.x + f3.y; s4 += f4.x + f4.y;
           blocks += 1.0;
           if (static_cast<double>(am) > asum - static_cast<double>(am)) dom += 1.0;
-          rn2 = b2;
+          rn2 = f2.x + f2.y;
           if (quant) {
             // the quantiser's arithmetic (block scale, reciprocal, codes)
             const float s = (am / 6.0f) / g;
@@ -179,13 +215,19 @@ __global__ void __launch_bounds__(kThreads, 2) stats_kernel(const __grid_constan
             const float denom = S * g;
             float inv = denom > 0.0f ? 1.0f / denom : 0.0f;
             inv = fminf(inv, FLT_MAX);
+            const uint64_t inv2 = pk(inv, inv), S2 = pk(S, S), g2 = pk(g, g);
+            uint64_t e2 = 0;
 #pragma unroll
-            for (int e = 0; e < 16; ++e) {
-              // x_hat rounded to FP32 on its own (no contraction into the subtraction)
-              const float xh = __fmul_rn(__fmul_rn(e2m1_round(v[e] * inv), S), g);
-              const float d = v[e] - xh;
-              re2 += d * d;
+            for (int e = 0; e < 16; e += 2) {
+              const uint64_t xv = pk(v[e], v[e + 1]);
+              const float2 c = e2m1_round2(upk(mul2(xv, inv2)));
+              // x_hat = (e2m1 * S) * g, each product rounded on its own
+              const uint64_t xh = mul2(mul2(pk(c.x, c.y), S2), g2);
+              const uint64_t d = add2(xv, xh ^ 0x8000000080000000ull);  // x - x_hat
+              e2 = fma2(d, d, e2);
             }
+            const float2 fe = upk(e2);
+            re2 = fe.x + fe.y;
           }
         }
         rn2 = warp_sumf(rn2);

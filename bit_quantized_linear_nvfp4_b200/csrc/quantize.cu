@@ -36,6 +36,7 @@
 #include <cstdint>
 
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
 #include "internal.h"
@@ -550,12 +551,6 @@ struct RequantArgs {
   int32_t old_begin[kMaxSeg + 1];
 };
 
-__device__ __forceinline__ float e2m1_value(uint32_t c) {
-  // twice the magnitudes 0, .5, 1, 1.5, 2, 3, 4, 6 as nibbles
-  const float v = static_cast<float>((0xC8643210u >> (4 * (c & 7u))) & 15u) * 0.5f;
-  return (c & 8u) ? -v : v;
-}
-
 __global__ void __launch_bounds__(kThreads, 1) requant_kernel(const __grid_constant__ RequantArgs r) {
   const QuantArgs& a = r.q;
   __shared__ float g_sh[kMaxSeg];
@@ -615,10 +610,21 @@ __global__ void __launch_bounds__(kThreads, 1) requant_kernel(const __grid_const
           if (k < r.nseg_old && rows[u] >= r.old_begin[k]) s = k;
         const float S = e4m3_value(sfb[u]), g = g_old_sh[s];
 #pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          const uint32_t word = e < 8 ? c[u].x : c[u].y;
-          const uint32_t code = (word >> (4 * (e & 7))) & 15u;
-          b.w[e] = __float_as_uint(__fmul_rn(e2m1_value(code) * S, g));  // e2m1 * S exact, one rounding
+        for (int h = 0; h < 2; ++h) {
+          // two codes per byte -> an exact FP16 pair (element 2j in the low half)
+          uint32_t h2[4];
+          asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\tmov.b32 {b0, b1, b2, b3}, %4;\n\t"
+              "cvt.rn.f16x2.e2m1x2 %0, b0;\n\tcvt.rn.f16x2.e2m1x2 %1, b1;\n\t"
+              "cvt.rn.f16x2.e2m1x2 %2, b2;\n\tcvt.rn.f16x2.e2m1x2 %3, b3;\n\t}"
+              : "=r"(h2[0]), "=r"(h2[1]), "=r"(h2[2]), "=r"(h2[3])
+              : "r"(h ? c[u].y : c[u].x));
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&h2[q]));
+            // e2m1 * S is exact; one rounding for the global scale
+            b.w[8 * h + 2 * q] = __float_as_uint(__fmul_rn(f.x * S, g));
+            b.w[8 * h + 2 * q + 1] = __float_as_uint(__fmul_rn(f.y * S, g));
+          }
         }
       }
       quantize_block<NVFP4_DTYPE_F32>(a, g_sh, b, have[u], rows[u], cols[u]);
