@@ -31,9 +31,22 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 FP4_PER_BF16 = 4.0  # nominal dense ratio: 9 PF FP4 / 2.25 PF BF16
 ROTATE = 4          # rotating input sets so consecutive steps miss in L2
 # DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) per launch of the
-# dominant kernel, from one ncu capture of the kernel as it is now; None once
-# the kernel changes until it is captured again.
-TRAFFIC_BYTES = {}
+# dominant kernel, from one ncu capture of the kernel as it is now (the
+# commands are in profiles/); an entry is removed when its kernel changes,
+# until it is captured again.  "quant": both passes, captured on X[8192, 17408]
+# and scaled by 4 rows-wise (the traffic grows with the rows).
+TRAFFIC_BYTES = {
+    "actstats": 339406592,
+    "decode1": 50362112,
+    "decode64": 50922752,
+    "decode8": 50422528,
+    "gdn": 1401560576,
+    "kvfp8": 73506560,
+    "mlp": 381300224,
+    "oproj": 28804864,
+    "quant": 2563600000,
+    "requant": 36475136,
+}
 
 
 def load_peaks():
@@ -347,7 +360,13 @@ def run_product(args):
     kernels = {"quantize_stage_ms": q_ms,
                "quantize_stage_gbs": (qb["amax"] + qb["quantize"]) / (q_ms * 1e-3) / 1e9,
                "quantize_stage_frac_hbm": (qb["amax"] + qb["quantize"]) / (q_ms * 1e-3) / 1e9 / hbm}
-    if step.w is not None:
+    if step.w is not None and args.workload.startswith("decode"):
+        # few tokens: the GEMM streams W from HBM, so its roofline is bandwidth
+        gbs = step.alg_bytes_gemm() / (g_ms * 1e-3) / 1e9
+        roof = {"bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s", "frac": gbs / hbm,
+                "traffic": TRAFFIC_BYTES.get(args.workload), "peak_source": f"{peak_src} copy bandwidth",
+                "kernel": "nvfp4 decode gemm (tcgen05 mxf4nvf4, split-K cluster)", "ms_per_launch": g_ms}
+    elif step.w is not None:
         fp4_peak = float(peaks["bf16_tflops_sustained"]) * FP4_PER_BF16
         ach = step.flops / (g_ms * 1e-3) / 1e12
         roof = {"bound": "tensor", "achieved": ach, "peak": fp4_peak, "unit": "TFLOP/s",
@@ -364,7 +383,7 @@ def run_product(args):
         bytes_step = qb["amax"] + qb["quantize"]
         ach = bytes_step / (q_ms * 1e-3) / 1e9
         roof = {"bound": "hbm", "achieved": ach, "peak": hbm, "unit": "GB/s", "frac": ach / hbm,
-                "traffic": None, "peak_source": f"{peak_src} copy bandwidth",
+                "traffic": TRAFFIC_BYTES.get(args.workload), "peak_source": f"{peak_src} copy bandwidth",
                 "kernel": "nvfp4 amax + quantize", "ms_per_launch": q_ms}
         value = bytes_step * world / (ms_step * 1e-3) / 1e9
         unit = "GB/s"
