@@ -24,7 +24,12 @@ Readings taken where the pages are silent (each one is listed in the design doc):
   * g <= 0 (an all-zero tensor) gives all-zero codes and scale bytes;
   * GEMM and epilogues in FP64 on the dequantised operands;
   * decay gate: g = -exp(A_log[h]) * softplus(y + dt_bias[h]), head h = column
-    within the segment; SwiGLU: silu(gate) * up.
+    within the segment; SwiGLU: silu(gate) * up;
+  * delta-rule recurrence (the consumer of the projection's q, k, v, beta, g):
+    one state S[d_v, d_k] per value head, alpha = exp(g),
+    S_t = alpha_t S_{t-1} + beta_t (v_t - alpha_t S_{t-1} k_t) k_t^T and
+    o_t = S_t q_t, with k and q L2-normalised per head (x / sqrt(sum x^2 + eps))
+    and q scaled by d_k^-1/2; value head h reads query/key head h // (H / H_k).
 
 Parity pins for every function live in tests/test_oracle_*.py.
 """
@@ -384,6 +389,67 @@ def activation_summary(st: dict) -> dict:
             "a4_err_min": float(err.min()) if err.size else 0.0,
             "a4_err_max": float(err.max()) if err.size else 0.0,
             "hot_channel_ratio": float(col_rms.max() / med) if med > 0 else 0.0}
+
+
+# --------------------------------------------------------------------------
+# Gated delta-rule recurrence (Paper summary page (ai.info), "Main Findings",
+# recurrence bullet: a fixed-size state in which every write overwrites along
+# the current key direction, with a decay alpha and a write strength beta;
+# gate-parameterisation bullet: alpha comes from the log-space decay gate g,
+# alpha = exp(g)).  The plain token-by-token definition, in FP64.
+# --------------------------------------------------------------------------
+
+
+def l2_normalise(x: np.ndarray, eps: float = 1e-6) -> np.ndarray:
+    """x / sqrt(sum(x^2) + eps) along the last axis, FP64."""
+    x = np.asarray(x, dtype=np.float64)
+    return x / np.sqrt((x * x).sum(axis=-1, keepdims=True) + eps)
+
+
+def gdn_recurrence(q, k, v, beta, g, h0=None, scale=None, eps=1e-6, normalise=True, row_norms=False):
+    """Run the gated delta rule over T tokens.
+
+    q, k: [T, H_k, d_k]; v: [T, H, d_v]; beta, g: [T, H] (write strength and
+    log-space decay, as the projection's epilogue emits them); h0: [H, d_v, d_k]
+    or None (zeros).  Value head h uses query/key head h // (H / H_k).
+    Returns (o [T, H, d_v], S_T [H, d_v, d_k]) and, with row_norms, also
+    |S_t[i, :]|_2 for every token ([T, H, d_v]): the natural size of o_t[i],
+    since |o_t[i]| <= |S_t[i, :]| * |q_t|.
+
+    Per token, with alpha = exp(g_t):
+        u   = beta_t * (v_t - alpha * S_{t-1} k_t)      (the correction written)
+        S_t = alpha * S_{t-1} + u k_t^T
+        o_t = S_t q_t
+    which is S_t = alpha S_{t-1} (I - beta k k^T) + beta v k^T written out."""
+    q = np.asarray(q, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    beta = np.asarray(beta, dtype=np.float64)
+    g = np.asarray(g, dtype=np.float64)
+    T, H, dv = v.shape
+    hk, dk = q.shape[1], q.shape[2]
+    assert k.shape == q.shape and H % hk == 0 and beta.shape == (T, H) and g.shape == (T, H)
+    rep = H // hk
+    qh = np.repeat(q, rep, axis=1)
+    kh = np.repeat(k, rep, axis=1)
+    if normalise:
+        qh = l2_normalise(qh, eps)
+        kh = l2_normalise(kh, eps)
+    qh = qh * (dk ** -0.5 if scale is None else scale)
+    S = np.zeros((H, dv, dk)) if h0 is None else np.array(h0, dtype=np.float64)
+    o = np.empty((T, H, dv))
+    rn = np.empty((T, H, dv)) if row_norms else None
+    for t in range(T):
+        a = np.exp(g[t])
+        Sk = np.einsum("hvk,hk->hv", S, kh[t])
+        u = beta[t][:, None] * (v[t] - a[:, None] * Sk)
+        S = a[:, None, None] * S + u[:, :, None] * kh[t][:, None, :]
+        o[t] = np.einsum("hvk,hk->hv", S, qh[t])
+        if row_norms:
+            rn[t] = np.sqrt((S * S).sum(axis=2))
+    if row_norms:
+        return o, S, rn
+    return o, S
 
 
 def bf16_round(y) -> np.ndarray:
