@@ -208,6 +208,8 @@ class ProductStep:
             "codes": torch.empty((M, K // 2), dtype=torch.uint8, device=self.device),
             "sf": torch.empty(nv.nvfp4_sf_bytes(M, K), dtype=torch.uint8, device=self.device),
             "g": torch.empty(1, dtype=torch.float32, device=self.device),
+            # calibrated static activation scale for the one-pass leg (set in capture())
+            "gs": torch.empty(1, dtype=torch.float32, device=self.device),
             "ws": torch.empty(nv.nvfp4_quantize_workspace_bytes(1), dtype=torch.uint8, device=self.device),
         }
         s["A"] = nv.Operand(s["codes"], s["sf"], M, K)
@@ -246,17 +248,29 @@ class ProductStep:
         self.nv.nvfp4_linear(s["x"], s["W"], s["gw"], s["segs"], a_codes=s["codes"], a_sf=s["sf"],
                              g_a=s["g"], workspace=s["ws"])
 
+    # one-pass forms: a calibrated static activation scale is given, so the
+    # amax pass is skipped (quantiser alone, and the whole layer call)
+    def quantize_static(self, s):
+        self.nv.nvfp4_quantize(s["x"], s["gs"], codes=s["codes"], sf=s["sf"], g_out=s["g"])
+
+    def linear_static(self, s):
+        self.nv.nvfp4_linear(s["x"], s["W"], s["gw"], s["segs"], s["gs"], a_codes=s["codes"], a_sf=s["sf"],
+                             g_a=s["g"])
+
     def launches_per_step(self):
         return 2 if self.w is None else 3  # amax, quantize (+ GEMM)
 
     def capture(self):
         torch = self.torch
-        self.gq, self.gg, self.gl = [], [], []
+        self.gq, self.gg, self.gl, self.gqs, self.gls = [], [], [], [], []
         for s in self.sets:  # warm the launch path once outside capture
             self.quantize(s)
+            s["gs"].copy_(s["g"])  # "calibration": this input's own amax scale, fixed from here on
+            self.quantize_static(s)
             if self.w is not None:
                 self.gemm(s)
                 self.linear(s)
+                self.linear_static(s)
         torch.cuda.synchronize()
 
         def graph(fn, s):
@@ -267,9 +281,11 @@ class ProductStep:
 
         for s in self.sets:
             self.gq.append(graph(self.quantize, s))
+            self.gqs.append(graph(self.quantize_static, s))
             if self.w is not None:
                 self.gg.append(graph(self.gemm, s))
                 self.gl.append(graph(self.linear, s))
+                self.gls.append(graph(self.linear_static, s))
         torch.cuda.synchronize()
 
     def step_graph(self, r):
@@ -343,6 +359,23 @@ def run_product(args):
     for i in range(K):
         staged(i, evs[i])
     torch.cuda.synchronize()
+
+    def replay_ms(graphs):
+        # K replays of one graph form, after a short warm-up
+        for i in range(min(Wm, 3)):
+            graphs[i % R].replay()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for i in range(K):
+            graphs[i % R].replay()
+        b.record(stream)
+        torch.cuda.synchronize()
+        return a.elapsed_time(b) / K
+
+    # one-pass (calibrated static scale) forms beside the two-pass ones
+    q1_ms = replay_ms(step.gqs)
+    l1_ms = replay_ms(step.gls) if step.w is not None else None
     clk = clocks.stop()
     total_ms = t0.elapsed_time(t1)
     total_ms = dist_max(dist, total_ms, device)
@@ -359,7 +392,14 @@ def run_product(args):
     hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
     kernels = {"quantize_stage_ms": q_ms,
                "quantize_stage_gbs": (qb["amax"] + qb["quantize"]) / (q_ms * 1e-3) / 1e9,
-               "quantize_stage_frac_hbm": (qb["amax"] + qb["quantize"]) / (q_ms * 1e-3) / 1e9 / hbm}
+               "quantize_stage_frac_hbm": (qb["amax"] + qb["quantize"]) / (q_ms * 1e-3) / 1e9 / hbm,
+               "quantize_one_pass_ms": q1_ms,
+               "quantize_one_pass_gbs": qb["quantize"] / (q1_ms * 1e-3) / 1e9,
+               "quantize_one_pass_frac_hbm": qb["quantize"] / (q1_ms * 1e-3) / 1e9 / hbm}
+    if l1_ms is not None:
+        kernels["layer_one_pass_ms"] = l1_ms
+        kernels["layer_two_pass_ms"] = ms_step
+        kernels["layer_one_pass_tflops"] = step.flops / (l1_ms * 1e-3) / 1e12
     if step.w is not None and args.workload.startswith("decode"):
         # few tokens: the GEMM streams W from HBM, so its roofline is bandwidth
         gbs = step.alg_bytes_gemm() / (g_ms * 1e-3) / 1e9
@@ -403,7 +443,7 @@ def run_product(args):
         line["cpu_baseline"] = cpu_baseline(args.workload, target_s=args.cpu_seconds)
     if rank == 0:
         print(json.dumps(line), flush=True)
-    for g in step.gq + step.gg + step.gl:
+    for g in step.gq + step.gg + step.gl + step.gqs + step.gls:
         del g
     if dist is not None:
         dist.destroy_process_group()
