@@ -899,9 +899,173 @@ def run_actstats(args):
         dist.destroy_process_group()
 
 
+GDN_REC_TOKENS = 32768  # the GDN projection's prefill length
+
+
+def gdnrec_alg_bytes(T, H, H_k=None):
+    """Bytes the delta-rule recurrence must move: q and k (BF16, 64 per head),
+    v (BF16, 128 per head), beta and g (FP32), the BF16 output and the final
+    FP32 state."""
+    H_k = H if H_k is None else H_k
+    per_token = 2 * (2 * H_k * 64) + 2 * H * 128 + 2 * 4 * H + 2 * H * 128
+    return T * per_token + H * 128 * 64 * 4
+
+
+def gdnrec_tensor_macs(T, H):
+    """MACs the chunked kernels issue per step (TF32 m16n8k8 MMAs, 1024 MACs each):
+    2016 per (chunk, head) in the per-chunk pass and 1024 in the state pass."""
+    return -(-T // 64) * H * (2016 + 1024) * 1024
+
+
+def run_gdnrec(args):
+    """Delta-rule recurrence over the fused GDN projection's outputs at
+    long-context prefill: q, k [32768, 32 x 64], v [32768, 32 x 128] BF16,
+    beta and g [32768, 32] FP32, as the projection's epilogue writes them (one
+    untimed layer call produces them); one nvfp4_gdn_recurrence call per step
+    (two launches), BF16 output and the final state.  Inputs (545 MB) are
+    larger than L2."""
+    import torch
+    from bit_quantized_linear_nvfp4_b200 import nvfp4 as nv
+    from bit_quantized_linear_nvfp4_b200 import workloads as wl
+    world, rank, local = dist_env()
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    dist = dist_init(world)
+    peaks, peak_src = load_peaks()
+    w = wl.GDN
+    T, H = GDN_REC_TOKENS, wl.GDN_HEADS
+    proj = ProductStep("gdn", device)
+    s0 = proj.sets[0]
+    proj.linear(s0)
+    torch.cuda.synchronize()
+    q, k, v, _, beta, g = s0["outs"]
+    for extra in proj.sets[1:]:
+        extra.clear()
+    proj.sets = [s0]
+    out = torch.empty((T, H * 128), dtype=torch.bfloat16, device=device)
+    h_out = torch.empty((H, 128, 64), dtype=torch.float32, device=device)
+    ws = torch.empty(nv.nvfp4_gdn_workspace_bytes(T, H), dtype=torch.uint8, device=device)
+    stream = torch.cuda.current_stream()
+
+    def call():
+        nv.nvfp4_gdn_recurrence(q, k, v, beta, g, out=out, h_out=h_out, workspace=ws)
+
+    call()
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        call()
+    Kst, Wm = args.steps, args.warmup
+    for _ in range(Wm):
+        graph.replay()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    dist_barrier(dist)
+    torch.cuda.synchronize()
+    t0.record(stream)
+    for _ in range(Kst):
+        graph.replay()
+    t1.record(stream)
+    torch.cuda.synchronize()
+    dist_barrier(dist)
+    clk = clocks.stop()
+    ms = dist_max(dist, t0.elapsed_time(t1), device) / Kst
+    nv.nvfp4_check()
+    bytes_step = gdnrec_alg_bytes(T, H)
+    hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    ach = bytes_step / (ms * 1e-3) / 1e9
+    macs = gdnrec_tensor_macs(T, H)
+    tf32_peak = float(peaks["bf16_tflops_sustained"]) / 2.0
+    # end to end: q, k, v, beta, g from pinned host memory, output and state back
+    h_in = [t.cpu().pin_memory() for t in (q, k, v, beta, g)]
+    h_res = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in (out, h_out)]
+
+    def e2e_one():
+        for d, hh in zip((q, k, v, beta, g), h_in):
+            d.copy_(hh, non_blocking=True)
+        graph.replay()
+        for hh, d in zip(h_res, (out, h_out)):
+            hh.copy_(d, non_blocking=True)
+
+    for _ in range(Wm):
+        e2e_one()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(Kst):
+        e2e_one()
+    b.record(stream)
+    torch.cuda.synchronize()
+    ms_e2e = a.elapsed_time(b) / Kst
+    line = {
+        "metric": METRIC, "value": bytes_step * world / (ms * 1e-3) / 1e9, "unit": "GB/s", "n_gpus": world,
+        "steps": Kst, "warmup": Wm, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "tf32 products, f32 state (bf16 in/out)",
+        "data": "synthetic (the GDN projection's outputs on seeded N(0,1) activations and N(0,0.02) weights)",
+        "config": {"workload": f"gdn_recurrence_{T}x{H}h_dk64_dv128", "tokens": T, "heads": H, "d_k": 64,
+                   "d_v": 128, "chunk": 64, "parallelism": "replicas" if world > 1 else "single",
+                   "l2": "inputs (545 MB) larger than the 126 MB L2"},
+        "roofline": {"bound": "hbm", "achieved": ach, "peak": hbm, "unit": "GB/s", "frac": ach / hbm,
+                     "traffic": TRAFFIC_BYTES.get("gdnrec"), "peak_source": f"{peak_src} copy bandwidth",
+                     "kernel": "gdn recurrence (per-chunk pass + state pass)", "ms_per_launch": ms},
+        "kernels": {"tensor_macs_per_step": macs, "tensor_tflops": 2 * macs / (ms * 1e-3) / 1e12,
+                    "tf32_peak_tflops": tf32_peak, "workspace_bytes": ws.numel()},
+        "clocks": clk,
+        "e2e": {"value": bytes_step / (ms_e2e * 1e-3) / 1e9, "unit": "GB/s",
+                "h2d_bytes_per_step": sum(t.numel() * t.element_size() for t in h_in),
+                "d2h_bytes_per_step": sum(t.numel() * t.element_size() for t in h_res), "ms_per_step": ms_e2e},
+        "gpu_launches": 2 * Kst,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = _gdnrec_oracle_baseline(args.cpu_seconds / 2)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    del graph
+    if dist is not None:
+        dist.destroy_process_group()
+
+
+def _gdnrec_oracle_baseline(seconds, steps=None):
+    """The oracle's token loop on a bounded sample: 4 heads x 2048 tokens of
+    seeded inputs with the recurrence's shapes, per pass."""
+    from bit_quantized_linear_nvfp4_b200 import workloads as wl
+    from oracle import nvfp4_oracle as o
+    T, H = 2048, 4
+    q, k, v, beta, g = wl.make_recurrence_inputs(T, H, H, 3)
+    args = (q.reshape(T, H, 64), k.reshape(T, H, 64), v.reshape(T, H, 128), beta, g)
+    t = time.perf_counter()
+    n = 0
+    while (steps is None and (time.perf_counter() - t < seconds or n == 0)) or (steps is not None and n < steps):
+        o.gdn_recurrence(*args)
+        n += 1
+    per = (time.perf_counter() - t) / n
+    val = gdnrec_alg_bytes(T, H) / per / 1e9
+    return {"value": val, "unit": "GB/s", "cores": _blas_threads(), "kind": "oracle",
+            "sample": f"{H} heads x {T} tokens per pass ({n} passes, oracle token loop)", "ms_per_pass": per * 1e3,
+            "host_cpus": os.cpu_count()}
+
+
 def run_reference(args):
     world, rank, _ = dist_env()
     if rank != 0:
+        return
+    if args.workload == "gdnrec":
+        for _ in range(min(args.warmup, 1)):
+            _gdnrec_oracle_baseline(0.0, steps=1)
+        cb = _gdnrec_oracle_baseline(0.0, steps=max(1, min(args.steps, 20)))
+        val = cb["value"]
+        print(json.dumps({"impl": "reference", "metric": METRIC, "value": val, "unit": "GB/s", "n_gpus": world,
+                          "steps": args.steps, "warmup": args.warmup, "ms_per_step": cb["ms_per_pass"],
+                          "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+                          "dtype": "f64 (oracle)", "data": "synthetic",
+                          "config": {"workload": f"gdn_recurrence_{GDN_REC_TOKENS}x32h_dk64_dv128",
+                                     "tokens": GDN_REC_TOKENS, "heads": 32},
+                          "cpu_baseline": cb,
+                          "e2e": {"value": val, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}),
+              flush=True)
         return
     if args.workload == "actstats":
         from bit_quantized_linear_nvfp4_b200 import workloads as wl
@@ -1010,7 +1174,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--workload", default="oproj",
                     choices=["oproj", "mlp", "gdn", "tiny", "decode1", "decode8", "decode64", "quant", "requant",
-                             "kvfp8", "actstats"])
+                             "kvfp8", "actstats", "gdnrec"])
     ap.add_argument("--impl", default="product", choices=["product", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
@@ -1027,6 +1191,8 @@ def main():
         run_kvfp8(args)
     elif args.workload == "actstats":
         run_actstats(args)
+    elif args.workload == "gdnrec":
+        run_gdnrec(args)
     else:
         run_product(args)
 

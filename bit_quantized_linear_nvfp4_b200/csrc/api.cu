@@ -377,6 +377,96 @@ int nvfp4_gemm(const nvfp4_operand* A, const float* g_a, const nvfp4_operand* W,
   return nvfp4_fused_proj(A, g_a, W, g_w, &seg, 1, workspace, workspace_bytes, stream);
 }
 
+size_t nvfp4_gdn_workspace_bytes(int64_t T, int64_t H) {
+  if (T <= 0 || H <= 0) return 0;
+  return nvfp4::gdn_workspace_bytes(T, H);
+}
+
+int nvfp4_gdn_recurrence(const void* q, const void* k, const void* v, int in_dtype, int64_t T, int64_t H,
+                         int64_t H_k, int64_t d_k, int64_t d_v, int64_t ld_q, int64_t ld_k, int64_t ld_v,
+                         const float* beta, int64_t ld_beta, const float* g, int64_t ld_g, float scale,
+                         const float* h0, float* h_out, void* o, int out_dtype, int64_t ld_o,
+                         void* workspace, size_t workspace_bytes, void* stream) {
+  if (in_dtype != NVFP4_DTYPE_BF16 && in_dtype != NVFP4_DTYPE_F32) return NVFP4_ERR_INVALID_ARG;
+  if (out_dtype != NVFP4_DTYPE_BF16 && out_dtype != NVFP4_DTYPE_F32) return NVFP4_ERR_INVALID_ARG;
+  if (T < 0 || H <= 0 || H_k <= 0 || H % H_k != 0) return NVFP4_ERR_INVALID_ARG;
+  if (!(scale >= 0.0f) || scale > 3.4028234663852886e38f) return NVFP4_ERR_INVALID_ARG;
+  if (d_k != 64 || d_v != 128) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+  if (H > 65535 || nvfp4::ceil_div(T, 64) > (int64_t(1) << 31) - 1) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+  const size_t state_bytes = static_cast<size_t>(H) * 128 * 64 * sizeof(float);
+  if ((reinterpret_cast<uintptr_t>(h0) & 3u) != 0 || (reinterpret_cast<uintptr_t>(h_out) & 3u) != 0)
+    return NVFP4_ERR_MISALIGNED;
+  if (h_out != nullptr && h0 != nullptr && h_out != h0 && overlap(h_out, state_bytes, h0, state_bytes))
+    return NVFP4_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (T == 0) {
+    if (h_out == nullptr || h_out == h0) return NVFP4_OK;
+    int st = check_device();
+    if (st != NVFP4_OK) return st;
+    cudaError_t e = h0 ? cudaMemcpyAsync(h_out, h0, state_bytes, cudaMemcpyDeviceToDevice, s)
+                       : cudaMemsetAsync(h_out, 0, state_bytes, s);
+    if (e != cudaSuccess) return cuda_fail(e);
+    return NVFP4_OK;
+  }
+  if (q == nullptr || k == nullptr || v == nullptr || beta == nullptr || g == nullptr || o == nullptr)
+    return NVFP4_ERR_INVALID_ARG;
+  if (ld_q < H_k * 64 || ld_k < H_k * 64 || ld_v < H * 128 || ld_o < H * 128 || ld_beta < H || ld_g < H)
+    return NVFP4_ERR_INVALID_ARG;
+  const int esz = in_dtype == NVFP4_DTYPE_BF16 ? 2 : 4, osz = out_dtype == NVFP4_DTYPE_BF16 ? 2 : 4;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || (ld_q * esz) % 16 != 0 ||
+      (ld_k * esz) % 16 != 0 || (ld_v * esz) % 16 != 0 || (ld_o * osz) % 16 != 0)
+    return NVFP4_ERR_MISALIGNED;
+  if ((reinterpret_cast<uintptr_t>(beta) & 3u) != 0 || (reinterpret_cast<uintptr_t>(g) & 3u) != 0)
+    return NVFP4_ERR_MISALIGNED;
+  const size_t ws_need = nvfp4::gdn_workspace_bytes(T, H);
+  if (workspace == nullptr || workspace_bytes < ws_need || !aligned16(workspace)) return NVFP4_ERR_WORKSPACE;
+  // o and the workspace are written: neither may overlap anything read
+  const size_t nq = static_cast<size_t>((T - 1) * ld_q + H_k * 64) * esz;
+  const size_t nk = static_cast<size_t>((T - 1) * ld_k + H_k * 64) * esz;
+  const size_t nv = static_cast<size_t>((T - 1) * ld_v + H * 128) * esz;
+  const size_t nb = static_cast<size_t>((T - 1) * ld_beta + H) * sizeof(float);
+  const size_t ng = static_cast<size_t>((T - 1) * ld_g + H) * sizeof(float);
+  const size_t no = static_cast<size_t>((T - 1) * ld_o + H * 128) * osz;
+  const void* written[3] = {o, workspace, h_out};
+  const size_t wbytes[3] = {no, ws_need, h_out ? state_bytes : 0};
+  for (int i = 0; i < 3; ++i) {
+    if (overlap(written[i], wbytes[i], q, nq) || overlap(written[i], wbytes[i], k, nk) ||
+        overlap(written[i], wbytes[i], v, nv) || overlap(written[i], wbytes[i], beta, nb) ||
+        overlap(written[i], wbytes[i], g, ng))
+      return NVFP4_ERR_INVALID_ARG;
+    for (int j = i + 1; j < 3; ++j)
+      if (overlap(written[i], wbytes[i], written[j], wbytes[j])) return NVFP4_ERR_INVALID_ARG;
+    if (i < 2 && overlap(written[i], wbytes[i], h0, h0 ? state_bytes : 0)) return NVFP4_ERR_INVALID_ARG;
+  }
+  int st = check_device();
+  if (st != NVFP4_OK) return st;
+  nvfp4::GdnProblem p{};
+  p.q = q;
+  p.k = k;
+  p.v = v;
+  p.in_dtype = in_dtype;
+  p.T = T;
+  p.H = H;
+  p.H_k = H_k;
+  p.ld_q = ld_q;
+  p.ld_k = ld_k;
+  p.ld_v = ld_v;
+  p.beta = beta;
+  p.g = g;
+  p.ld_beta = ld_beta;
+  p.ld_g = ld_g;
+  p.scale = scale == 0.0f ? 0.125f : scale;  // d_k^-1/2 for d_k = 64
+  p.h0 = h0;
+  p.h_out = h_out;
+  p.o = o;
+  p.out_dtype = out_dtype;
+  p.ld_o = ld_o;
+  p.workspace = workspace;
+  cudaError_t e = nvfp4::launch_gdn(p, s);
+  if (e != cudaSuccess) return cuda_fail(e);
+  return NVFP4_OK;
+}
+
 int nvfp4_check(void* stream) {
   cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e);

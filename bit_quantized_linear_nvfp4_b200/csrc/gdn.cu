@@ -1,0 +1,626 @@
+// Gated delta-rule recurrence over the fused projection's outputs, sm_100a.
+//
+// "Why Gated DeltaNet Survives 4-Bit Quantization" (ai.info summary), "Main
+// Findings", recurrence bullet: a fixed-size state per head, every write
+// overwrites along the current key, with a decay alpha and a write strength
+// beta; gate-parameterisation bullet: the decay gate is emitted in log space
+// (g = -exp(A_log) softplus(a + dt_bias)), so alpha = exp(g).  Per value head,
+// with the state S [d_v, d_k] in FP32 and q, k L2-normalised (q also scaled):
+//     S_t = alpha_t S_{t-1} + beta_t (v_t - alpha_t S_{t-1} k_t) k_t^T,
+//     o_t = S_t q_t.
+//
+// Chunked evaluation, C = 64 tokens per chunk.  With S the state entering a
+// chunk and gam the inclusive running sum of g inside it:
+//     A[t][j] = beta_t e^(gam_t - gam_j) k_t.k_j   (j < t),   L = (I + A)^-1
+//     W = L diag(beta e^gam) K,     U~ = L diag(beta) V
+//     P[t][j] = e^(gam_t - gam_j) q_t.k_j          (j <= t)
+//     Kd = diag(e^(gam_C - gam)) K
+//     M = e^gam_C I - W^T Kd,  N = U~^T Kd,  R = diag(e^gam) Q - P W,  Y = P U~
+//     S' = S M + N,   O = R S^T + Y.
+// (Unrolling the token recurrence over the chunk gives these: the corrections
+// u_t written inside the chunk solve (I + A) U = diag(beta) (V - diag(e^gam) K S^T).)
+// Only the last line depends on S.  gdn_prep_kernel builds [M^T; R], N and
+// Y^T for every (chunk, head) at once; gdn_state_kernel then walks the chunks
+// in order, one CTA per (head, 32 state rows) -- rows of S evolve
+// independently -- keeping S in shared memory.
+//
+// The contractions run on the tensor cores as warp-level TF32 MMAs
+// (m16n8k8, FP32 accumulate): every product here is a 64-wide tile inside a
+// chain of dependent steps (Gram matrix -> triangular solve -> products ->
+// state), where register fragments avoid a round trip through tensor memory
+// between steps.  Operands are rounded to TF32 (nearest, ties away); the
+// triangular solve, the state and all sums stay FP32.
+#include <cstdint>
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "internal.h"
+#include "ptx.cuh"
+
+namespace nvfp4 {
+namespace gdn {
+
+constexpr int C = 64;        // tokens per chunk
+constexpr int DK = 64;       // key / query head dimension
+constexpr int DV = 128;      // value head dimension
+constexpr int LD64 = 68;     // padded row stride (floats) of 64-wide tiles in shared memory
+constexpr int LD128 = 132;   // of 128-wide tiles
+constexpr int kThreads = 256;
+constexpr int kRows = 32;    // state rows per CTA of the state pass
+constexpr int kRec = 3 * 128 * 64;  // floats per (chunk, head) record: [M^T; R], N, Y^T
+
+struct GdnArgs {
+  const uint8_t* q;
+  const uint8_t* k;
+  const uint8_t* v;
+  int64_t ld_q, ld_k, ld_v;  // bytes
+  const float* beta;
+  const float* g;
+  int64_t ld_beta, ld_g;     // elements
+  int64_t T;
+  int H, rep;                // value heads; value heads per query/key head
+  int nchunks;
+  float scale, eps;
+  const float* h0;           // [H, DV, DK] or null
+  float* h_out;              // [H, DV, DK] or null
+  uint8_t* o;
+  int64_t ld_o;              // bytes
+  int out_f32;
+  float* ws;                 // nchunks * H records
+};
+
+__device__ __forceinline__ uint32_t tf32(float x) {
+  uint32_t r;
+  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+  return r;
+}
+
+// D += A B, m16n8k8, A row-major 16x8, B 8x8 (k rows), TF32 in, FP32 accumulate.
+__device__ __forceinline__ void mma(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+      "{%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// Fragment loaders.  gid = lane / 4, tig = lane % 4.  An A fragment holds
+// (m0+gid, k0+tig), (m0+gid+8, k0+tig), (m0+gid, k0+tig+4), (m0+gid+8, k0+tig+4);
+// a B fragment (k0+tig, n0+gid), (k0+tig+4, n0+gid); the accumulator
+// (m0+gid, n0+2tig), (m0+gid, n0+2tig+1), (m0+gid+8, n0+2tig), (m0+gid+8, n0+2tig+1).
+
+// A[m][k] = X[m][k] (X row-major, stride ld).
+__device__ __forceinline__ void frag_a(uint32_t (&a)[4], const float* X, int ld, int m0, int k0, int gid, int tig) {
+  a[0] = tf32(X[(m0 + gid) * ld + k0 + tig]);
+  a[1] = tf32(X[(m0 + gid + 8) * ld + k0 + tig]);
+  a[2] = tf32(X[(m0 + gid) * ld + k0 + tig + 4]);
+  a[3] = tf32(X[(m0 + gid + 8) * ld + k0 + tig + 4]);
+}
+// A[m][k] = s[k] X[k][m] (X stored with k as the row).
+__device__ __forceinline__ void frag_at(uint32_t (&a)[4], const float* X, int ld, const float* s, int m0, int k0,
+                                        int gid, int tig) {
+  const float s0 = s ? s[k0 + tig] : 1.0f, s1 = s ? s[k0 + tig + 4] : 1.0f;
+  a[0] = tf32(s0 * X[(k0 + tig) * ld + m0 + gid]);
+  a[1] = tf32(s0 * X[(k0 + tig) * ld + m0 + gid + 8]);
+  a[2] = tf32(s1 * X[(k0 + tig + 4) * ld + m0 + gid]);
+  a[3] = tf32(s1 * X[(k0 + tig + 4) * ld + m0 + gid + 8]);
+}
+// B[k][n] = X[n][k] (X stored with n as the row).
+__device__ __forceinline__ void frag_bt(uint32_t& b0, uint32_t& b1, const float* X, int ld, int n0, int k0, int gid,
+                                        int tig) {
+  b0 = tf32(X[(n0 + gid) * ld + k0 + tig]);
+  b1 = tf32(X[(n0 + gid) * ld + k0 + tig + 4]);
+}
+// B[k][n] = s[k] X[k][n] (X stored with k as the row).
+__device__ __forceinline__ void frag_b(uint32_t& b0, uint32_t& b1, const float* X, int ld, const float* s, int n0,
+                                       int k0, int gid, int tig) {
+  const float s0 = s ? s[k0 + tig] : 1.0f, s1 = s ? s[k0 + tig + 4] : 1.0f;
+  b0 = tf32(s0 * X[(k0 + tig) * ld + n0 + gid]);
+  b1 = tf32(s1 * X[(k0 + tig + 4) * ld + n0 + gid]);
+}
+
+// 16 consecutive elements (BF16 or F32) -> FP32.
+template <int DTYPE>
+__device__ __forceinline__ void load16(const uint8_t* p, float (&f)[16]) {
+  if constexpr (DTYPE == NVFP4_DTYPE_BF16) {
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const uint4 w = *reinterpret_cast<const uint4*>(p + 16 * h);
+      const uint32_t u[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        f[8 * h + 2 * i] = __uint_as_float(u[i] << 16);
+        f[8 * h + 2 * i + 1] = __uint_as_float(u[i] & 0xFFFF0000u);
+      }
+    }
+  } else {
+#pragma unroll
+    for (int h = 0; h < 4; ++h) {
+      const float4 w = *reinterpret_cast<const float4*>(p + 16 * h);
+      f[4 * h] = w.x;
+      f[4 * h + 1] = w.y;
+      f[4 * h + 2] = w.z;
+      f[4 * h + 3] = w.w;
+    }
+  }
+}
+
+struct PrepSmem {
+  float q[C * LD64];   // q^ (normalised and scaled)
+  float k[C * LD64];   // k^
+  float al[C * LD64];  // A, then L, then W
+  float p[C * LD64];   // P
+  float v[C * LD128];  // V, then U~
+  float gam[C];        // inclusive running sum of g
+  float beta[C];
+  float bg[C];         // beta e^gam
+  float eg[C];         // e^gam
+  float kdec[C];       // e^(gam_C - gam)
+};
+
+// One CTA per (chunk, value head): the S-independent matrices of the chunk.
+template <int DTYPE>
+__global__ void __launch_bounds__(kThreads, 2) gdn_prep_kernel(const __grid_constant__ GdnArgs a) {
+  extern __shared__ __align__(16) uint8_t smem_raw[];
+  PrepSmem& s = *reinterpret_cast<PrepSmem*>(smem_raw);
+  constexpr int kEsz = DTYPE == NVFP4_DTYPE_BF16 ? 2 : 4;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int gid = lane >> 2, tig = lane & 3;
+  const int c = blockIdx.x, h = blockIdx.y, hq = h / a.rep;
+  const int64_t t0 = static_cast<int64_t>(c) * C;
+
+  grid_dependency_wait();
+  if (tid == 0) grid_launch_dependents();
+
+  // ---- q, k rows: four threads per row, 16 elements each; L2 norms in FP32
+  {
+    const int row = tid >> 2, part = tid & 3;
+    const int64_t t = t0 + row;
+    float fq[16], fk[16];
+    if (t < a.T) {
+      load16<DTYPE>(a.q + t * a.ld_q + (static_cast<int64_t>(hq) * DK + part * 16) * kEsz, fq);
+      load16<DTYPE>(a.k + t * a.ld_k + (static_cast<int64_t>(hq) * DK + part * 16) * kEsz, fk);
+    } else {
+#pragma unroll
+      for (int i = 0; i < 16; ++i) fq[i] = fk[i] = 0.0f;
+    }
+    float sq = 0.0f, sk = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      sq = fmaf(fq[i], fq[i], sq);
+      sk = fmaf(fk[i], fk[i], sk);
+    }
+    sq += __shfl_xor_sync(0xffffffffu, sq, 1);
+    sk += __shfl_xor_sync(0xffffffffu, sk, 1);
+    sq += __shfl_xor_sync(0xffffffffu, sq, 2);
+    sk += __shfl_xor_sync(0xffffffffu, sk, 2);
+    const float iq = a.scale / sqrtf(sq + a.eps), ik = 1.0f / sqrtf(sk + a.eps);
+#pragma unroll
+    for (int i = 0; i < 16; i += 4) {
+      *reinterpret_cast<float4*>(&s.q[row * LD64 + part * 16 + i]) =
+          make_float4(fq[i] * iq, fq[i + 1] * iq, fq[i + 2] * iq, fq[i + 3] * iq);
+      *reinterpret_cast<float4*>(&s.k[row * LD64 + part * 16 + i]) =
+          make_float4(fk[i] * ik, fk[i + 1] * ik, fk[i + 2] * ik, fk[i + 3] * ik);
+    }
+    // ---- v rows: 32 elements per thread
+    float fv[16];
+#pragma unroll
+    for (int hh = 0; hh < 2; ++hh) {
+      const int col = part * 32 + hh * 16;
+      if (t < a.T) {
+        load16<DTYPE>(a.v + t * a.ld_v + (static_cast<int64_t>(h) * DV + col) * kEsz, fv);
+      } else {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) fv[i] = 0.0f;
+      }
+#pragma unroll
+      for (int i = 0; i < 16; i += 4)
+        *reinterpret_cast<float4*>(&s.v[row * LD128 + col + i]) = make_float4(fv[i], fv[i + 1], fv[i + 2], fv[i + 3]);
+    }
+  }
+  // ---- gates: running sum of the log decay inside the chunk (warp 0)
+  if (warp == 0) {
+    const int64_t ta = t0 + 2 * lane, tb = ta + 1;
+    const float ga = ta < a.T ? a.g[ta * a.ld_g + h] : 0.0f;
+    const float gb = tb < a.T ? a.g[tb * a.ld_g + h] : 0.0f;
+    const float ba = ta < a.T ? a.beta[ta * a.ld_beta + h] : 0.0f;
+    const float bb = tb < a.T ? a.beta[tb * a.ld_beta + h] : 0.0f;
+    const float pair = ga + gb;
+    float run = pair;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const float y = __shfl_up_sync(0xffffffffu, run, off);
+      if (lane >= off) run += y;
+    }
+    const float excl = run - pair;
+    const float gma = excl + ga, gmb = excl + ga + gb;
+    const float gC = __shfl_sync(0xffffffffu, gmb, 31);
+    s.gam[2 * lane] = gma;
+    s.gam[2 * lane + 1] = gmb;
+    s.beta[2 * lane] = ba;
+    s.beta[2 * lane + 1] = bb;
+    const float ea = expf(gma), eb = expf(gmb);
+    s.eg[2 * lane] = ea;
+    s.eg[2 * lane + 1] = eb;
+    s.bg[2 * lane] = ba * ea;
+    s.bg[2 * lane + 1] = bb * eb;
+    s.kdec[2 * lane] = expf(gC - gma);
+    s.kdec[2 * lane + 1] = expf(gC - gmb);
+  }
+  __syncthreads();
+
+  // ---- step 1: Gram matrices K K^T (-> A) and Q K^T (-> P), lower triangle
+  {
+    const int mat = warp >> 2, mt = warp & 3;
+    const float* X = mat == 0 ? s.k : s.q;
+    float* out = mat == 0 ? s.al : s.p;
+    uint32_t af[8][4];
+#pragma unroll
+    for (int ks = 0; ks < 8; ++ks) frag_a(af[ks], X, LD64, 16 * mt, 8 * ks, gid, tig);
+    for (int nt = 0; nt < 8; ++nt) {
+      float d[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+      if (nt < 2 * mt + 2) {
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks) {
+          uint32_t b0, b1;
+          frag_bt(b0, b1, s.k, LD64, 8 * nt, 8 * ks, gid, tig);
+          mma(d, af[ks], b0, b1);
+        }
+      }
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int t = 16 * mt + gid + (e >= 2 ? 8 : 0), j = 8 * nt + 2 * tig + (e & 1);
+        float val = 0.0f;
+        if (mat == 0) {
+          if (j < t) val = s.beta[t] * expf(s.gam[t] - s.gam[j]) * d[e];
+        } else {
+          if (j <= t) val = expf(s.gam[t] - s.gam[j]) * d[e];
+        }
+        out[t * LD64 + j] = val;
+      }
+    }
+  }
+  __syncthreads();
+
+  // ---- step 2: L = (I + A)^-1 by forward substitution, one column per thread
+  if (tid < C) {
+    const int j = tid;
+    float col[C];
+#pragma unroll
+    for (int i = 0; i < C; ++i) {
+      float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll
+      for (int m = 0; m + 4 <= i; m += 4) {
+        const float4 r = *reinterpret_cast<const float4*>(&s.al[i * LD64 + m]);
+        acc[0] = fmaf(r.x, col[m], acc[0]);
+        acc[1] = fmaf(r.y, col[m + 1], acc[1]);
+        acc[2] = fmaf(r.z, col[m + 2], acc[2]);
+        acc[3] = fmaf(r.w, col[m + 3], acc[3]);
+      }
+#pragma unroll
+      for (int m = (i / 4) * 4; m < i; ++m) acc[m & 3] = fmaf(s.al[i * LD64 + m], col[m], acc[m & 3]);
+      col[i] = (i == j ? 1.0f : 0.0f) - ((acc[0] + acc[1]) + (acc[2] + acc[3]));
+    }
+    asm volatile("bar.sync 1, 64;" ::: "memory");  // every thread is done reading A
+#pragma unroll
+    for (int i = 0; i < C; ++i) s.al[i * LD64 + j] = col[i];
+  }
+  __syncthreads();
+
+  // ---- step 3: W = L diag(beta e^gam) K  and  U~ = L diag(beta) V
+  {
+    const int mt = warp & 3, half = warp >> 2;
+    const int nks = 2 * mt + 2;  // L is lower triangular: k-steps past the diagonal block are zero
+    uint32_t af[8][4];
+#pragma unroll
+    for (int ks = 0; ks < 8; ++ks)
+      if (ks < nks) frag_a(af[ks], s.al, LD64, 16 * mt, 8 * ks, gid, tig);
+    float d[12][4];
+#pragma unroll
+    for (int i = 0; i < 12; ++i) d[i][0] = d[i][1] = d[i][2] = d[i][3] = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 12; ++i) {
+      const int nt = half * 12 + i;  // 0..7: W columns, 8..23: U~ columns
+#pragma unroll
+      for (int ks = 0; ks < 8; ++ks) {
+        if (ks >= nks) continue;
+        uint32_t b0, b1;
+        if (nt < 8) frag_b(b0, b1, s.k, LD64, s.bg, 8 * nt, 8 * ks, gid, tig);
+        else frag_b(b0, b1, s.v, LD128, s.beta, 8 * (nt - 8), 8 * ks, gid, tig);
+        mma(d[i], af[ks], b0, b1);
+      }
+    }
+    __syncthreads();  // L and V are read; W goes over L, U~ over V
+#pragma unroll
+    for (int i = 0; i < 12; ++i) {
+      const int nt = half * 12 + i;
+      const int r = 16 * mt + gid;
+      float* dst = nt < 8 ? &s.al[r * LD64 + 8 * nt + 2 * tig] : &s.v[r * LD128 + 8 * (nt - 8) + 2 * tig];
+      const int ld = nt < 8 ? LD64 : LD128;
+      *reinterpret_cast<float2*>(dst) = make_float2(d[i][0], d[i][1]);
+      *reinterpret_cast<float2*>(dst + 8 * ld) = make_float2(d[i][2], d[i][3]);
+    }
+  }
+  __syncthreads();
+
+  // ---- step 4: the record: [M^T; R] (128 x 64), N (128 x 64), Y^T (128 x 64)
+  float* rec = a.ws + (static_cast<int64_t>(c) * a.H + h) * kRec;
+  {
+    const float eC = s.eg[C - 1];
+    // M^T (warps 0-3) or R (warps 4-7): 16 rows each
+    {
+      const bool is_r = warp >= 4;
+      const int mt = warp & 3;
+      const int nks = is_r ? 2 * mt + 2 : 8;  // P is lower triangular
+      uint32_t af[8][4];
+#pragma unroll
+      for (int ks = 0; ks < 8; ++ks) {
+        if (ks >= nks) continue;
+        if (is_r) frag_a(af[ks], s.p, LD64, 16 * mt, 8 * ks, gid, tig);
+        else frag_at(af[ks], s.k, LD64, s.kdec, 16 * mt, 8 * ks, gid, tig);
+      }
+      float* dst = rec + (is_r ? 64 : 0) * 64;
+#pragma unroll
+      for (int nt = 0; nt < 8; ++nt) {
+        float d[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks) {
+          if (ks >= nks) continue;
+          uint32_t b0, b1;
+          frag_b(b0, b1, s.al, LD64, nullptr, 8 * nt, 8 * ks, gid, tig);
+          mma(d, af[ks], b0, b1);
+        }
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+          const int r = 16 * mt + gid + 8 * hh, col = 8 * nt + 2 * tig;
+          float v0, v1;
+          if (is_r) {
+            v0 = s.eg[r] * s.q[r * LD64 + col] - d[2 * hh];
+            v1 = s.eg[r] * s.q[r * LD64 + col + 1] - d[2 * hh + 1];
+          } else {
+            v0 = (r == col ? eC : 0.0f) - d[2 * hh];
+            v1 = (r == col + 1 ? eC : 0.0f) - d[2 * hh + 1];
+          }
+          *reinterpret_cast<float2*>(dst + r * 64 + col) = make_float2(v0, v1);
+        }
+      }
+    }
+    // N = U~^T Kd and Y^T = U~^T P^T: rows 16*warp .. +16 of both
+    {
+      const int mt = warp;
+      uint32_t af[8][4];
+#pragma unroll
+      for (int ks = 0; ks < 8; ++ks) frag_at(af[ks], s.v, LD128, nullptr, 16 * mt, 8 * ks, gid, tig);
+#pragma unroll
+      for (int nt = 0; nt < 16; ++nt) {
+        const bool is_y = nt >= 8;
+        const int n0 = 8 * (nt & 7);
+        float d[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks) {
+          if (is_y && ks > (nt & 7)) continue;  // P[t][j] = 0 for j > t
+          uint32_t b0, b1;
+          if (is_y) frag_bt(b0, b1, s.p, LD64, n0, 8 * ks, gid, tig);
+          else frag_b(b0, b1, s.k, LD64, s.kdec, n0, 8 * ks, gid, tig);
+          mma(d, af[ks], b0, b1);
+        }
+        float* dst = rec + (is_y ? 2 : 1) * 128 * 64;
+        const int r = 16 * mt + gid, col = n0 + 2 * tig;
+        *reinterpret_cast<float2*>(dst + r * 64 + col) = make_float2(d[0], d[1]);
+        *reinterpret_cast<float2*>(dst + (r + 8) * 64 + col) = make_float2(d[2], d[3]);
+      }
+    }
+  }
+}
+
+struct StateSmem {
+  float bc[2][128 * LD64];    // [M^T; R]
+  float nn[2][kRows * LD64];  // N rows of this CTA
+  float yt[2][kRows * LD64];  // Y^T rows of this CTA
+  float st[2][kRows * LD64];  // the state rows, current and next
+  float os[C * 36];           // output staging [t][i]
+};
+
+__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_1() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+
+__device__ __forceinline__ void load_record(StateSmem& s, int buf, const float* rec, int i0, int tid) {
+  for (int idx = tid; idx < 3072; idx += kThreads) {
+    const int c16 = idx & 15;
+    if (idx < 2048) {
+      const int r = idx >> 4;
+      cp_async16(&s.bc[buf][r * LD64 + 4 * c16], rec + r * 64 + 4 * c16);
+    } else if (idx < 2560) {
+      const int r = (idx - 2048) >> 4;
+      cp_async16(&s.nn[buf][r * LD64 + 4 * c16], rec + 128 * 64 + (i0 + r) * 64 + 4 * c16);
+    } else {
+      const int r = (idx - 2560) >> 4;
+      cp_async16(&s.yt[buf][r * LD64 + 4 * c16], rec + 2 * 128 * 64 + (i0 + r) * 64 + 4 * c16);
+    }
+  }
+}
+
+// One CTA per (value head, 32 state rows): the chunks in order.
+__global__ void __launch_bounds__(kThreads, 1) gdn_state_kernel(const __grid_constant__ GdnArgs a) {
+  extern __shared__ __align__(16) uint8_t smem_raw[];
+  StateSmem& s = *reinterpret_cast<StateSmem*>(smem_raw);
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int gid = lane >> 2, tig = lane & 3;
+  const int h = blockIdx.x, i0 = blockIdx.y * kRows;
+
+  grid_dependency_wait();
+  if (tid == 0) grid_launch_dependents();
+
+  auto rec_of = [&](int c) { return a.ws + (static_cast<int64_t>(c) * a.H + h) * kRec; };
+  load_record(s, 0, rec_of(0), i0, tid);
+  cp_async_commit();
+  if (a.nchunks > 1) load_record(s, 1, rec_of(1), i0, tid);
+  cp_async_commit();
+  // entering state
+  for (int idx = tid; idx < kRows * DK; idx += kThreads) {
+    const int r = idx / DK, col = idx % DK;
+    s.st[0][r * LD64 + col] = a.h0 ? a.h0[(static_cast<int64_t>(h) * DV + i0 + r) * DK + col] : 0.0f;
+  }
+  int cur = 0;
+  for (int c = 0; c < a.nchunks; ++c) {
+    const int buf = c & 1;
+    cp_async_wait_1();
+    __syncthreads();
+    // D[i][n] = sum_k S[i][k] Bc[n][k]: n < 64 -> (S M)[i][n], n >= 64 -> (S R^T)[i][t = n - 64]
+    {
+      uint32_t af[2][8][4];
+#pragma unroll
+      for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks) frag_a(af[mt][ks], s.st[cur], LD64, 16 * mt, 8 * ks, gid, tig);
+      float d[2][2][4];
+#pragma unroll
+      for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt) d[mt][nt][0] = d[mt][nt][1] = d[mt][nt][2] = d[mt][nt][3] = 0.0f;
+      const int nbase = 16 * warp;  // warps 0-3: state columns, 4-7: tokens
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks) {
+          uint32_t b0, b1;
+          frag_bt(b0, b1, s.bc[buf], LD64, nbase + 8 * nt, 8 * ks, gid, tig);
+          mma(d[0][nt], af[0][ks], b0, b1);
+          mma(d[1][nt], af[1][ks], b0, b1);
+        }
+      if (warp < 4) {
+#pragma unroll
+        for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+          for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+              const int r = 16 * mt + gid + 8 * hh, col = nbase + 8 * nt + 2 * tig;
+              const float2 n2 = *reinterpret_cast<const float2*>(&s.nn[buf][r * LD64 + col]);
+              *reinterpret_cast<float2*>(&s.st[cur ^ 1][r * LD64 + col]) =
+                  make_float2(d[mt][nt][2 * hh] + n2.x, d[mt][nt][2 * hh + 1] + n2.y);
+            }
+      } else {
+#pragma unroll
+        for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+          for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int r = 16 * mt + gid + (e >= 2 ? 8 : 0);
+              const int t = nbase - 64 + 8 * nt + 2 * tig + (e & 1);
+              s.os[t * 36 + r] = d[mt][nt][e] + s.yt[buf][r * LD64 + t];
+            }
+      }
+    }
+    __syncthreads();
+    if (c + 2 < a.nchunks) load_record(s, buf, rec_of(c + 2), i0, tid);
+    cp_async_commit();
+    // O rows of this chunk: 64 tokens x 32 values
+    {
+      const int t = tid >> 2, part = tid & 3;
+      const int64_t tok = static_cast<int64_t>(c) * C + t;
+      if (tok < a.T) {
+        const float* src = &s.os[t * 36 + 8 * part];
+        uint8_t* dst = a.o + tok * a.ld_o;
+        const int64_t col = static_cast<int64_t>(h) * DV + i0 + 8 * part;
+        if (a.out_f32) {
+          float4* p = reinterpret_cast<float4*>(dst + col * 4);
+          p[0] = make_float4(src[0], src[1], src[2], src[3]);
+          p[1] = make_float4(src[4], src[5], src[6], src[7]);
+        } else {
+          uint32_t w[4];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const __nv_bfloat162 b = __floats2bfloat162_rn(src[2 * i], src[2 * i + 1]);
+            w[i] = *reinterpret_cast<const uint32_t*>(&b);
+          }
+          *reinterpret_cast<uint4*>(dst + col * 2) = make_uint4(w[0], w[1], w[2], w[3]);
+        }
+      }
+    }
+    cur ^= 1;
+  }
+  cp_async_wait_all();
+  if (a.h_out) {
+    __syncthreads();
+    for (int idx = tid; idx < kRows * DK; idx += kThreads) {
+      const int r = idx / DK, col = idx % DK;
+      a.h_out[(static_cast<int64_t>(h) * DV + i0 + r) * DK + col] = s.st[cur][r * LD64 + col];
+    }
+  }
+}
+
+template <class Kern>
+cudaError_t launch(Kern kern, dim3 grid, int smem, const GdnArgs& a, cudaStream_t stream) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, a);
+}
+
+}  // namespace gdn
+
+size_t gdn_workspace_bytes(int64_t T, int64_t H) {
+  return static_cast<size_t>(ceil_div(T, gdn::C)) * static_cast<size_t>(H) * gdn::kRec * sizeof(float);
+}
+
+cudaError_t launch_gdn(const GdnProblem& p, cudaStream_t stream) {
+  using namespace gdn;
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(gdn_prep_kernel<NVFP4_DTYPE_BF16>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, sizeof(PrepSmem));
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(gdn_prep_kernel<NVFP4_DTYPE_F32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               sizeof(PrepSmem));
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(gdn_state_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, sizeof(StateSmem));
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  const int esz = p.in_dtype == NVFP4_DTYPE_BF16 ? 2 : 4;
+  GdnArgs a{};
+  a.q = static_cast<const uint8_t*>(p.q);
+  a.k = static_cast<const uint8_t*>(p.k);
+  a.v = static_cast<const uint8_t*>(p.v);
+  a.ld_q = p.ld_q * esz;
+  a.ld_k = p.ld_k * esz;
+  a.ld_v = p.ld_v * esz;
+  a.beta = p.beta;
+  a.g = p.g;
+  a.ld_beta = p.ld_beta;
+  a.ld_g = p.ld_g;
+  a.T = p.T;
+  a.H = static_cast<int>(p.H);
+  a.rep = static_cast<int>(p.H / p.H_k);
+  a.nchunks = static_cast<int>(ceil_div(p.T, C));
+  a.scale = p.scale;
+  a.eps = 1e-6f;
+  a.h0 = p.h0;
+  a.h_out = p.h_out;
+  a.o = static_cast<uint8_t*>(p.o);
+  a.out_f32 = p.out_dtype == NVFP4_DTYPE_F32 ? 1 : 0;
+  a.ld_o = p.ld_o * (a.out_f32 ? 4 : 2);
+  a.ws = static_cast<float*>(p.workspace);
+  const dim3 gp(static_cast<unsigned>(a.nchunks), static_cast<unsigned>(a.H));
+  cudaError_t e = p.in_dtype == NVFP4_DTYPE_BF16
+                      ? launch(gdn_prep_kernel<NVFP4_DTYPE_BF16>, gp, sizeof(PrepSmem), a, stream)
+                      : launch(gdn_prep_kernel<NVFP4_DTYPE_F32>, gp, sizeof(PrepSmem), a, stream);
+  if (e != cudaSuccess) return e;
+  return launch(gdn_state_kernel, dim3(static_cast<unsigned>(a.H), DV / kRows), sizeof(StateSmem), a, stream);
+}
+
+}  // namespace nvfp4

@@ -56,6 +56,30 @@ cudaError_t launch_act_stats(const void* x, int dtype, int64_t M, int64_t K, int
                              double* moments, float* row_err2, float* row_norm2, float* col_sq, float* col_max,
                              cudaStream_t stream);
 
+// Gated delta-rule recurrence (see nvfp4_gdn_recurrence); leading dimensions
+// in elements, d_k = 64 and d_v = 128.
+struct GdnProblem {
+  const void* q;
+  const void* k;
+  const void* v;
+  int in_dtype;
+  int64_t T, H, H_k;
+  int64_t ld_q, ld_k, ld_v;
+  const float* beta;
+  const float* g;
+  int64_t ld_beta, ld_g;
+  float scale;
+  const float* h0;
+  float* h_out;
+  void* o;
+  int out_dtype;
+  int64_t ld_o;
+  void* workspace;
+};
+
+size_t gdn_workspace_bytes(int64_t T, int64_t H);
+cudaError_t launch_gdn(const GdnProblem& p, cudaStream_t stream);
+
 // GEMM epilogue description handed to the kernels.
 struct EpiSegment {
   int64_t n_begin, n_end;

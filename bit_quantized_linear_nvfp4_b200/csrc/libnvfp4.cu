@@ -7,3 +7,4 @@
 #include "noalloc.cu"
 #include "kv_fp8.cu"
 #include "act_stats.cu"
+#include "gdn.cu"

@@ -45,6 +45,7 @@ EXPORTED = (
     "nvfp4_gemm_workspace_bytes", "nvfp4_gemm", "nvfp4_fused_proj", "nvfp4_check",
     "nvfp4_quantize_noalloc", "nvfp4_linear", "nvfp4_requantize_segments",
     "nvfp4_kv_fp8_quantize", "nvfp4_kv_fp8_dequantize", "nvfp4_activation_stats",
+    "nvfp4_gdn_workspace_bytes", "nvfp4_gdn_recurrence",
 )
 
 
@@ -124,6 +125,14 @@ def _lib():
         lib.nvfp4_activation_stats.argtypes = [c.c_void_p, c.c_int, c.c_int64, c.c_int64, c.c_int64, c.c_void_p,
                                                c.c_void_p, c.c_void_p, c.c_void_p, c.c_void_p, c.c_void_p,
                                                c.c_void_p]
+        lib.nvfp4_gdn_workspace_bytes.restype = c.c_size_t
+        lib.nvfp4_gdn_workspace_bytes.argtypes = [c.c_int64, c.c_int64]
+        lib.nvfp4_gdn_recurrence.restype = c.c_int
+        lib.nvfp4_gdn_recurrence.argtypes = [c.c_void_p, c.c_void_p, c.c_void_p, c.c_int, c.c_int64, c.c_int64,
+                                             c.c_int64, c.c_int64, c.c_int64, c.c_int64, c.c_int64, c.c_int64,
+                                             c.c_void_p, c.c_int64, c.c_void_p, c.c_int64, c.c_float,
+                                             c.c_void_p, c.c_void_p, c.c_void_p, c.c_int, c.c_int64,
+                                             c.c_void_p, c.c_size_t, c.c_void_p]
         lib.nvfp4_check.restype = c.c_int
         lib.nvfp4_check.argtypes = [c.c_void_p]
         _LIB = lib
@@ -322,6 +331,43 @@ def nvfp4_requantize_segments(W: Operand, row_bounds: Sequence[int], g_old: torc
     _call("nvfp4_requantize_segments", ctypes.byref(w), bounds, nseg, _ptr(g_old), _ptr(g_new), _ptr(codes),
           _ptr(sf), _ptr(g_out), _stream(stream))
     return Operand(codes, sf, W.rows, W.K), g_out
+
+
+def nvfp4_gdn_workspace_bytes(T: int, H: int) -> int:
+    return int(_lib().nvfp4_gdn_workspace_bytes(T, H))
+
+
+GDN_DK, GDN_DV = 64, 128
+
+
+def nvfp4_gdn_recurrence(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, beta: torch.Tensor, g: torch.Tensor,
+                         h0: Optional[torch.Tensor] = None, scale: float = 0.0, *, d_k: int = GDN_DK,
+                         d_v: int = GDN_DV, out=None, out_dtype=None, h_out=None, workspace=None, stream=None):
+    """Gated delta rule over one sequence: q, k [T, H_k*64], v [T, H*128]
+    (BF16/F32, same dtype), beta, g [T, H] FP32 -> o [T, H*128] (v's dtype
+    unless out/out_dtype says otherwise).  h0 / h_out: FP32 [H, 128, 64]
+    entering / final state (h_out may be h0).  scale 0 selects 64^-1/2."""
+    for t in (q, k, v, beta, g):
+        _check_2d(t)
+    if q.dtype != v.dtype or k.dtype != v.dtype:
+        raise TypeError("q, k and v must share one dtype")
+    if beta.dtype != torch.float32 or g.dtype != torch.float32:
+        raise TypeError("beta and g must be float32")
+    T = v.shape[0]
+    H = v.shape[1] // d_v
+    H_k = q.shape[1] // d_k
+    dev = v.device
+    if out is None:
+        out = torch.empty((T, H * GDN_DV), dtype=out_dtype or v.dtype, device=dev)
+    if workspace is None:
+        workspace = torch.empty(max(1, nvfp4_gdn_workspace_bytes(T, H)), dtype=torch.uint8, device=dev)
+    ws_bytes = workspace.numel() * workspace.element_size()
+    in_code = _dtype_code(v)
+    out_code = DTYPE_BF16 if out.dtype == torch.bfloat16 else DTYPE_F32
+    _call("nvfp4_gdn_recurrence", _ptr(q), _ptr(k), _ptr(v), in_code, T, H, H_k, d_k, d_v, q.stride(0),
+          k.stride(0), v.stride(0), _ptr(beta), beta.stride(0), _ptr(g), g.stride(0), float(scale), _ptr(h0),
+          _ptr(h_out), _ptr(out), out_code, out.stride(0), _ptr(workspace), ws_bytes, _stream(stream))
+    return out
 
 
 def nvfp4_kv_fp8_quantize(x: torch.Tensor, scale: torch.Tensor, *, out=None, stream=None) -> torch.Tensor:

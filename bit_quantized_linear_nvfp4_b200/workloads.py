@@ -20,6 +20,13 @@ Recipe (every draw uses ``numpy.random.default_rng``):
     .standard_normal((n_s, K), float32)``, rounded to BF16 for BF16 workloads.
   * GDN gate parameters: ``default_rng(seed + 7)``: A_log ~ U(-1, 1) then
     dt_bias ~ N(0, 0.5) (0.5 read as the standard deviation), one per head.
+  * Delta-rule recurrence inputs drawn directly (the parity cases; the
+    benchmark feeds the recurrence from the GDN projection itself):
+    ``default_rng(seed)``: q, k [T, H_k*64] and v [T, H*128] N(0,1) (BF16
+    workloads round them), beta [T, H] ~ U(0, 1), and the log decay
+    g = -exp(mu_h + 0.5 z) with one level mu_h ~ U(ln 1e-3, ln 2) per head and
+    z ~ N(0, 1) per token, so heads range from slow (alpha ~ 0.999) to fast
+    (alpha ~ 0.1) forgetting.
 """
 from __future__ import annotations
 
@@ -158,3 +165,22 @@ def sample_rows(M: int, n: int, seed: int = 12345) -> np.ndarray:
     rng = np.random.default_rng(seed)
     inner = rng.choice(np.arange(1, M - 1), size=n - 2, replace=False)
     return np.sort(np.concatenate([[0, M - 1], inner])).astype(np.int64)
+
+
+GDN_HEADS, GDN_DK, GDN_DV = 32, 64, 128  # the projection's q/k (2048 = 32 x 64) and v (4096 = 32 x 128)
+
+
+def make_recurrence_inputs(T: int, H: int, H_k: int, seed: int, dtype: str = "bf16", slow: bool = False):
+    """(q, k, v, beta, g) float32 arrays for the delta-rule recurrence.  With
+    slow, every head decays slowly (mu_h ~ U(ln 1e-4, ln 1e-2))."""
+    rng = np.random.default_rng(seed)
+    q = rng.standard_normal((T, H_k * GDN_DK), dtype=np.float32)
+    k = rng.standard_normal((T, H_k * GDN_DK), dtype=np.float32)
+    v = rng.standard_normal((T, H * GDN_DV), dtype=np.float32)
+    beta = rng.uniform(0.0, 1.0, size=(T, H)).astype(np.float32)
+    lo, hi = (np.log(1e-4), np.log(1e-2)) if slow else (np.log(1e-3), np.log(2.0))
+    mu = rng.uniform(lo, hi, size=H)
+    g = (-np.exp(mu[None, :] + 0.5 * rng.standard_normal((T, H)))).astype(np.float32)
+    if dtype == "bf16":
+        q, k, v = round_to_bf16(q), round_to_bf16(k), round_to_bf16(v)
+    return q, k, v, beta, g

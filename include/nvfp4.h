@@ -310,6 +310,43 @@ int nvfp4_activation_stats(const void* x, int x_dtype, int64_t M, int64_t K, int
                            void* stream);
 
 /*
+ * nvfp4_gdn_recurrence — the gated delta-rule recurrence that consumes the
+ * fused GDN projection's q, k, v, beta and g ("Main Findings", recurrence
+ * bullet: a fixed-size state in which every write overwrites along the
+ * current key, with a decay and a write strength; gate-parameterisation
+ * bullet: the decay gate is log-space, alpha = exp(g)).  Per value head h,
+ * with the state S [d_v, d_k] in FP32:
+ *     S_t = alpha_t S_{t-1} + beta_t (v_t - alpha_t S_{t-1} k_t) k_t^T,
+ *     o_t = S_t q_t,   alpha_t = exp(g_t),
+ * q and k L2-normalised per head (x / sqrt(sum x^2 + 1e-6)) and q scaled by
+ * `scale`.  One sequence of T tokens; value head h reads query/key head
+ * h / (H / H_k).  Evaluated in chunks of 64 tokens with TF32 tensor-core
+ * products and FP32 state (results differ from an exact evaluation by the
+ * rounding of the products' operands to TF32).
+ *   q, k     device [T, H_k * d_k] (BF16 or F32, in_dtype), row strides ld_q,
+ *            ld_k elements; head j in columns [j d_k, (j+1) d_k).
+ *   v        device [T, H * d_v], same dtype, row stride ld_v.
+ *   beta, g  device FP32 [T, H] (the projection's sigmoid and decay outputs),
+ *            row strides ld_beta, ld_g elements.
+ *   scale    query scale; 0 selects d_k^-1/2.  Must be finite and >= 0.
+ *   h0       device FP32 [H, d_v, d_k] entering state, or NULL for zeros.
+ *   h_out    device FP32 [H, d_v, d_k] receives the final state, or NULL;
+ *            may equal h0 (the update is then in place) but no other overlap.
+ *   o        device [T, H * d_v] (BF16 or F32, out_dtype), row stride ld_o.
+ *   workspace, workspace_bytes   device, 16-byte aligned, at least
+ *            nvfp4_gdn_workspace_bytes(T, H) bytes (per-chunk matrices).
+ * Shapes: d_k == 64 and d_v == 128 (else NVFP4_ERR_UNSUPPORTED_SHAPE);
+ * H_k divides H; q, k, v and o rows 16-byte aligned.  o must not overlap any
+ * input or the workspace.  T == 0 only copies h0 (or zeros) to h_out.
+ */
+size_t nvfp4_gdn_workspace_bytes(int64_t T, int64_t H);
+int nvfp4_gdn_recurrence(const void* q, const void* k, const void* v, int in_dtype, int64_t T, int64_t H,
+                         int64_t H_k, int64_t d_k, int64_t d_v, int64_t ld_q, int64_t ld_k, int64_t ld_v,
+                         const float* beta, int64_t ld_beta, const float* g, int64_t ld_g, float scale,
+                         const float* h0, float* h_out, void* o, int out_dtype, int64_t ld_o,
+                         void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * nvfp4_check — synchronise `stream`, then report (and clear) the library's
  * device error word: NVFP4_ERR_DEVICE_TIMEOUT if a bounded wait inside a
  * kernel gave up since the last check, NVFP4_ERR_CUDA on a CUDA error.

@@ -211,3 +211,31 @@ def test_activation_stats_rejects_bad_arguments(lib):
     assert call(cs=FAKE + 2) == 3
     assert call(ld=32) == 1
     assert call(M=0) == 0
+
+
+def test_gdn_recurrence_rejects_bad_arguments(lib):
+    v = ctypes.c_void_p
+    T, H, Hk = 100, 4, 2
+    Q, K, V, B, G, O, WS = (FAKE + i * 0x1000000 for i in range(7))
+
+    def call(q=Q, k=K, vv=V, dt=0, T=T, H=H, Hk=Hk, dk=64, dv=128, ldq=Hk * 64, ldk=Hk * 64, ldv=H * 128,
+             beta=B, ldb=H, g=G, ldg=H, scale=0.0, h0=0, hout=0, o=O, odt=0, ldo=H * 128, ws=WS, wsb=1 << 40):
+        p = lambda a: v(a) if a else None
+        return lib.nvfp4_gdn_recurrence(p(q), p(k), p(vv), dt, T, H, Hk, dk, dv, ldq, ldk, ldv, p(beta), ldb, p(g),
+                                        ldg, scale, p(h0), p(hout), p(o), odt, ldo, p(ws), wsb, None)
+    assert lib.nvfp4_gdn_workspace_bytes(T, H) == 2 * H * 3 * 128 * 64 * 4  # two chunks of 64 tokens
+    assert lib.nvfp4_gdn_workspace_bytes(0, H) == 0
+    assert call(dt=2) == 1 and call(odt=7) == 1
+    assert call(Hk=3) == 1                    # H_k must divide H
+    assert call(dk=128) == 2 and call(dv=64) == 2
+    assert call(scale=-1.0) == 1 and call(scale=float("nan")) == 1
+    assert call(q=0) == 1 and call(beta=0) == 1 and call(o=0) == 1
+    assert call(ldq=64) == 1 and call(ldv=500) == 1 and call(ldb=2) == 1
+    assert call(q=Q + 8) == 3 and call(o=O + 4) == 3
+    assert call(ldk=Hk * 64 + 4) == 3         # BF16 row of k not a multiple of 16 bytes
+    assert call(beta=B + 2) == 3
+    assert call(ws=0) == 6 and call(wsb=1000) == 6 and call(ws=WS + 8) == 6
+    assert call(o=V + 256) == 1               # output overlapping v
+    assert call(ws=O) == 1                    # workspace overlapping the output
+    assert call(h0=FAKE + 0x9000000, hout=FAKE + 0x9000000 + 64) == 1  # partial state overlap
+    assert call(T=0) == 0                     # nothing to do without h_out
