@@ -942,6 +942,9 @@ def run_gdnrec(args):
     for extra in proj.sets[1:]:
         extra.clear()
     proj.sets = [s0]
+    if args.rows is not None:  # the first rows only: a smaller case of the same kernels (profiling)
+        T = args.rows
+        q, k, v, beta, g = (t[:T] for t in (q, k, v, beta, g))
     out = torch.empty((T, H * 128), dtype=torch.bfloat16, device=device)
     h_out = torch.empty((H, 128, 64), dtype=torch.float32, device=device)
     ws = torch.empty(nv.nvfp4_gdn_workspace_bytes(T, H), dtype=torch.uint8, device=device)
@@ -1179,7 +1182,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--rows", type=int, default=None,
-                    help="quant workload only: quantise [rows, 17408] instead of the full tensor (for profiler captures)")
+                    help="quant: quantise [rows, 17408]; gdnrec: the first rows tokens (smaller cases for profiler captures)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

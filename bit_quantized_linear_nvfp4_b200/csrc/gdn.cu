@@ -157,6 +157,7 @@ struct PrepSmem {
   float bg[C];         // beta e^gam
   float eg[C];         // e^gam
   float kdec[C];       // e^(gam_C - gam)
+  float tmp[3 * 272];  // block products of the triangular inverse (16 x 17 each)
 };
 
 // One CTA per (chunk, value head): the S-independent matrices of the chunk.
@@ -273,9 +274,9 @@ __global__ void __launch_bounds__(kThreads, 2) gdn_prep_kernel(const __grid_cons
         const int t = 16 * mt + gid + (e >= 2 ? 8 : 0), j = 8 * nt + 2 * tig + (e & 1);
         float val = 0.0f;
         if (mat == 0) {
-          if (j < t) val = s.beta[t] * expf(s.gam[t] - s.gam[j]) * d[e];
+          if (j < t) val = s.beta[t] * __expf(s.gam[t] - s.gam[j]) * d[e];
         } else {
-          if (j <= t) val = expf(s.gam[t] - s.gam[j]) * d[e];
+          if (j <= t) val = __expf(s.gam[t] - s.gam[j]) * d[e];
         }
         out[t * LD64 + j] = val;
       }
@@ -283,28 +284,74 @@ __global__ void __launch_bounds__(kThreads, 2) gdn_prep_kernel(const __grid_cons
   }
   __syncthreads();
 
-  // ---- step 2: L = (I + A)^-1 by forward substitution, one column per thread
-  if (tid < C) {
-    const int j = tid;
-    float col[C];
+  // ---- step 2: L = (I + A)^-1 with A strictly lower triangular, in 16 x 16
+  // blocks: the diagonal blocks by forward substitution (one column per
+  // thread), then one block diagonal at a time
+  //     L_ij = -L_ii T,  T = sum_{m=j}^{i-1} A_im L_mj   (i > j).
+  // While A is still read, L is built transposed in al's strict upper triangle.
+  {
+    auto lval = [&](int r, int c) -> float {  // L[r][c], r >= c known to be built
+      return r == c ? 1.0f : s.al[c * LD64 + r];
+    };
+    if (tid < C) {
+      const int base = 16 * (tid >> 4), jj = tid & 15;
+      float col[16];
 #pragma unroll
-    for (int i = 0; i < C; ++i) {
-      float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+      for (int i = 0; i < 16; ++i) {
+        float acc0 = 0.0f, acc1 = 0.0f;
 #pragma unroll
-      for (int m = 0; m + 4 <= i; m += 4) {
-        const float4 r = *reinterpret_cast<const float4*>(&s.al[i * LD64 + m]);
-        acc[0] = fmaf(r.x, col[m], acc[0]);
-        acc[1] = fmaf(r.y, col[m + 1], acc[1]);
-        acc[2] = fmaf(r.z, col[m + 2], acc[2]);
-        acc[3] = fmaf(r.w, col[m + 3], acc[3]);
+        for (int m = 0; m < i; ++m) {
+          const float a = s.al[(base + i) * LD64 + base + m];
+          if (m & 1) acc1 = fmaf(a, col[m], acc1);
+          else acc0 = fmaf(a, col[m], acc0);
+        }
+        col[i] = (i == jj ? 1.0f : 0.0f) - (acc0 + acc1);
       }
 #pragma unroll
-      for (int m = (i / 4) * 4; m < i; ++m) acc[m & 3] = fmaf(s.al[i * LD64 + m], col[m], acc[m & 3]);
-      col[i] = (i == j ? 1.0f : 0.0f) - ((acc[0] + acc[1]) + (acc[2] + acc[3]));
+      for (int i = 0; i < 16; ++i)
+        if (i > jj) s.al[(base + jj) * LD64 + base + i] = col[i];
     }
-    asm volatile("bar.sync 1, 64;" ::: "memory");  // every thread is done reading A
+    __syncthreads();
+    for (int dd = 1; dd < 4; ++dd) {
+      const int nblk = 4 - dd;
+      for (int idx = tid; idx < nblk * 256; idx += kThreads) {
+        const int bi = dd + (idx >> 8), bj = bi - dd, r = (idx >> 4) & 15, c = idx & 15;
+        float acc = 0.0f;
+        for (int mb = bj; mb < bi; ++mb) {
+          const float* arow = &s.al[(16 * bi + r) * LD64 + 16 * mb];
 #pragma unroll
-    for (int i = 0; i < C; ++i) s.al[i * LD64 + j] = col[i];
+          for (int m = 0; m < 16; ++m) {
+            const int lr = 16 * mb + m, lc = 16 * bj + c;
+            if (lr >= lc) acc = fmaf(arow[m], lval(lr, lc), acc);
+          }
+        }
+        s.tmp[(idx >> 8) * 272 + r * 17 + c] = acc;
+      }
+      __syncthreads();
+      for (int idx = tid; idx < nblk * 256; idx += kThreads) {
+        const int bi = dd + (idx >> 8), bj = bi - dd, r = (idx >> 4) & 15, c = idx & 15;
+        const float* t = &s.tmp[(idx >> 8) * 272];
+        float acc = 0.0f;
+#pragma unroll
+        for (int m = 0; m < 16; ++m)
+          if (m <= r) acc = fmaf(lval(16 * bi + r, 16 * bi + m), t[m * 17 + c], acc);
+        s.al[(16 * bj + c) * LD64 + 16 * bi + r] = -acc;
+      }
+      __syncthreads();
+    }
+    // move L to the lower triangle (unit diagonal, zeros above) for the products
+    float mv[16];
+#pragma unroll
+    for (int e = 0; e < 16; ++e) {
+      const int idx = tid + e * kThreads, r = idx >> 6, c = idx & 63;
+      mv[e] = r > c ? s.al[c * LD64 + r] : (r == c ? 1.0f : 0.0f);
+    }
+    __syncthreads();
+#pragma unroll
+    for (int e = 0; e < 16; ++e) {
+      const int idx = tid + e * kThreads, r = idx >> 6, c = idx & 63;
+      s.al[r * LD64 + c] = mv[e];
+    }
   }
   __syncthreads();
 
@@ -478,21 +525,30 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_state_kernel(const __grid_con
       for (int mt = 0; mt < 2; ++mt)
 #pragma unroll
         for (int ks = 0; ks < 8; ++ks) frag_a(af[mt][ks], s.st[cur], LD64, 16 * mt, 8 * ks, gid, tig);
-      float d[2][2][4];
+      // two accumulators per tile (even and odd k-steps) halve the dependent MMA chain
+      float d[2][2][4], d2[2][2][4];
 #pragma unroll
       for (int mt = 0; mt < 2; ++mt)
 #pragma unroll
-        for (int nt = 0; nt < 2; ++nt) d[mt][nt][0] = d[mt][nt][1] = d[mt][nt][2] = d[mt][nt][3] = 0.0f;
+        for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) d[mt][nt][e] = d2[mt][nt][e] = 0.0f;
       const int nbase = 16 * warp;  // warps 0-3: state columns, 4-7: tokens
 #pragma unroll
-      for (int nt = 0; nt < 2; ++nt)
+      for (int ks = 0; ks < 8; ++ks)
 #pragma unroll
-        for (int ks = 0; ks < 8; ++ks) {
+        for (int nt = 0; nt < 2; ++nt) {
           uint32_t b0, b1;
           frag_bt(b0, b1, s.bc[buf], LD64, nbase + 8 * nt, 8 * ks, gid, tig);
-          mma(d[0][nt], af[0][ks], b0, b1);
-          mma(d[1][nt], af[1][ks], b0, b1);
+          mma((ks & 1) ? d2[0][nt] : d[0][nt], af[0][ks], b0, b1);
+          mma((ks & 1) ? d2[1][nt] : d[1][nt], af[1][ks], b0, b1);
         }
+#pragma unroll
+      for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) d[mt][nt][e] += d2[mt][nt][e];
       if (warp < 4) {
 #pragma unroll
         for (int mt = 0; mt < 2; ++mt)
