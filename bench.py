@@ -34,9 +34,11 @@ ROTATE = 4          # rotating input sets so consecutive steps miss in L2
 # dominant kernel, from one ncu capture of the kernel as it is now (the
 # commands are in profiles/); an entry is removed when its kernel changes,
 # until it is captured again.  "quant": both passes, captured on X[8192, 17408]
-# and scaled by 4 rows-wise (the traffic grows with the rows).
+# and scaled by 4 rows-wise (the traffic grows with the rows).  "gdnrec": both
+# recurrence launches, captured at 8192 tokens and scaled by 4 (all of it is per chunk).
 TRAFFIC_BYTES = {
     "actstats": 339406592,
+    "gdnrec": 3791627264,
     "decode1": 50362112,
     "decode64": 50922752,
     "decode8": 50422528,
