@@ -8,7 +8,7 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libnvfp4.so")
-SOURCES = ["libnvfp4.cu", "quantize.cu", "gemm.cu", "gemm_decode.cu", "api.cu", "noalloc.cu", "kv_fp8.cu", "act_stats.cu", "gdn.cu", "ptx.cuh",
+SOURCES = ["libnvfp4.cu", "quantize.cu", "gemm.cu", "gemm_decode.cu", "api.cu", "noalloc.cu", "kv_fp8.cu", "act_stats.cu", "gdn.cu", "selftest.cu", "ptx.cuh",
            "internal.h"]
 
 

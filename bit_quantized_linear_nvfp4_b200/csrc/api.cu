@@ -467,6 +467,15 @@ int nvfp4_gdn_recurrence(const void* q, const void* k, const void* v, int in_dty
   return NVFP4_OK;
 }
 
+int nvfp4_selftest_bounded_wait(uint64_t limit_ns, void* stream) {
+  if (limit_ns < 1000000ull || limit_ns > 2000000000ull) return NVFP4_ERR_INVALID_ARG;
+  int st = check_device();
+  if (st != NVFP4_OK) return st;
+  cudaError_t e = nvfp4::launch_wait_selftest(limit_ns, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e);
+  return NVFP4_OK;
+}
+
 int nvfp4_check(void* stream) {
   cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e);

@@ -29,7 +29,9 @@
 // chain of dependent steps (Gram matrix -> triangular solve -> products ->
 // state), where register fragments avoid a round trip through tensor memory
 // between steps.  Operands are rounded to TF32 (nearest, ties away); the
-// triangular solve, the state and all sums stay FP32.
+// state and all sums stay FP32, and the triangular inverse keeps about FP32
+// accuracy (FP32 substitution inside the 16 x 16 diagonal blocks, 3xTF32
+// products for the blocks below them).
 #include <cstdint>
 
 #include <cuda_bf16.h>
@@ -83,6 +85,23 @@ __device__ __forceinline__ void mma(float (&d)[4], const uint32_t (&a)[4], uint3
       "{%0, %1, %2, %3};"
       : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// d += a b to about FP32 accuracy with three TF32 products (x = hi + lo, both
+// TF32; the lo * lo term, below 2^-22 relative, is dropped).
+__device__ __forceinline__ void split_tf32(float x, uint32_t& hi, uint32_t& lo) {
+  hi = tf32(x);
+  lo = tf32(x - __uint_as_float(hi));
+}
+__device__ __forceinline__ void mma_3xtf32(float (&d)[4], const float (&a)[4], float b0, float b1) {
+  uint32_t ah[4], alo[4], bh0, bl0, bh1, bl1;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) split_tf32(a[i], ah[i], alo[i]);
+  split_tf32(b0, bh0, bl0);
+  split_tf32(b1, bh1, bl1);
+  mma(d, alo, bh0, bh1);
+  mma(d, ah, bl0, bl1);
+  mma(d, ah, bh0, bh1);
 }
 
 // Fragment loaders.  gid = lane / 4, tig = lane % 4.  An A fragment holds
@@ -157,7 +176,7 @@ struct PrepSmem {
   float bg[C];         // beta e^gam
   float eg[C];         // e^gam
   float kdec[C];       // e^(gam_C - gam)
-  float tmp[3 * 272];  // block products of the triangular inverse (16 x 17 each)
+  float tmp[3 * 272];  // per-warp T blocks of the triangular inverse (16 x 17 each)
 };
 
 // One CTA per (chunk, value head): the S-independent matrices of the chunk.
@@ -286,13 +305,11 @@ __global__ void __launch_bounds__(kThreads, 2) gdn_prep_kernel(const __grid_cons
 
   // ---- step 2: L = (I + A)^-1 with A strictly lower triangular, in 16 x 16
   // blocks: the diagonal blocks by forward substitution (one column per
-  // thread), then one block diagonal at a time
-  //     L_ij = -L_ii T,  T = sum_{m=j}^{i-1} A_im L_mj   (i > j).
-  // While A is still read, L is built transposed in al's strict upper triangle.
+  // thread, FP32), then one block diagonal at a time
+  //     L_ij = -L_ii T,  T = sum_{m=j}^{i-1} A_im L_mj   (i > j)
+  // with 3xTF32 tensor products (about FP32 accuracy).  While A is still
+  // read, L is built transposed in al's strict upper triangle.
   {
-    auto lval = [&](int r, int c) -> float {  // L[r][c], r >= c known to be built
-      return r == c ? 1.0f : s.al[c * LD64 + r];
-    };
     if (tid < C) {
       const int base = 16 * (tid >> 4), jj = tid & 15;
       float col[16];
@@ -312,30 +329,59 @@ __global__ void __launch_bounds__(kThreads, 2) gdn_prep_kernel(const __grid_cons
         if (i > jj) s.al[(base + jj) * LD64 + base + i] = col[i];
     }
     __syncthreads();
+    // Off-diagonal blocks, one block diagonal dd at a time, one warp per block
+    // (i, j) = (j + dd, j): T = sum_{m=j}^{i-1} A_im L_mj, then L_ij = -L_ii T,
+    // both 16 x 16 x 16k products on the tensor cores in 3xTF32.
+    // lval(mb, j, r, c) = L[16mb + r][16j + c] (mb >= j), read from the transposed copy.
+    auto lval = [&](int mb, int j, int r, int c) -> float {
+      if (mb > j) return s.al[(16 * j + c) * LD64 + 16 * mb + r];
+      return r > c ? s.al[(16 * j + c) * LD64 + 16 * j + r] : (r == c ? 1.0f : 0.0f);
+    };
     for (int dd = 1; dd < 4; ++dd) {
-      const int nblk = 4 - dd;
-      for (int idx = tid; idx < nblk * 256; idx += kThreads) {
-        const int bi = dd + (idx >> 8), bj = bi - dd, r = (idx >> 4) & 15, c = idx & 15;
-        float acc = 0.0f;
-        for (int mb = bj; mb < bi; ++mb) {
-          const float* arow = &s.al[(16 * bi + r) * LD64 + 16 * mb];
+      if (warp < 4 - dd) {
+        const int j = warp, i = warp + dd;
+        float* tw = &s.tmp[warp * 272];  // this warp's T, 16 x 17
+        float t[2][4];
 #pragma unroll
-          for (int m = 0; m < 16; ++m) {
-            const int lr = 16 * mb + m, lc = 16 * bj + c;
-            if (lr >= lc) acc = fmaf(arow[m], lval(lr, lc), acc);
+        for (int nt = 0; nt < 2; ++nt) t[nt][0] = t[nt][1] = t[nt][2] = t[nt][3] = 0.0f;
+        for (int mb = j; mb < i; ++mb) {
+#pragma unroll
+          for (int kk = 0; kk < 2; ++kk) {
+            const float* arow = &s.al[(16 * i) * LD64 + 16 * mb + 8 * kk];
+            const float a[4] = {arow[gid * LD64 + tig], arow[(gid + 8) * LD64 + tig], arow[gid * LD64 + tig + 4],
+                                arow[(gid + 8) * LD64 + tig + 4]};
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt)
+              mma_3xtf32(t[nt], a, lval(mb, j, 8 * kk + tig, 8 * nt + gid), lval(mb, j, 8 * kk + tig + 4, 8 * nt + gid));
           }
         }
-        s.tmp[(idx >> 8) * 272 + r * 17 + c] = acc;
-      }
-      __syncthreads();
-      for (int idx = tid; idx < nblk * 256; idx += kThreads) {
-        const int bi = dd + (idx >> 8), bj = bi - dd, r = (idx >> 4) & 15, c = idx & 15;
-        const float* t = &s.tmp[(idx >> 8) * 272];
-        float acc = 0.0f;
 #pragma unroll
-        for (int m = 0; m < 16; ++m)
-          if (m <= r) acc = fmaf(lval(16 * bi + r, 16 * bi + m), t[m * 17 + c], acc);
-        s.al[(16 * bj + c) * LD64 + 16 * bi + r] = -acc;
+        for (int nt = 0; nt < 2; ++nt) {
+          tw[gid * 17 + 8 * nt + 2 * tig] = t[nt][0];
+          tw[gid * 17 + 8 * nt + 2 * tig + 1] = t[nt][1];
+          tw[(gid + 8) * 17 + 8 * nt + 2 * tig] = t[nt][2];
+          tw[(gid + 8) * 17 + 8 * nt + 2 * tig + 1] = t[nt][3];
+        }
+        __syncwarp();
+        float l[2][4];
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt) l[nt][0] = l[nt][1] = l[nt][2] = l[nt][3] = 0.0f;
+#pragma unroll
+        for (int kk = 0; kk < 2; ++kk) {
+          const float a[4] = {lval(i, i, gid, 8 * kk + tig), lval(i, i, gid + 8, 8 * kk + tig),
+                              lval(i, i, gid, 8 * kk + tig + 4), lval(i, i, gid + 8, 8 * kk + tig + 4)};
+#pragma unroll
+          for (int nt = 0; nt < 2; ++nt)
+            mma_3xtf32(l[nt], a, tw[(8 * kk + tig) * 17 + 8 * nt + gid], tw[(8 * kk + tig + 4) * 17 + 8 * nt + gid]);
+        }
+        // L_ij, negated, into the transposed copy: L[16i + r][16j + c] at al[16j + c][16i + r]
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int r = gid + (e >= 2 ? 8 : 0), c = 8 * nt + 2 * tig + (e & 1);
+            s.al[(16 * j + c) * LD64 + 16 * i + r] = -l[nt][e];
+          }
       }
       __syncthreads();
     }

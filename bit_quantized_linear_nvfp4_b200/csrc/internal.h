@@ -78,6 +78,9 @@ struct GdnProblem {
 };
 
 size_t gdn_workspace_bytes(int64_t T, int64_t H);
+
+// One kernel whose bounded wait is left to run out (see nvfp4_selftest_bounded_wait).
+cudaError_t launch_wait_selftest(uint64_t limit_ns, cudaStream_t stream);
 cudaError_t launch_gdn(const GdnProblem& p, cudaStream_t stream);
 
 // GEMM epilogue description handed to the kernels.

@@ -8,3 +8,4 @@
 #include "kv_fp8.cu"
 #include "act_stats.cu"
 #include "gdn.cu"
+#include "selftest.cu"

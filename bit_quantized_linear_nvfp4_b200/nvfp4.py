@@ -45,7 +45,7 @@ EXPORTED = (
     "nvfp4_gemm_workspace_bytes", "nvfp4_gemm", "nvfp4_fused_proj", "nvfp4_check",
     "nvfp4_quantize_noalloc", "nvfp4_linear", "nvfp4_requantize_segments",
     "nvfp4_kv_fp8_quantize", "nvfp4_kv_fp8_dequantize", "nvfp4_activation_stats",
-    "nvfp4_gdn_workspace_bytes", "nvfp4_gdn_recurrence",
+    "nvfp4_gdn_workspace_bytes", "nvfp4_gdn_recurrence", "nvfp4_selftest_bounded_wait",
 )
 
 
@@ -133,6 +133,8 @@ def _lib():
                                              c.c_void_p, c.c_int64, c.c_void_p, c.c_int64, c.c_float,
                                              c.c_void_p, c.c_void_p, c.c_void_p, c.c_int, c.c_int64,
                                              c.c_void_p, c.c_size_t, c.c_void_p]
+        lib.nvfp4_selftest_bounded_wait.restype = c.c_int
+        lib.nvfp4_selftest_bounded_wait.argtypes = [c.c_uint64, c.c_void_p]
         lib.nvfp4_check.restype = c.c_int
         lib.nvfp4_check.argtypes = [c.c_void_p]
         _LIB = lib

@@ -347,6 +347,18 @@ int nvfp4_gdn_recurrence(const void* q, const void* k, const void* v, int in_dty
                          void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * nvfp4_selftest_bounded_wait — exercises the device-side failure path for
+ * tests of failure detection.  It enqueues one small kernel whose single
+ * thread waits, through the same bounded wait the library's kernels use, on a
+ * barrier that nothing arrives on.  The wait gives up after limit_ns
+ * nanoseconds (1 ms to 2 s, else NVFP4_ERR_INVALID_ARG), sets the device error
+ * word and returns, so the next nvfp4_check on the stream reports
+ * NVFP4_ERR_DEVICE_TIMEOUT and the context stays usable.  Nothing faults or
+ * hangs.
+ */
+int nvfp4_selftest_bounded_wait(uint64_t limit_ns, void* stream);
+
+/*
  * nvfp4_check — synchronise `stream`, then report (and clear) the library's
  * device error word: NVFP4_ERR_DEVICE_TIMEOUT if a bounded wait inside a
  * kernel gave up since the last check, NVFP4_ERR_CUDA on a CUDA error.

@@ -239,3 +239,9 @@ def test_gdn_recurrence_rejects_bad_arguments(lib):
     assert call(ws=O) == 1                    # workspace overlapping the output
     assert call(h0=FAKE + 0x9000000, hout=FAKE + 0x9000000 + 64) == 1  # partial state overlap
     assert call(T=0) == 0                     # nothing to do without h_out
+
+
+def test_bounded_wait_selftest_rejects_bad_limits(lib):
+    assert lib.nvfp4_selftest_bounded_wait(0, None) == 1
+    assert lib.nvfp4_selftest_bounded_wait(999_999, None) == 1          # below 1 ms
+    assert lib.nvfp4_selftest_bounded_wait(2_000_000_001, None) == 1    # above 2 s

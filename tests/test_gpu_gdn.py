@@ -1,8 +1,9 @@
 """GPU parity of the chunked delta-rule recurrence with the oracle's token loop.
 
 Tolerance, derived from the arithmetic.  The kernels round every product
-operand to TF32 (nearest: relative error <= 2^-11) and accumulate, solve and
-keep the state in FP32.  A rounded product sum_k a_k b_k is off by at most
+operand to TF32 (nearest: relative error <= 2^-11) and accumulate and keep the
+state in FP32; the triangular inverse is FP32 substitution plus 3xTF32 block
+products (about FP32).  A rounded product sum_k a_k b_k is off by at most
 2^-10 sum_k |a_k b_k|; between the inputs and an output sit four such
 products in sequence (W and U~ through L, then M, N, R and Y, then S M and
 S R^T), each amplified by at most |L| = |(I + A)^-1|, which stays below 4 for
