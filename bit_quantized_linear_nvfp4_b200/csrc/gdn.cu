@@ -131,6 +131,30 @@ __device__ __forceinline__ void frag_bt(uint32_t& b0, uint32_t& b1, const float*
   b0 = tf32(X[(n0 + gid) * ld + k0 + tig]);
   b1 = tf32(X[(n0 + gid) * ld + k0 + tig + 4]);
 }
+// The same two loaders for values already rounded to TF32 (no conversion).
+__device__ __forceinline__ void frag_a_raw(uint32_t (&a)[4], const float* X, int ld, int m0, int k0, int gid, int tig) {
+  a[0] = __float_as_uint(X[(m0 + gid) * ld + k0 + tig]);
+  a[1] = __float_as_uint(X[(m0 + gid + 8) * ld + k0 + tig]);
+  a[2] = __float_as_uint(X[(m0 + gid) * ld + k0 + tig + 4]);
+  a[3] = __float_as_uint(X[(m0 + gid + 8) * ld + k0 + tig + 4]);
+}
+__device__ __forceinline__ void frag_bt_raw(uint32_t& b0, uint32_t& b1, const float* X, int ld, int n0, int k0,
+                                            int gid, int tig) {
+  b0 = __float_as_uint(X[(n0 + gid) * ld + k0 + tig]);
+  b1 = __float_as_uint(X[(n0 + gid) * ld + k0 + tig + 4]);
+}
+__device__ __forceinline__ void frag_at_raw(uint32_t (&a)[4], const float* X, int ld, int m0, int k0, int gid,
+                                            int tig) {
+  a[0] = __float_as_uint(X[(k0 + tig) * ld + m0 + gid]);
+  a[1] = __float_as_uint(X[(k0 + tig) * ld + m0 + gid + 8]);
+  a[2] = __float_as_uint(X[(k0 + tig + 4) * ld + m0 + gid]);
+  a[3] = __float_as_uint(X[(k0 + tig + 4) * ld + m0 + gid + 8]);
+}
+__device__ __forceinline__ void frag_b_raw(uint32_t& b0, uint32_t& b1, const float* X, int ld, int n0, int k0,
+                                           int gid, int tig) {
+  b0 = __float_as_uint(X[(k0 + tig) * ld + n0 + gid]);
+  b1 = __float_as_uint(X[(k0 + tig + 4) * ld + n0 + gid]);
+}
 // B[k][n] = s[k] X[k][n] (X stored with k as the row).
 __device__ __forceinline__ void frag_b(uint32_t& b0, uint32_t& b1, const float* X, int ld, const float* s, int n0,
                                        int k0, int gid, int tig) {
@@ -295,10 +319,16 @@ __global__ void __launch_bounds__(kThreads, 2) gdn_prep_kernel(const __grid_cons
         if (mat == 0) {
           if (j < t) val = s.beta[t] * __expf(s.gam[t] - s.gam[j]) * d[e];
         } else {
-          if (j <= t) val = __expf(s.gam[t] - s.gam[j]) * d[e];
+          // P is read only as a TF32 MMA operand: rounded here once
+          if (j <= t) val = __uint_as_float(tf32(__expf(s.gam[t] - s.gam[j]) * d[e]));
         }
         out[t * LD64 + j] = val;
       }
+    }
+    // V is read only as diag(beta) V, a TF32 operand: scale and round it in place
+    for (int idx = tid; idx < C * DV; idx += kThreads) {
+      const int j = idx >> 7, n = idx & 127;
+      s.v[j * LD128 + n] = __uint_as_float(tf32(s.beta[j] * s.v[j * LD128 + n]));
     }
   }
   __syncthreads();
@@ -396,7 +426,7 @@ __global__ void __launch_bounds__(kThreads, 2) gdn_prep_kernel(const __grid_cons
 #pragma unroll
     for (int e = 0; e < 16; ++e) {
       const int idx = tid + e * kThreads, r = idx >> 6, c = idx & 63;
-      s.al[r * LD64 + c] = mv[e];
+      s.al[r * LD64 + c] = __uint_as_float(tf32(mv[e]));  // read only as a TF32 operand
     }
   }
   __syncthreads();
@@ -408,7 +438,7 @@ __global__ void __launch_bounds__(kThreads, 2) gdn_prep_kernel(const __grid_cons
     uint32_t af[8][4];
 #pragma unroll
     for (int ks = 0; ks < 8; ++ks)
-      if (ks < nks) frag_a(af[ks], s.al, LD64, 16 * mt, 8 * ks, gid, tig);
+      if (ks < nks) frag_a_raw(af[ks], s.al, LD64, 16 * mt, 8 * ks, gid, tig);
     float d[12][4];
 #pragma unroll
     for (int i = 0; i < 12; ++i) d[i][0] = d[i][1] = d[i][2] = d[i][3] = 0.0f;
@@ -420,19 +450,26 @@ __global__ void __launch_bounds__(kThreads, 2) gdn_prep_kernel(const __grid_cons
         if (ks >= nks) continue;
         uint32_t b0, b1;
         if (nt < 8) frag_b(b0, b1, s.k, LD64, s.bg, 8 * nt, 8 * ks, gid, tig);
-        else frag_b(b0, b1, s.v, LD128, s.beta, 8 * (nt - 8), 8 * ks, gid, tig);
+        else frag_b_raw(b0, b1, s.v, LD128, 8 * (nt - 8), 8 * ks, gid, tig);
         mma(d[i], af[ks], b0, b1);
       }
     }
-    __syncthreads();  // L and V are read; W goes over L, U~ over V
+    __syncthreads();  // L, V and K are read; W goes over L, U~ over V, K_d over K
+    // W and U~ are read only as TF32 operands: rounded here once
 #pragma unroll
     for (int i = 0; i < 12; ++i) {
       const int nt = half * 12 + i;
       const int r = 16 * mt + gid;
       float* dst = nt < 8 ? &s.al[r * LD64 + 8 * nt + 2 * tig] : &s.v[r * LD128 + 8 * (nt - 8) + 2 * tig];
       const int ld = nt < 8 ? LD64 : LD128;
-      *reinterpret_cast<float2*>(dst) = make_float2(d[i][0], d[i][1]);
-      *reinterpret_cast<float2*>(dst + 8 * ld) = make_float2(d[i][2], d[i][3]);
+      *reinterpret_cast<float2*>(dst) = make_float2(__uint_as_float(tf32(d[i][0])), __uint_as_float(tf32(d[i][1])));
+      *reinterpret_cast<float2*>(dst + 8 * ld) =
+          make_float2(__uint_as_float(tf32(d[i][2])), __uint_as_float(tf32(d[i][3])));
+    }
+    // from here on K is read only as K_d = diag(e^(gam_C - gam)) K, a TF32 operand
+    for (int idx = tid; idx < C * DK; idx += kThreads) {
+      const int j = idx >> 6, n = idx & 63;
+      s.k[j * LD64 + n] = __uint_as_float(tf32(s.kdec[j] * s.k[j * LD64 + n]));
     }
   }
   __syncthreads();
@@ -450,8 +487,8 @@ __global__ void __launch_bounds__(kThreads, 2) gdn_prep_kernel(const __grid_cons
 #pragma unroll
       for (int ks = 0; ks < 8; ++ks) {
         if (ks >= nks) continue;
-        if (is_r) frag_a(af[ks], s.p, LD64, 16 * mt, 8 * ks, gid, tig);
-        else frag_at(af[ks], s.k, LD64, s.kdec, 16 * mt, 8 * ks, gid, tig);
+        if (is_r) frag_a_raw(af[ks], s.p, LD64, 16 * mt, 8 * ks, gid, tig);
+        else frag_at_raw(af[ks], s.k, LD64, 16 * mt, 8 * ks, gid, tig);
       }
       float* dst = rec + (is_r ? 64 : 0) * 64;
 #pragma unroll
@@ -461,7 +498,7 @@ __global__ void __launch_bounds__(kThreads, 2) gdn_prep_kernel(const __grid_cons
         for (int ks = 0; ks < 8; ++ks) {
           if (ks >= nks) continue;
           uint32_t b0, b1;
-          frag_b(b0, b1, s.al, LD64, nullptr, 8 * nt, 8 * ks, gid, tig);
+          frag_b_raw(b0, b1, s.al, LD64, 8 * nt, 8 * ks, gid, tig);
           mma(d, af[ks], b0, b1);
         }
 #pragma unroll
@@ -475,7 +512,9 @@ __global__ void __launch_bounds__(kThreads, 2) gdn_prep_kernel(const __grid_cons
             v0 = (r == col ? eC : 0.0f) - d[2 * hh];
             v1 = (r == col + 1 ? eC : 0.0f) - d[2 * hh + 1];
           }
-          *reinterpret_cast<float2*>(dst + r * 64 + col) = make_float2(v0, v1);
+          // rounded here once: the state pass reads these rows only as TF32 MMA operands
+          *reinterpret_cast<float2*>(dst + r * 64 + col) =
+              make_float2(__uint_as_float(tf32(v0)), __uint_as_float(tf32(v1)));
         }
       }
     }
@@ -484,7 +523,7 @@ __global__ void __launch_bounds__(kThreads, 2) gdn_prep_kernel(const __grid_cons
       const int mt = warp;
       uint32_t af[8][4];
 #pragma unroll
-      for (int ks = 0; ks < 8; ++ks) frag_at(af[ks], s.v, LD128, nullptr, 16 * mt, 8 * ks, gid, tig);
+      for (int ks = 0; ks < 8; ++ks) frag_at_raw(af[ks], s.v, LD128, 16 * mt, 8 * ks, gid, tig);
 #pragma unroll
       for (int nt = 0; nt < 16; ++nt) {
         const bool is_y = nt >= 8;
@@ -494,8 +533,8 @@ __global__ void __launch_bounds__(kThreads, 2) gdn_prep_kernel(const __grid_cons
         for (int ks = 0; ks < 8; ++ks) {
           if (is_y && ks > (nt & 7)) continue;  // P[t][j] = 0 for j > t
           uint32_t b0, b1;
-          if (is_y) frag_bt(b0, b1, s.p, LD64, n0, 8 * ks, gid, tig);
-          else frag_b(b0, b1, s.k, LD64, s.kdec, n0, 8 * ks, gid, tig);
+          if (is_y) frag_bt_raw(b0, b1, s.p, LD64, n0, 8 * ks, gid, tig);
+          else frag_b_raw(b0, b1, s.k, LD64, n0, 8 * ks, gid, tig);
           mma(d, af[ks], b0, b1);
         }
         float* dst = rec + (is_y ? 2 : 1) * 128 * 64;
@@ -507,12 +546,14 @@ __global__ void __launch_bounds__(kThreads, 2) gdn_prep_kernel(const __grid_cons
   }
 }
 
+constexpr int kBufs = 3;  // record buffers of the state pass
+
 struct StateSmem {
-  float bc[2][128 * LD64];    // [M^T; R]
-  float nn[2][kRows * LD64];  // N rows of this CTA
-  float yt[2][kRows * LD64];  // Y^T rows of this CTA
-  float st[2][kRows * LD64];  // the state rows, current and next
-  float os[C * 36];           // output staging [t][i]
+  float bc[kBufs][128 * LD64];    // [M^T; R] (TF32 values)
+  float nn[kBufs][kRows * LD64];  // N rows of this CTA
+  float yt[kBufs][kRows * LD64];  // Y^T rows of this CTA
+  float st[2][kRows * LD64];      // the state rows, current and next (TF32 values but the last)
+  float os[2][C * 36];            // output staging [t][i], two chunks
 };
 
 __device__ __forceinline__ void cp_async16(void* dst, const void* src) {
@@ -538,7 +579,32 @@ __device__ __forceinline__ void load_record(StateSmem& s, int buf, const float* 
   }
 }
 
-// One CTA per (value head, 32 state rows): the chunks in order.
+// O rows of chunk c from the staging buffer: 64 tokens x 32 values, 8 per thread.
+__device__ __forceinline__ void store_out(const GdnArgs& a, const float* os, int c, int h, int i0, int tid) {
+  const int t = tid >> 2, part = tid & 3;
+  const int64_t tok = static_cast<int64_t>(c) * C + t;
+  if (tok >= a.T) return;
+  const float* src = &os[t * 36 + 8 * part];
+  uint8_t* dst = a.o + tok * a.ld_o;
+  const int64_t col = static_cast<int64_t>(h) * DV + i0 + 8 * part;
+  if (a.out_f32) {
+    float4* p = reinterpret_cast<float4*>(dst + col * 4);
+    p[0] = make_float4(src[0], src[1], src[2], src[3]);
+    p[1] = make_float4(src[4], src[5], src[6], src[7]);
+  } else {
+    uint32_t w[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const __nv_bfloat162 b = __floats2bfloat162_rn(src[2 * i], src[2 * i + 1]);
+      w[i] = *reinterpret_cast<const uint32_t*>(&b);
+    }
+    *reinterpret_cast<uint4*>(dst + col * 2) = make_uint4(w[0], w[1], w[2], w[3]);
+  }
+}
+
+// One CTA per (value head, 32 state rows): the chunks in order, one block
+// barrier per chunk.  Chunk c's record lands in buffer c % 3 (requested two
+// chunks ahead); its output goes out from the staging buffer during chunk c + 1.
 __global__ void __launch_bounds__(kThreads, 1) gdn_state_kernel(const __grid_constant__ GdnArgs a) {
   extern __shared__ __align__(16) uint8_t smem_raw[];
   StateSmem& s = *reinterpret_cast<StateSmem*>(smem_raw);
@@ -554,23 +620,28 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_state_kernel(const __grid_con
   cp_async_commit();
   if (a.nchunks > 1) load_record(s, 1, rec_of(1), i0, tid);
   cp_async_commit();
-  // entering state
+  // entering state, as the TF32 operand it is used as
   for (int idx = tid; idx < kRows * DK; idx += kThreads) {
     const int r = idx / DK, col = idx % DK;
-    s.st[0][r * LD64 + col] = a.h0 ? a.h0[(static_cast<int64_t>(h) * DV + i0 + r) * DK + col] : 0.0f;
+    const float v = a.h0 ? a.h0[(static_cast<int64_t>(h) * DV + i0 + r) * DK + col] : 0.0f;
+    s.st[0][r * LD64 + col] = __uint_as_float(tf32(v));
   }
   int cur = 0;
   for (int c = 0; c < a.nchunks; ++c) {
-    const int buf = c & 1;
+    const int buf = c % kBufs;
     cp_async_wait_1();
     __syncthreads();
+    // buffer (c + 2) % 3 was last read during chunk c - 1
+    if (c + 2 < a.nchunks) load_record(s, (c + 2) % kBufs, rec_of(c + 2), i0, tid);
+    cp_async_commit();
+    if (c > 0) store_out(a, s.os[(c - 1) & 1], c - 1, h, i0, tid);
     // D[i][n] = sum_k S[i][k] Bc[n][k]: n < 64 -> (S M)[i][n], n >= 64 -> (S R^T)[i][t = n - 64]
     {
       uint32_t af[2][8][4];
 #pragma unroll
       for (int mt = 0; mt < 2; ++mt)
 #pragma unroll
-        for (int ks = 0; ks < 8; ++ks) frag_a(af[mt][ks], s.st[cur], LD64, 16 * mt, 8 * ks, gid, tig);
+        for (int ks = 0; ks < 8; ++ks) frag_a_raw(af[mt][ks], s.st[cur], LD64, 16 * mt, 8 * ks, gid, tig);
       // two accumulators per tile (even and odd k-steps) halve the dependent MMA chain
       float d[2][2][4], d2[2][2][4];
 #pragma unroll
@@ -585,7 +656,7 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_state_kernel(const __grid_con
 #pragma unroll
         for (int nt = 0; nt < 2; ++nt) {
           uint32_t b0, b1;
-          frag_bt(b0, b1, s.bc[buf], LD64, nbase + 8 * nt, 8 * ks, gid, tig);
+          frag_bt_raw(b0, b1, s.bc[buf], LD64, nbase + 8 * nt, 8 * ks, gid, tig);
           mma((ks & 1) ? d2[0][nt] : d[0][nt], af[0][ks], b0, b1);
           mma((ks & 1) ? d2[1][nt] : d[1][nt], af[1][ks], b0, b1);
         }
@@ -596,6 +667,8 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_state_kernel(const __grid_con
 #pragma unroll
           for (int e = 0; e < 4; ++e) d[mt][nt][e] += d2[mt][nt][e];
       if (warp < 4) {
+        // the next state: FP32 after the last chunk (it is the result), else the TF32 operand
+        const bool last = c + 1 == a.nchunks;
 #pragma unroll
         for (int mt = 0; mt < 2; ++mt)
 #pragma unroll
@@ -604,10 +677,15 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_state_kernel(const __grid_con
             for (int hh = 0; hh < 2; ++hh) {
               const int r = 16 * mt + gid + 8 * hh, col = nbase + 8 * nt + 2 * tig;
               const float2 n2 = *reinterpret_cast<const float2*>(&s.nn[buf][r * LD64 + col]);
-              *reinterpret_cast<float2*>(&s.st[cur ^ 1][r * LD64 + col]) =
-                  make_float2(d[mt][nt][2 * hh] + n2.x, d[mt][nt][2 * hh + 1] + n2.y);
+              float v0 = d[mt][nt][2 * hh] + n2.x, v1 = d[mt][nt][2 * hh + 1] + n2.y;
+              if (!last) {
+                v0 = __uint_as_float(tf32(v0));
+                v1 = __uint_as_float(tf32(v1));
+              }
+              *reinterpret_cast<float2*>(&s.st[cur ^ 1][r * LD64 + col]) = make_float2(v0, v1);
             }
       } else {
+        float* os = s.os[c & 1];
 #pragma unroll
         for (int mt = 0; mt < 2; ++mt)
 #pragma unroll
@@ -616,41 +694,16 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_state_kernel(const __grid_con
             for (int e = 0; e < 4; ++e) {
               const int r = 16 * mt + gid + (e >= 2 ? 8 : 0);
               const int t = nbase - 64 + 8 * nt + 2 * tig + (e & 1);
-              s.os[t * 36 + r] = d[mt][nt][e] + s.yt[buf][r * LD64 + t];
+              os[t * 36 + r] = d[mt][nt][e] + s.yt[buf][r * LD64 + t];
             }
-      }
-    }
-    __syncthreads();
-    if (c + 2 < a.nchunks) load_record(s, buf, rec_of(c + 2), i0, tid);
-    cp_async_commit();
-    // O rows of this chunk: 64 tokens x 32 values
-    {
-      const int t = tid >> 2, part = tid & 3;
-      const int64_t tok = static_cast<int64_t>(c) * C + t;
-      if (tok < a.T) {
-        const float* src = &s.os[t * 36 + 8 * part];
-        uint8_t* dst = a.o + tok * a.ld_o;
-        const int64_t col = static_cast<int64_t>(h) * DV + i0 + 8 * part;
-        if (a.out_f32) {
-          float4* p = reinterpret_cast<float4*>(dst + col * 4);
-          p[0] = make_float4(src[0], src[1], src[2], src[3]);
-          p[1] = make_float4(src[4], src[5], src[6], src[7]);
-        } else {
-          uint32_t w[4];
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const __nv_bfloat162 b = __floats2bfloat162_rn(src[2 * i], src[2 * i + 1]);
-            w[i] = *reinterpret_cast<const uint32_t*>(&b);
-          }
-          *reinterpret_cast<uint4*>(dst + col * 2) = make_uint4(w[0], w[1], w[2], w[3]);
-        }
       }
     }
     cur ^= 1;
   }
   cp_async_wait_all();
+  __syncthreads();
+  if (a.nchunks > 0) store_out(a, s.os[(a.nchunks - 1) & 1], a.nchunks - 1, h, i0, tid);
   if (a.h_out) {
-    __syncthreads();
     for (int idx = tid; idx < kRows * DK; idx += kThreads) {
       const int r = idx / DK, col = idx % DK;
       a.h_out[(static_cast<int64_t>(h) * DV + i0 + r) * DK + col] = s.st[cur][r * LD64 + col];
