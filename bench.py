@@ -38,7 +38,7 @@ ROTATE = 4          # rotating input sets so consecutive steps miss in L2
 # recurrence launches, captured at 8192 tokens and scaled by 4 (all of it is per chunk).
 TRAFFIC_BYTES = {
     "actstats": 339406592,
-    "gdnrec": 3791627264,
+    "gdnrec": 3817484288,
     "decode1": 50362112,
     "decode64": 50922752,
     "decode8": 50422528,
