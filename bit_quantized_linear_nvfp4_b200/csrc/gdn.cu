@@ -116,22 +116,14 @@ __device__ __forceinline__ void frag_a(uint32_t (&a)[4], const float* X, int ld,
   a[2] = tf32(X[(m0 + gid) * ld + k0 + tig + 4]);
   a[3] = tf32(X[(m0 + gid + 8) * ld + k0 + tig + 4]);
 }
-// A[m][k] = s[k] X[k][m] (X stored with k as the row).
-__device__ __forceinline__ void frag_at(uint32_t (&a)[4], const float* X, int ld, const float* s, int m0, int k0,
-                                        int gid, int tig) {
-  const float s0 = s ? s[k0 + tig] : 1.0f, s1 = s ? s[k0 + tig + 4] : 1.0f;
-  a[0] = tf32(s0 * X[(k0 + tig) * ld + m0 + gid]);
-  a[1] = tf32(s0 * X[(k0 + tig) * ld + m0 + gid + 8]);
-  a[2] = tf32(s1 * X[(k0 + tig + 4) * ld + m0 + gid]);
-  a[3] = tf32(s1 * X[(k0 + tig + 4) * ld + m0 + gid + 8]);
-}
 // B[k][n] = X[n][k] (X stored with n as the row).
 __device__ __forceinline__ void frag_bt(uint32_t& b0, uint32_t& b1, const float* X, int ld, int n0, int k0, int gid,
                                         int tig) {
   b0 = tf32(X[(n0 + gid) * ld + k0 + tig]);
   b1 = tf32(X[(n0 + gid) * ld + k0 + tig + 4]);
 }
-// The same two loaders for values already rounded to TF32 (no conversion).
+// Loaders for values already rounded to TF32 (no conversion); frag_at_raw
+// reads A[m][k] = X[k][m] (X stored with k as the row).
 __device__ __forceinline__ void frag_a_raw(uint32_t (&a)[4], const float* X, int ld, int m0, int k0, int gid, int tig) {
   a[0] = __float_as_uint(X[(m0 + gid) * ld + k0 + tig]);
   a[1] = __float_as_uint(X[(m0 + gid + 8) * ld + k0 + tig]);
