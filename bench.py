@@ -118,19 +118,28 @@ def dist_env():
     return world, rank, local
 
 
-def dist_init(world):
+def dist_init(world, backend=None):
+    """Process group for N > 1 replicas: NCCL on GPUs (gloo for host-only runs
+    of the timing plumbing).  Replicas exchange only the timing maximum and
+    barriers; the path itself has no collective."""
     if world <= 1:
         return None
     import datetime
+    import torch
     import torch.distributed as dist
-    dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    if backend is None:
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+    dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
     return dist
 
 
 def dist_max(dist, value: float, device) -> float:
+    """Max over ranks (device-timed milliseconds)."""
     if dist is None:
         return value
     import torch
+    if dist.get_backend() == "gloo":
+        device = "cpu"
     t = torch.tensor([value], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
