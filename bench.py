@@ -1072,6 +1072,25 @@ def _gdnrec_oracle_baseline(seconds, steps=None):
             "host_cpus": os.cpu_count()}
 
 
+REFERENCE_BUDGET_S = 60.0  # timed oracle work of one reference-arm run, at most
+
+
+def _time_oracle(fn, steps, warmup, budget_s=REFERENCE_BUDGET_S):
+    """Run the oracle step fn min(warmup, 3) times untimed, then up to `steps`
+    timed times, stopping once budget_s seconds are spent so that the whole run
+    ends within a few minutes.  Returns (seconds per step, steps timed)."""
+    for _ in range(min(warmup, 3)):
+        fn()
+    t = time.perf_counter()
+    n = 0
+    while n < steps:
+        fn()
+        n += 1
+        if time.perf_counter() - t > budget_s:
+            break
+    return (time.perf_counter() - t) / n, n
+
+
 def run_reference(args):
     world, rank, _ = dist_env()
     if rank != 0:
@@ -1079,10 +1098,11 @@ def run_reference(args):
     if args.workload == "gdnrec":
         for _ in range(min(args.warmup, 1)):
             _gdnrec_oracle_baseline(0.0, steps=1)
-        cb = _gdnrec_oracle_baseline(0.0, steps=max(1, min(args.steps, 20)))
+        n = max(1, min(args.steps, 20))
+        cb = _gdnrec_oracle_baseline(0.0, steps=n)
         val = cb["value"]
         print(json.dumps({"impl": "reference", "metric": METRIC, "value": val, "unit": "GB/s", "n_gpus": world,
-                          "steps": args.steps, "warmup": args.warmup, "ms_per_step": cb["ms_per_pass"],
+                          "steps": n, "steps_requested": args.steps, "warmup": args.warmup, "ms_per_step": cb["ms_per_pass"],
                           "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
                           "dtype": "f64 (oracle)", "data": "synthetic",
                           "config": {"workload": f"gdn_recurrence_{GDN_REC_TOKENS}x32h_dk64_dv128",
@@ -1097,15 +1117,10 @@ def run_reference(args):
         rows = 256
         x = wl.make_x(wl.GDN, rows=rows)
         g = o.global_scale(x)
-        for _ in range(args.warmup):
-            o.activation_stats(x, g)
-        t = time.perf_counter()
-        for _ in range(args.steps):
-            o.activation_stats(x, g)
-        per = (time.perf_counter() - t) / args.steps
+        per, n = _time_oracle(lambda: o.activation_stats(x, g), args.steps, args.warmup)
         val = rows * x.shape[1] * 2 / per / 1e9
         print(json.dumps({"impl": "reference", "metric": METRIC, "value": val, "unit": "GB/s", "n_gpus": world,
-                          "steps": args.steps, "warmup": args.warmup, "ms_per_step": per * 1e3,
+                          "steps": n, "steps_requested": args.steps, "warmup": args.warmup, "ms_per_step": per * 1e3,
                           "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
                           "dtype": "f64 (oracle)", "data": "synthetic",
                           "config": {"workload": "activation_stats_32768x5120", "M": 32768, "K": x.shape[1]},
@@ -1120,15 +1135,10 @@ def run_reference(args):
         rows, C = 2048, 1024
         x = rng.standard_normal((rows, C)).astype(np.float32)
         s = np.float32(np.abs(x).max() / 448)
-        for _ in range(args.warmup):
-            o.kv_fp8_quantize(x, s)
-        t = time.perf_counter()
-        for _ in range(args.steps):
-            o.kv_fp8_quantize(x, s)
-        per = (time.perf_counter() - t) / args.steps
+        per, n = _time_oracle(lambda: o.kv_fp8_quantize(x, s), args.steps, args.warmup)
         val = rows * C * 3 / per / 1e9
         print(json.dumps({"impl": "reference", "metric": METRIC, "value": val, "unit": "GB/s", "n_gpus": world,
-                          "steps": args.steps, "warmup": args.warmup, "ms_per_step": per * 1e3,
+                          "steps": n, "steps_requested": args.steps, "warmup": args.warmup, "ms_per_step": per * 1e3,
                           "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
                           "dtype": "f32 (oracle)", "data": "synthetic",
                           "config": {"workload": "kv_fp8_encode_2x32768x1024", "tokens": 32768, "cols": C},
@@ -1147,16 +1157,11 @@ def run_reference(args):
         s_all = np.concatenate([sf for _, sf, _ in wq])[:rows]
         g_rows = np.repeat(np.array([g for _, _, g in wq], np.float32), [sg.width for sg in w.segments])[:rows]
         g_c = max(g for _, _, g in wq)
-        for _ in range(args.warmup):
-            o.requantize(c_all, s_all, g_rows, g_c)
-        t = time.perf_counter()
-        for _ in range(args.steps):
-            o.requantize(c_all, s_all, g_rows, g_c)
-        per = (time.perf_counter() - t) / args.steps
+        per, n = _time_oracle(lambda: o.requantize(c_all, s_all, g_rows, g_c), args.steps, args.warmup)
         val = 2 * rows * w.K * 0.5625 / per / 1e9
         sample = f"{rows} rows x {w.K} of the GDN weight per step (oracle requantize)"
         print(json.dumps({"impl": "reference", "metric": METRIC, "value": val, "unit": "GB/s", "n_gpus": world,
-                          "steps": args.steps, "warmup": args.warmup, "ms_per_step": per * 1e3,
+                          "steps": n, "steps_requested": args.steps, "warmup": args.warmup, "ms_per_step": per * 1e3,
                           "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
                           "dtype": "f32 (oracle)", "data": "synthetic",
                           "config": {"workload": "requant_gdn_weight_12352x5120", "N": 12352, "K": w.K},
@@ -1168,13 +1173,8 @@ def run_reference(args):
     w, x, wq, g_a, extra = _prepare_oracle(args.workload)
     K = x.shape[1]
     rows = 16
-    for _ in range(args.warmup):
-        _oracle_sample_step(args.workload, rows, x, wq, g_a, extra)
-    t = time.perf_counter()
-    for _ in range(args.steps):
-        _oracle_sample_step(args.workload, rows, x, wq, g_a, extra)
-    el = time.perf_counter() - t
-    per = el / args.steps
+    per, n = _time_oracle(lambda: _oracle_sample_step(args.workload, rows, x, wq, g_a, extra), args.steps,
+                          args.warmup)
     if w is not None:
         val, unit = 2.0 * rows * w.N * K / per / 1e12, "TFLOP/s"
         cfg = {"workload": w.name, "M": w.M, "N": w.N, "K": w.K}
@@ -1183,7 +1183,7 @@ def run_reference(args):
         cfg = {"workload": "quant", "M": x.shape[0], "K": K}
     sample = f"{rows} rows of the workload per step (quantise + FP64 GEMM + epilogue)"
     line = {"impl": "reference", "metric": METRIC, "value": val, "unit": unit, "n_gpus": world,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": per * 1e3, "higher_is_better": True,
+            "steps": n, "steps_requested": args.steps, "warmup": args.warmup, "ms_per_step": per * 1e3, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64 (oracle)", "data": "synthetic",
             "config": cfg,
             "cpu_baseline": {"value": val, "unit": unit, "cores": _blas_threads(), "kind": "oracle", "sample": sample},
