@@ -726,8 +726,8 @@ size_t gdn_workspace_bytes(int64_t T, int64_t H) {
 
 cudaError_t launch_gdn(const GdnProblem& p, cudaStream_t stream) {
   using namespace gdn;
-  static bool attr_set = false;
-  if (!attr_set) {
+  static std::atomic<uint64_t> attr_done{0};
+  cudaError_t ea = once_per_device(attr_done, [] {
     cudaError_t e = cudaFuncSetAttribute(gdn_prep_kernel<NVFP4_DTYPE_BF16>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, sizeof(PrepSmem));
     if (e == cudaSuccess)
@@ -735,9 +735,9 @@ cudaError_t launch_gdn(const GdnProblem& p, cudaStream_t stream) {
                                sizeof(PrepSmem));
     if (e == cudaSuccess)
       e = cudaFuncSetAttribute(gdn_state_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, sizeof(StateSmem));
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
+    return e;
+  });
+  if (ea != cudaSuccess) return ea;
   const int esz = p.in_dtype == NVFP4_DTYPE_BF16 ? 2 : 4;
   GdnArgs a{};
   a.q = static_cast<const uint8_t*>(p.q);

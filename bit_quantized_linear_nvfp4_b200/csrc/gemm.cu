@@ -1023,12 +1023,11 @@ cudaError_t launch_gemm(const GemmProblem& p, void*, size_t, cudaStream_t stream
   const int tiles = a.num_m_blocks * a.num_n_blocks;
   if (tiles == 0) return cudaSuccess;
   if (!pair_kernel) {
-    static bool attr_set = false;
-    if (!attr_set) {
-      cudaError_t e = cudaFuncSetAttribute(gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
-      if (e != cudaSuccess) return e;
-      attr_set = true;
-    }
+    static std::atomic<uint64_t> attr_done{0};
+    cudaError_t ea = once_per_device(attr_done, [] {
+      return cudaFuncSetAttribute(gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+    });
+    if (ea != cudaSuccess) return ea;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(tiles < sms ? tiles : sms);
     cfg.blockDim = dim3(kThreads);
@@ -1059,12 +1058,11 @@ cudaError_t launch_gemm(const GemmProblem& p, void*, size_t, cudaStream_t stream
     CUtensorMap tm_b3, tm_sfb3;
     if (!make_codes_map(&tm_b3, p.w_codes, p.N, p.K, kBRows3) || !make_sf_map(&tm_sfb3, p.w_sf, p.N, p.K, 4, kSFBBlocks3))
       return cudaErrorInvalidValue;
-    static bool attr3_set = false;
-    if (!attr3_set) {
-      cudaError_t e = cudaFuncSetAttribute(gemm_pair_db_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes3);
-      if (e != cudaSuccess) return e;
-      attr3_set = true;
-    }
+    static std::atomic<uint64_t> attr3_done{0};
+    cudaError_t ea = once_per_device(attr3_done, [] {
+      return cudaFuncSetAttribute(gemm_pair_db_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes3);
+    });
+    if (ea != cudaSuccess) return ea;
     const int tiles3 = b.num_m_blocks * b.num_n_blocks;
     const int pairs3 = tiles3 < sms / 2 ? tiles3 : sms / 2;
     cudaLaunchConfig_t cfg = {};
@@ -1087,12 +1085,11 @@ cudaError_t launch_gemm(const GemmProblem& p, void*, size_t, cudaStream_t stream
   if (!make_sf_map(&tm_sfa4, p.a_sf, p.M, p.K, 4 * kSFGroup, 1) || !make_sf_map(&tm_sfb4, p.w_sf, p.N, p.K, 4 * kSFGroup, 1) ||
       !make_sf_map(&tm_sfb8, p.w_sf, p.N, p.K, 4 * kSFGroup, 2))
     return cudaErrorInvalidValue;
-  static bool attr2_set = false;
-  if (!attr2_set) {
-    cudaError_t e = cudaFuncSetAttribute(gemm_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes2);
-    if (e != cudaSuccess) return e;
-    attr2_set = true;
-  }
+  static std::atomic<uint64_t> attr2_done{0};
+  cudaError_t ea = once_per_device(attr2_done, [] {
+    return cudaFuncSetAttribute(gemm_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes2);
+  });
+  if (ea != cudaSuccess) return ea;
   const int pairs = tiles < sms / 2 ? tiles : sms / 2;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(2 * pairs);

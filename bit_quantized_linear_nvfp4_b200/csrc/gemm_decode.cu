@@ -425,12 +425,11 @@ cudaError_t launch_bn(const GemmProblem& p, cudaStream_t stream) {
   if (S > a.num_k_stages) S = a.num_k_stages;
   if (S < 1) S = 1;
   a.split = S;
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(decode_kernel<BN, CH>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
+  static std::atomic<uint64_t> attr_done{0};
+  cudaError_t ea = once_per_device(attr_done, [] {
+    return cudaFuncSetAttribute(decode_kernel<BN, CH>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+  });
+  if (ea != cudaSuccess) return ea;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(rbs * S);
   cfg.blockDim = dim3(kThreads);

@@ -1,6 +1,7 @@
 // Internal host-side interfaces between the C ABI layer and the kernels.
 #pragma once
 
+#include <atomic>
 #include <cstddef>
 #include <cstdint>
 #include <cuda_runtime.h>
@@ -18,6 +19,21 @@ struct RowSegments {
 };
 
 inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+// Runs set() -- raising a kernel's dynamic shared-memory limit, which is a
+// per-device setting -- once for each device a process launches on.  `done`
+// holds one bit per device (devices 64 and up set it on every launch).
+template <class F>
+cudaError_t once_per_device(std::atomic<uint64_t>& done, F set) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const uint64_t bit = dev < 64 ? (uint64_t{1} << dev) : 0;
+  if (bit != 0 && (done.load(std::memory_order_acquire) & bit) != 0) return cudaSuccess;
+  e = set();
+  if (e == cudaSuccess && bit != 0) done.fetch_or(bit, std::memory_order_acq_rel);
+  return e;
+}
 inline size_t sf_bytes(int64_t rows, int64_t K) {
   return static_cast<size_t>(ceil_div(rows, 128) * 128) * static_cast<size_t>(ceil_div(K, 64) * 4);
 }

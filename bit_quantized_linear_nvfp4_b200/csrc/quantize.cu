@@ -671,12 +671,11 @@ cudaError_t launch_pdl(Kern kern, int grid, int cluster, int smem, const QuantAr
 template <int DTYPE, bool WIDE>
 cudaError_t launch_t(QuantArgs a, bool dynamic, cudaStream_t stream) {
   using C = Cfg<DTYPE>;
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(small_kernel<DTYPE>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmallSmem);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
+  static std::atomic<uint64_t> attr_done{0};
+  cudaError_t ea = once_per_device(attr_done, [] {
+    return cudaFuncSetAttribute(small_kernel<DTYPE>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmallSmem);
+  });
+  if (ea != cudaSuccess) return ea;
   constexpr int64_t kSmallChunks = kSmallSmem / C::kChunkBytes;  // per block
   const int64_t nsmall = (a.items + kSmallChunks - 1) / kSmallChunks;
   if (dynamic && nsmall <= kMaxSmallBlocks) {
