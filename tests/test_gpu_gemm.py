@@ -203,6 +203,70 @@ def test_full_size_oproj_sampled_rows():
     check_bf16(to_np(out[torch.from_numpy(rows).to(DEV)]), acc * s, TOL_ACC * mag * s, "oproj")
 
 
+def _check_gdn_sampled(x, segs, a_log, dt_bias, rows, outs_rows, g_gpu, ga_gpu, w):
+    """Oracle of the sampled rows of a full-size fused GDN projection, and the
+    comparison (outs_rows: the GPU outputs of those rows, per segment)."""
+    g_a = o.global_scale(x)
+    assert np.float32(ga_gpu) == g_a
+    wq = [o.quantize(sg) for sg in segs]
+    np.testing.assert_array_equal(g_gpu, np.array([g for _, _, g in wq], np.float32))
+    aq = o.quantize(x[rows], g_a)
+    o_outs, pre = o.fused_projection(aq, [(c, sf) for c, sf, _ in wq], [g for _, _, g in wq],
+                                     [sg.epilogue for sg in w.segments], (a_log, dt_bias))
+    _check_gdn(outs_rows, o_outs, pre, a_log, dt_bias, w)
+
+
+@pytest.mark.slow
+def test_full_size_gdn_sampled_rows():
+    """The fused GDN in-projection at full size, 32768x12352x5120 (activations
+    larger than L2: the grouped rasterisation) in the launch configuration the
+    benchmark times; 512 sampled rows (rows 0 and M-1 included) x all columns."""
+    w = wl.GDN
+    x = wl.make_x(w)
+    segs = wl.make_w_segments(w)
+    a_log, dt_bias = wl.make_gate_params(w)
+    outs, g_gpu, ga = _run_fused(w, x, segs, a_log, dt_bias)
+    rows = wl.sample_rows(w.M, 512)
+    rows_t = torch.from_numpy(rows).to(DEV)
+    _check_gdn_sampled(x, segs, a_log, dt_bias, rows, [t[rows_t] for t in outs], g_gpu, ga, w)
+
+
+def _check_swiglu_sampled(x, gate, up, rows, out_rows, gw_gpu, ga_gpu, label):
+    """Oracle of sampled rows of a fused gate+up projection with SwiGLU, and
+    the comparison with the tolerance propagated through silu(g) * u."""
+    g_a = o.global_scale(x)
+    assert np.float32(ga_gpu) == g_a
+    gq, uq = o.quantize(gate), o.quantize(up)
+    np.testing.assert_array_equal(gw_gpu, np.array([gq[2], uq[2]], np.float32))
+    aq = o.quantize(x[rows], g_a)
+    outs, pre = o.fused_projection(aq, [gq[:2], uq[:2]], [gq[2], uq[2]], ["swiglu_gate", "swiglu_up"])
+    yg, mg = pre[0]
+    yu, mu = pre[1]
+    sg = o.sigmoid(yg)
+    dsilu = sg * (1 + yg * (1 - sg))
+    tol = np.abs(dsilu * yu) * TOL_ACC * mg + np.abs(yg * sg) * TOL_ACC * mu + 8 * f32_ulp(outs[0])
+    check_bf16(out_rows, outs[0], tol, label)
+
+
+@pytest.mark.slow
+def test_full_size_mlp_sampled_rows():
+    """The fused MLP gate+up with SwiGLU at full size, 8192x34816x5120, in the
+    launch configuration the benchmark times; 256 sampled rows x all columns."""
+    w = wl.MLP
+    x = wl.make_x(w)
+    gate, up = wl.make_w_segments(w)
+    H = gate.shape[0]
+    A, ga = nv.nvfp4_quantize(_dev(x))
+    W, gw = nv.nvfp4_quantize_segments(_dev(np.concatenate([gate, up])), [0, H, 2 * H])
+    out = torch.empty((w.M, H), dtype=torch.bfloat16, device=DEV)
+    nv.nvfp4_fused_proj(A, ga, W, gw, [nv.Segment(0, H, "swiglu_gate", out), nv.Segment(H, 2 * H, "swiglu_up")])
+    torch.cuda.synchronize()
+    rows = wl.sample_rows(w.M, 256)
+    out_rows = to_np(out[torch.from_numpy(rows).to(DEV)])
+    del out, W, A
+    _check_swiglu_sampled(x, gate, up, rows, out_rows, gw.cpu().numpy(), float(ga.item()), "mlp full size")
+
+
 # ---------------------------------------------------------------- decode path (M <= 64)
 
 @pytest.mark.parametrize("M", [1, 5, 8, 64])
