@@ -199,3 +199,36 @@ def test_row_norms_bound_the_output():
     out, _, rn = o.gdn_recurrence(q, k, v, beta, g, row_norms=True)
     qn = np.linalg.norm(o.l2_normalise(q) * dk ** -0.5, axis=2)  # [T, H]
     assert np.all(np.abs(out) <= rn * qn[:, :, None] * (1 + 1e-12) + 1e-15)
+
+
+def _max_inverse_norm(q, k, beta, g, H, hk, C=64):
+    """Largest spectral norm of L = (I + A)^-1 over every (chunk, head), with
+    A[t][j] = beta_t exp(gam_t - gam_j) k_t.k_j (j < t) from unit keys."""
+    T = beta.shape[0]
+    kn = o.l2_normalise(np.repeat(k.reshape(T, hk, -1), H // hk, axis=1))
+    worst = 0.0
+    for c0 in range(0, T, C):
+        c1 = min(T, c0 + C)
+        n = c1 - c0
+        for h in range(H):
+            K = kn[c0:c1, h]
+            gam = np.cumsum(g[c0:c1, h].astype(np.float64))
+            A = np.tril(beta[c0:c1, h][:, None] * np.exp(gam[:, None] - gam[None, :]) * (K @ K.T), -1)
+            L = np.linalg.inv(np.eye(n) + A)
+            worst = max(worst, float(np.linalg.norm(L, 2)))
+    return worst
+
+
+def test_recurrence_tolerance_premise():
+    """The GPU tolerance of the chunked recurrence (2^-6 |S_t[i,:]| |q_t|) assumes
+    |(I + A)^-1| <= 4 for every chunk; check it on the parity cases' inputs."""
+    from bit_quantized_linear_nvfp4_b200 import workloads as wl
+    cases = [(150, 4, 2, 150 + 68, False), (321, 2, 2, 321 + 34, False), (64, 3, 3, 64 + 51, False),
+             (1, 2, 1, 1 + 34, False), (40, 8, 2, 40 + 136, False), (2000, 2, 2, 5, True), (200, 2, 2, 6, False),
+             (225, 2, 2, 7, False), (100, 2, 2, 9, False), (150, 2, 2, 21, False)]
+    for T, H, hk, seed, slow in cases:
+        q, k, v, beta, g = wl.make_recurrence_inputs(T, H, hk, seed, "bf16", slow)
+        assert _max_inverse_norm(q, k, beta, g, H, hk) <= 4.0, (T, H, seed)
+    # the full-length case: 32768 tokens x 32 heads
+    q, k, v, beta, g = wl.make_recurrence_inputs(32768, 32, 32, 11, "bf16")
+    assert _max_inverse_norm(q, k, beta, g, 32, 32) <= 4.0
