@@ -332,6 +332,23 @@ def test_full_size_decode(M):
     check_bf16(to_np(out), y, TOL_ACC * mag, f"decode M={M}")
 
 
+@pytest.mark.parametrize("M", [8, 64])
+def test_full_size_decode_fp32_accumulation(M):
+    """Decode down_proj W[5120,17408] with FP32 output, every element: the
+    accumulation over K = 17408 against the 1e-5 * sum|a w| bound (the ratio is
+    printed; on B200 it measured 4e-4 of the bound)."""
+    w = wl.decode_workload(M)
+    x = wl.make_x(w)
+    wt = wl.make_w_segment(w, 0)
+    A, ga = nv.nvfp4_quantize(_dev(x))
+    W, gw = nv.nvfp4_quantize(_dev(wt))
+    out = nv.nvfp4_gemm(A, ga, W, gw, out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    y, mag, _, _ = o.linear(x, wt)
+    ratio = check_fp32(to_np(out), y, mag, f"decode M={M} fp32")
+    print(f"decode M={M} K=17408 FP32: max error / bound = {ratio:.2e}")
+
+
 def test_wide_tiles_two_segments():
     """A shape that runs the 256-wide overlapped-accumulator kernel for a
     non-SwiGLU projection (one M block, N just above 74 x 192), with a BF16
