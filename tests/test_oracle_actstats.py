@@ -51,6 +51,12 @@ def test_dominated_blocks_and_exact_values():
     assert o.activation_summary(o.activation_stats(x))["dominated_share"] == 1.0
     y = np.full((4, 64), 0.3, np.float32)
     assert o.activation_summary(o.activation_stats(y))["dominated_share"] == 0.0
+    # dominance compares magnitudes: sixteen equal negative values are not
+    # dominated, and one large negative value among small ones is
+    assert o.activation_summary(o.activation_stats(-y))["dominated_share"] == 0.0
+    z = np.full((1, 16), 0.1, np.float32)
+    z[0, 3] = -5.0
+    assert o.activation_stats(z)["dominated"] == 1.0
     # a tensor NVFP4 represents exactly: every block holds +-6, so S = 448, and
     # the global scale 6 * 0.4375 / 2688 = 2^-10 is exact, as is e2m1 * S * g
     vals = (np.array([0.5, 1, 1.5, 2, 3, 4, 6, -6] * 8, np.float32) * np.float32(0.4375)).reshape(4, 16)

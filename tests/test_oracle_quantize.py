@@ -43,6 +43,21 @@ def test_tensor_max_block_gets_448():
     assert codes[r, c] & 7 == 7
 
 
+def test_block_max_maps_to_the_top_code():
+    """The largest value of a block fixes its scale: with the scale byte in
+    E4M3's normal, unsaturated range, the block maximum lands within E4M3's
+    relative rounding (2^-4) of 6, so it is coded as +-6 (code magnitude 7),
+    never as 4 or below."""
+    x = _rand((32, 256), 9, outliers=(3, 77))
+    codes, sf, g = o.quantize(x)
+    S = o.e4m3_decode(sf)
+    xb = np.abs(x).reshape(32, 16, 16)
+    top = np.take_along_axis(codes.reshape(32, 16, 16), np.argmax(xb, axis=2)[:, :, None], axis=2)[:, :, 0]
+    normal = (S >= 2.0 ** -6) & (sf < 0x7E)
+    assert normal.sum() > 400
+    assert np.all(top[normal] & 7 == 7)
+
+
 def _grid_step(mag):
     return np.where(mag < 2, 0.5, np.where(mag < 4, 1.0, 2.0))
 
