@@ -41,6 +41,10 @@ def test_gaussian_and_heavy_tailed_moments():
     s = o.activation_summary(o.activation_stats(x))
     assert abs(s["kurtosis"] - 3.0) < 0.05
     assert 4.0 < s["max_over_rms"] < 6.5  # the largest of 0.5 M normals sits near 5 sigma
+    # both are scale-free: x4 (exact in FP32) changes neither
+    s4 = o.activation_summary(o.activation_stats(4 * x))
+    assert abs(s4["kurtosis"] - s["kurtosis"]) <= 1e-9 * s["kurtosis"]
+    assert abs(s4["max_over_rms"] - s["max_over_rms"]) <= 1e-12 * s["max_over_rms"]
     t = rng.standard_t(3, (512, 1024)).astype(np.float32)
     assert o.activation_summary(o.activation_stats(t))["kurtosis"] > 10
 
@@ -72,4 +76,5 @@ def test_a4_error_within_the_half_step_bound_and_hot_channel():
     s = o.activation_summary(st)
     # the element error is at most half the top grid step (1 * S * g) and S * g <= amax_b / 5.5 or so: well below 25%
     assert 0.0 < s["a4_err_max"] < 0.25 and s["a4_err_min"] > 0.0
-    assert 60 < s["hot_channel_ratio"] < 140
+    # one channel x100 over N(0, 1) channels: about 100, within the sampling of 256 rows
+    assert 92 < s["hot_channel_ratio"] < 112

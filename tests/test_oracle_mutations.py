@@ -54,6 +54,34 @@ MUTANTS = [
      "test_oracle_gdn", ["test_pure_decay_closed_form", "test_orthonormal_keys_give_linear_attention"]),
     ("value heads mapped to q/k heads cyclically", "gdn_recurrence", "qh = np.repeat(q, rep, axis=1)",
      "qh = np.tile(q, (1, rep, 1))", "test_oracle_gdn", ["test_shared_query_key_heads"]),
+    ("write strength not applied", "gdn_recurrence", "u = beta[t][:, None] * (", "u = (", "test_oracle_gdn",
+     ["test_orthonormal_keys_give_linear_attention", "test_chunked_form_agrees"]),
+    ("L2 norm without the square root", "l2_normalise", "np.sqrt((x * x).sum(axis=-1, keepdims=True) + eps)",
+     "((x * x).sum(axis=-1, keepdims=True) + eps)", "test_oracle_gdn",
+     ["test_write_overwrites_along_the_key", "test_pure_decay_closed_form"]),
+    ("E2M1 exponent bias off by one", "e2m1_value", "2.0 ** (e - 1)", "2.0 ** e", "test_oracle_codecs",
+     ["test_e2m1_values_match_golden", "test_e2m1_decode_table_vs_ml_dtypes"]),
+    ("E4M3 exponent bias off by one", "e4m3_value", "2.0 ** (e - 7)", "2.0 ** (e - 8)", "test_oracle_codecs",
+     ["test_e4m3_values_match_golden", "test_e4m3_decode_all_256_vs_torch"]),
+    ("E4M3 subnormal step wrong", "e4m3_value", "(m / 8.0) * 2.0 ** -6", "(m / 8.0) * 2.0 ** -7",
+     "test_oracle_codecs", ["test_e4m3_values_match_golden", "test_e4m3_decode_all_256_vs_torch"]),
+    ("dequantise without the global scale", "dequantize", "* np.float64(g)", "* 1.0", "test_oracle_quantize",
+     ["test_per_element_error_bound", "test_quant_error_magnitude_sane"]),
+    ("every segment takes the first segment's scale", "fused_projection", "np.float64(seg_scales[s])",
+     "np.float64(seg_scales[0])", "test_oracle_gemm", ["test_fused_projection_equals_per_module_linears"]),
+    ("SwiGLU paired with itself", "fused_projection", 'up = epilogues.index("swiglu_up")', "up = s",
+     "test_oracle_gemm", ["test_swiglu_pairing_in_fused_projection"]),
+    ("common scale is the largest", "common_global_scale", "np.min(", "np.max(", "test_oracle_gemm",
+     ["test_common_scale_mismatch_closed_form"]),
+    ("KV decode divides by the scale", "kv_fp8_dequantize", "v * np.float32(scale)", "v / np.float32(scale)",
+     "test_oracle_kvfp8", ["test_bad_scale_gives_zeros_and_decoding_matches_torch",
+                           "test_every_code_round_trips_under_power_of_two_scales"]),
+    ("kurtosis over the variance", "activation_summary", "m4c / var ** 2", "m4c / var", "test_oracle_actstats",
+     ["test_gaussian_and_heavy_tailed_moments"]),
+    ("hot channel against the mean channel", "activation_summary", "col_rms.max() / med",
+     "col_rms.max() / col_rms.mean()", "test_oracle_actstats", ["test_a4_error_within_the_half_step_bound_and_hot_channel"]),
+    ("BF16 rounding truncates", "bf16_round", "np.round(y / q) * q", "np.floor(y / q) * q", "test_oracle_gemm",
+     ["test_bf16_round_and_ulp"]),
 ]
 
 
