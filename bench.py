@@ -405,6 +405,10 @@ def run_product(args):
 
     # end to end through host buffers: pinned X in, result out, every step
     e2e = measure_e2e(step, K, Wm, stream)
+    # whole job: the slowest rank's time, every rank's work
+    e2e_ms = dist_max(dist, e2e["ms_per_step"], device)
+    e2e["value"] = e2e["value"] * e2e["ms_per_step"] / e2e_ms * world
+    e2e["ms_per_step"] = e2e_ms
 
     qb = step.alg_bytes_quant()
     hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
@@ -656,7 +660,7 @@ def run_requant(args):
         e2e_one()
     b.record(stream)
     torch.cuda.synchronize()
-    ms_e2e = a.elapsed_time(b) / Kst
+    ms_e2e = dist_max(dist, a.elapsed_time(b) / Kst, device)  # max over ranks
     line = {
         "metric": METRIC, "value": bytes_step * world / (ms * 1e-3) / 1e9, "unit": "GB/s", "n_gpus": world,
         "steps": Kst, "warmup": Wm, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
@@ -668,7 +672,7 @@ def run_requant(args):
                      "traffic": TRAFFIC_BYTES.get("requant"), "peak_source": f"{peak_src} copy bandwidth",
                      "kernel": "nvfp4 requantize", "ms_per_launch": ms},
         "clocks": clk,
-        "e2e": {"value": bytes_step / (ms_e2e * 1e-3) / 1e9, "unit": "GB/s", "h2d_bytes_per_step": per_set,
+        "e2e": {"value": bytes_step * world / (ms_e2e * 1e-3) / 1e9, "unit": "GB/s", "h2d_bytes_per_step": per_set,
                 "d2h_bytes_per_step": per_set, "ms_per_step": ms_e2e},
         "gpu_launches": Kst,
     }
@@ -777,7 +781,7 @@ def run_kvfp8(args):
         e2e_one()
     b.record(stream)
     torch.cuda.synchronize()
-    ms_e2e = a.elapsed_time(b) / Kst
+    ms_e2e = dist_max(dist, a.elapsed_time(b) / Kst, device)  # max over ranks
     line = {
         "metric": METRIC, "value": bytes_step * world / (ms * 1e-3) / 1e9, "unit": "GB/s", "n_gpus": world,
         "steps": Kst, "warmup": Wm, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
@@ -789,7 +793,7 @@ def run_kvfp8(args):
                      "traffic": TRAFFIC_BYTES.get("kvfp8"), "peak_source": f"{peak_src} copy bandwidth",
                      "kernel": "nvfp4 kv fp8 encode", "ms_per_launch": ms / 2},
         "clocks": clk,
-        "e2e": {"value": bytes_step / (ms_e2e * 1e-3) / 1e9, "unit": "GB/s", "h2d_bytes_per_step": 2 * T * C * 2,
+        "e2e": {"value": bytes_step * world / (ms_e2e * 1e-3) / 1e9, "unit": "GB/s", "h2d_bytes_per_step": 2 * T * C * 2,
                 "d2h_bytes_per_step": 2 * T * C, "ms_per_step": ms_e2e},
         "gpu_launches": 2 * Kst,
     }
@@ -882,7 +886,7 @@ def run_actstats(args):
         e2e_one()
     b.record(stream)
     torch.cuda.synchronize()
-    ms_e2e = a.elapsed_time(b) / Kst
+    ms_e2e = dist_max(dist, a.elapsed_time(b) / Kst, device)  # max over ranks
     line = {
         "metric": METRIC, "value": bytes_step * world / (ms * 1e-3) / 1e9, "unit": "GB/s", "n_gpus": world,
         "steps": Kst, "warmup": Wm, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
@@ -894,7 +898,7 @@ def run_actstats(args):
                      "traffic": TRAFFIC_BYTES.get("actstats"), "peak_source": f"{peak_src} copy bandwidth",
                      "kernel": "nvfp4 activation stats", "ms_per_launch": ms},
         "clocks": clk,
-        "e2e": {"value": bytes_step / (ms_e2e * 1e-3) / 1e9, "unit": "GB/s", "h2d_bytes_per_step": bytes_step,
+        "e2e": {"value": bytes_step * world / (ms_e2e * 1e-3) / 1e9, "unit": "GB/s", "h2d_bytes_per_step": bytes_step,
                 "d2h_bytes_per_step": 64, "ms_per_step": ms_e2e},
         "gpu_launches": Kst,
         "summary": nv.activation_summary(acc0),
@@ -1023,7 +1027,7 @@ def run_gdnrec(args):
         e2e_one()
     b.record(stream)
     torch.cuda.synchronize()
-    ms_e2e = a.elapsed_time(b) / Kst
+    ms_e2e = dist_max(dist, a.elapsed_time(b) / Kst, device)  # max over ranks
     line = {
         "metric": METRIC, "value": bytes_step * world / (ms * 1e-3) / 1e9, "unit": "GB/s", "n_gpus": world,
         "steps": Kst, "warmup": Wm, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
@@ -1038,7 +1042,7 @@ def run_gdnrec(args):
         "kernels": {"tensor_macs_per_step": macs, "tensor_tflops": 2 * macs / (ms * 1e-3) / 1e12,
                     "tf32_peak_tflops": tf32_peak, "workspace_bytes": ws.numel()},
         "clocks": clk,
-        "e2e": {"value": bytes_step / (ms_e2e * 1e-3) / 1e9, "unit": "GB/s",
+        "e2e": {"value": bytes_step * world / (ms_e2e * 1e-3) / 1e9, "unit": "GB/s",
                 "h2d_bytes_per_step": sum(t.numel() * t.element_size() for t in h_in),
                 "d2h_bytes_per_step": sum(t.numel() * t.element_size() for t in h_res), "ms_per_step": ms_e2e},
         "gpu_launches": 2 * Kst,
