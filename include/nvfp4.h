@@ -28,11 +28,13 @@
  *     128 rows x 4 scales, scale (r, j) at byte
  *       ((r/128) * KA + j/4) * 512 + (r%32)*16 + ((r/32)%4)*4 + j%4,
  *     KA = ceil(K/64).  Padding bytes are zero (nvfp4_quantize writes them).
- *   - Every kernel is launched with programmatic stream serialization: it
- *     may start while the kernel before it on the stream is finishing, and
- *     waits for that kernel to complete before it reads or writes any
- *     argument buffer.  Only nvfp4_linear reads a buffer (the weights) before
- *     that point, and only while its own quantiser runs.
+ *   - Every kernel that reads or writes an argument buffer is launched with
+ *     programmatic stream serialization: it may start while the kernel
+ *     before it on the stream is finishing, and waits for that kernel to
+ *     complete before it touches any argument buffer.  Only nvfp4_linear
+ *     reads a buffer (the weights) before that point, and only while its own
+ *     quantiser runs.  (nvfp4_selftest_bounded_wait's kernel touches no
+ *     argument buffer and is launched plainly.)
  *   - Devices: compute capability 10.0 (B200) only.
  */
 #ifndef NVFP4_H
