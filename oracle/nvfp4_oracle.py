@@ -14,7 +14,7 @@ keep each module's own global scale.  "Main Findings", gate-parameterisation
 bullets: the write strength is a sigmoid of the b projection and the decay is
 log-space, softplus then exponential, of the a projection.
 
-Readings taken where the pages are silent (each one is listed in the design doc):
+Readings taken where the pages are silent:
   * global scale (dequantisation direction) g = amax(|x|) / (6 * 448), so the
     block holding the tensor maximum uses the full E4M3 range;
   * block scale byte = E4M3(RNE, saturating)((amax_block / 6) / g), FP32;
