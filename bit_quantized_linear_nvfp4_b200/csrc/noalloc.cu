@@ -9,6 +9,7 @@
 #include <cstdint>
 #include <mutex>
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include "internal.h"
@@ -24,18 +25,52 @@ static __device__ __align__(256) float g_scratch[kScratchBytes / sizeof(float)];
 constexpr int kMaxDevices = 64;
 std::mutex g_mutex;
 float* g_scratch_ptr[kMaxDevices] = {};
+unsigned long long g_scratch_ctx[kMaxDevices] = {};  // context the address belongs to
+
+// Unique id of the calling thread's current context (cuCtxGetId), 0 when the
+// driver does not provide it.  A context that is destroyed and created again
+// (cudaDeviceReset, a primary context released and retained) gets a new id,
+// and with it a new copy of g_scratch at a possibly different address.
+unsigned long long current_context_id() {
+  using GetCurrentFn = CUresult (*)(CUcontext*);
+  using GetIdFn = CUresult (*)(CUcontext, unsigned long long*);
+  static GetCurrentFn get_current = nullptr;
+  static GetIdFn get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<GetCurrentFn>(p);
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<GetIdFn>(p);
+  });
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (get_current == nullptr || get_id == nullptr || get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr ||
+      get_id(ctx, &id) != CUDA_SUCCESS)
+    return 0;
+  return id;
+}
 
 // Device address of g_scratch on the current device.  In host code the name
-// g_scratch is only a host-side stand-in, so the address is looked up once per
-// device (with that device current) and cached.
+// g_scratch is only a host-side stand-in, so the address is looked up with
+// cudaGetSymbolAddress while the device is current, once per device and
+// context, and cached; a call made in a new context of the device (after a
+// reset) looks it up again.
 cudaError_t scratch_address(int dev, float** out) {
   if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  const unsigned long long ctx = current_context_id();
   std::lock_guard<std::mutex> lock(g_mutex);
-  if (g_scratch_ptr[dev] == nullptr) {
+  if (g_scratch_ptr[dev] == nullptr || ctx != g_scratch_ctx[dev]) {
     void* p = nullptr;
     cudaError_t e = cudaGetSymbolAddress(&p, g_scratch);
     if (e != cudaSuccess) return e;
     g_scratch_ptr[dev] = static_cast<float*>(p);
+    // the lookup makes the device's context current if it was not yet
+    g_scratch_ctx[dev] = ctx != 0 ? ctx : current_context_id();
   }
   *out = g_scratch_ptr[dev];
   return cudaSuccess;

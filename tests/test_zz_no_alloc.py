@@ -6,9 +6,15 @@ memory, or code under a fixed memory plan.  Its amax scratch lives in a static
 array inside the library instead of a caller workspace.  This test calls it
 through the C ABI (ctypes, no Python wrapper) and checks that its codes, scale
 bytes and global scale equal those of nvfp4_quantize bit for bit (the
-tolerance the quantiser tests use), on two calls in a row.  The second input
-has a much smaller amax than the first, so a scratch word left over from the
-first call would show up as a wrong global scale.
+tolerance the quantiser tests use), on calls in a row.
+
+The first two inputs are larger than what the one-launch cluster path takes
+(about 1.6 MB of BF16), so both go through the two launches that pass the
+per-block maxima through the static scratch.  The first has a large amax
+(x40) and fills the scratch with large maxima; the second, FP32 with a much
+smaller amax (x0.01) and fewer rows (so fewer amax blocks), would show any
+scratch word left over from the first call as a wrong global scale.  Two
+small inputs (the cluster path, which needs no scratch) follow.
 """
 import ctypes
 
@@ -42,6 +48,8 @@ def test_noalloc_matches_quantize_on_consecutive_calls():
     lib = nv.library()
     rng = np.random.default_rng(77)
     inputs = [
+        torch.from_numpy((rng.standard_normal((4096, 1024)) * 40).astype(np.float32)).to(DEV).to(torch.bfloat16),
+        torch.from_numpy(rng.standard_normal((2048, 1024)).astype(np.float32) * 0.01).to(DEV),
         torch.from_numpy((rng.standard_normal((300, 512)) * 40).astype(np.float32)).to(DEV).to(torch.bfloat16),
         torch.from_numpy(rng.standard_normal((129, 272)).astype(np.float32) * 0.01).to(DEV),
     ]
