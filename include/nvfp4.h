@@ -167,8 +167,10 @@ int nvfp4_quantize_segments(const void* w, int w_dtype, int64_t N, int64_t K, in
  *   One call uses nvfp4_quantize_workspace_bytes(1) bytes of the scratch; a
  *   call needing more than NVFP4_NOALLOC_SCRATCH_BYTES is rejected with
  *   NVFP4_ERR_UNSUPPORTED_SHAPE.
- *   The first call on a device looks up the scratch address on that device;
- *   make that first call before any stream capture on the device.
+ *   The first call on a device looks up the scratch address on that device
+ *   (and so does the first call in a new context of the device, after a
+ *   cudaDeviceReset or after the primary context was released and created
+ *   again); make that first call before any stream capture on the device.
  *   Every call shares the one scratch array (each call writes the scratch it
  *   later reads, so it needs no clearing):
  *   calls whose work overlaps on the GPU, on different streams, race and must
