@@ -278,6 +278,137 @@ __global__ void __launch_bounds__(kThreads, 2) stats_kernel(const __grid_constan
   }
 }
 
+// Derived figures of the accumulators above, on the device (one block):
+//   out[0] max/RMS = max|x| / sqrt(sum x^2 / n)
+//   out[1] kurtosis = fourth central moment / variance^2, from the four raw
+//          moments: E x^4 - 4 mu E x^3 + 6 mu^2 E x^2 - 3 mu^4 over
+//          (E x^2 - mu^2)^2
+//   out[2] dominated share = dominated blocks / blocks
+//   out[3..5] per-token A4 error sqrt(row_err2) / sqrt(row_norm2) (a row with
+//          zero norm divides by 1): mean, min, max over the M rows (NaN when
+//          row_err2 is not given)
+//   out[6] hot-channel ratio = largest channel RMS / median channel RMS,
+//          channel RMS = sqrt(col_sq / M); the median of an even count is the
+//          mean of the two middle values
+//   out[7] the median channel RMS
+// All arithmetic is FP64, with every product and sum rounded on its own (no
+// fused multiply-add), in the order written above.  The two middle channel
+// values are found by radix selection on the FP32 bit patterns (col_sq is
+// non-negative, so its bit patterns order like its values).
+constexpr int kSumThreads = 1024;
+
+__device__ __forceinline__ double dmul(double a, double b) { return __dmul_rn(a, b); }
+__device__ __forceinline__ double dadd(double a, double b) { return __dadd_rn(a, b); }
+__device__ __forceinline__ double dsub(double a, double b) { return __dsub_rn(a, b); }
+
+__global__ void __launch_bounds__(kSumThreads, 1)
+    summary_kernel(const double* __restrict__ moments, const float* __restrict__ row_err2,
+                   const float* __restrict__ row_norm2, int64_t M, const float* __restrict__ col_sq, int64_t K,
+                   double* __restrict__ out) {
+  __shared__ double red_sum[kSumThreads / 32], red_min[kSumThreads / 32], red_max[kSumThreads / 32];
+  __shared__ uint32_t red_cmax[kSumThreads / 32];
+  __shared__ uint32_t hist[2][256];
+  __shared__ uint32_t sel_prefix[2], sel_rank[2];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  grid_dependency_wait();  // the accumulators come from the kernel before this one
+  if (tid == 0) grid_launch_dependents();
+
+  // per-token A4 error: sum, min, max over the rows (FP64)
+  double esum = 0.0, emin = INFINITY, emax = -INFINITY;
+  if (row_err2 != nullptr) {
+    for (int64_t r = tid; r < M; r += kSumThreads) {
+      const double nrm = __dsqrt_rn(static_cast<double>(row_norm2[r]));
+      const double e = __ddiv_rn(__dsqrt_rn(static_cast<double>(row_err2[r])), nrm > 0.0 ? nrm : 1.0);
+      esum = dadd(esum, e);
+      emin = fmin(emin, e);
+      emax = fmax(emax, e);
+    }
+  }
+  // largest column sum of squares (bit patterns order like the values)
+  uint32_t cmax = 0;
+  for (int64_t c = tid; c < K; c += kSumThreads) cmax = max(cmax, __float_as_uint(col_sq[c]));
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) {
+    esum = dadd(esum, __shfl_xor_sync(0xffffffffu, esum, off));
+    emin = fmin(emin, __shfl_xor_sync(0xffffffffu, emin, off));
+    emax = fmax(emax, __shfl_xor_sync(0xffffffffu, emax, off));
+    cmax = max(cmax, __shfl_xor_sync(0xffffffffu, cmax, off));
+  }
+  if (lane == 0) {
+    red_sum[warp] = esum;
+    red_min[warp] = emin;
+    red_max[warp] = emax;
+    red_cmax[warp] = cmax;
+  }
+  // radix selection of ranks (K-1)/2 and K/2 of col_sq, 8 bits per pass
+  if (tid < 2) {
+    sel_prefix[tid] = 0;
+    sel_rank[tid] = static_cast<uint32_t>(tid == 0 ? (K - 1) / 2 : K / 2);
+  }
+  for (int shift = 24; shift >= 0; shift -= 8) {
+    for (int i = tid; i < 512; i += kSumThreads) hist[i >> 8][i & 255] = 0;
+    __syncthreads();
+    const uint32_t hi_mask = shift == 24 ? 0u : (0xFFFFFFFFu << (shift + 8));
+    const uint32_t p0 = sel_prefix[0], p1 = sel_prefix[1];
+    for (int64_t c = tid; c < K; c += kSumThreads) {
+      const uint32_t key = __float_as_uint(col_sq[c]);
+      const uint32_t digit = (key >> shift) & 255u;
+      if ((key & hi_mask) == p0) atomicAdd(&hist[0][digit], 1u);
+      if ((key & hi_mask) == p1) atomicAdd(&hist[1][digit], 1u);
+    }
+    __syncthreads();
+    if (tid < 2) {
+      uint32_t k = sel_rank[tid], d = 0;
+      for (; d < 255; ++d) {
+        const uint32_t h = hist[tid][d];
+        if (k < h) break;
+        k -= h;
+      }
+      sel_rank[tid] = k;
+      sel_prefix[tid] |= d << shift;
+    }
+    __syncthreads();
+  }
+  if (warp == 0) {
+    const int nw = kSumThreads / 32;
+    double s = lane < nw ? red_sum[lane] : 0.0;
+    double lo = lane < nw ? red_min[lane] : INFINITY;
+    double hi = lane < nw ? red_max[lane] : -INFINITY;
+    uint32_t cm = lane < nw ? red_cmax[lane] : 0u;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+      s = dadd(s, __shfl_xor_sync(0xffffffffu, s, off));
+      lo = fmin(lo, __shfl_xor_sync(0xffffffffu, lo, off));
+      hi = fmax(hi, __shfl_xor_sync(0xffffffffu, hi, off));
+      cm = max(cm, __shfl_xor_sync(0xffffffffu, cm, off));
+    }
+    if (lane == 0) {
+      const double n = moments[5];
+      const double mean = __ddiv_rn(moments[0], n);
+      const double m2 = __ddiv_rn(moments[1], n);
+      const double mean2 = dmul(mean, mean);
+      const double var = dsub(m2, mean2);
+      double m4c = dsub(__ddiv_rn(moments[3], n), __ddiv_rn(dmul(dmul(4.0, mean), moments[2]), n));
+      m4c = dadd(m4c, dmul(dmul(6.0, mean2), m2));
+      m4c = dsub(m4c, dmul(3.0, dmul(mean2, mean2)));
+      out[0] = m2 > 0.0 ? __ddiv_rn(moments[4], __dsqrt_rn(m2)) : 0.0;
+      out[1] = var > 0.0 ? __ddiv_rn(m4c, dmul(var, var)) : 0.0;
+      out[2] = moments[6] != 0.0 ? __ddiv_rn(moments[7], moments[6]) : 0.0;
+      const bool have_err = row_err2 != nullptr && M > 0;
+      out[3] = have_err ? __ddiv_rn(s, static_cast<double>(M)) : __longlong_as_double(0x7FF8000000000000ll);
+      out[4] = have_err ? lo : __longlong_as_double(0x7FF8000000000000ll);
+      out[5] = have_err ? hi : __longlong_as_double(0x7FF8000000000000ll);
+      const double inv_rows = M > 0 ? __ddiv_rn(1.0, static_cast<double>(M)) : 1.0;
+      const double r_lo = __dsqrt_rn(dmul(static_cast<double>(__uint_as_float(sel_prefix[0])), inv_rows));
+      const double r_hi = __dsqrt_rn(dmul(static_cast<double>(__uint_as_float(sel_prefix[1])), inv_rows));
+      const double med = K > 0 ? __ddiv_rn(dadd(r_lo, r_hi), 2.0) : 0.0;
+      const double rmax = __dsqrt_rn(dmul(static_cast<double>(__uint_as_float(cm)), inv_rows));
+      out[6] = med > 0.0 ? __ddiv_rn(rmax, med) : 0.0;
+      out[7] = med;
+    }
+  }
+}
+
 int sm_count() {
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
@@ -326,6 +457,21 @@ cudaError_t launch_act_stats(const void* x, int dtype, int64_t M, int64_t K, int
                 : cudaLaunchKernelEx(&cfg, stats_kernel<NVFP4_DTYPE_BF16, false>, a);
   return wide ? cudaLaunchKernelEx(&cfg, stats_kernel<NVFP4_DTYPE_F32, true>, a)
               : cudaLaunchKernelEx(&cfg, stats_kernel<NVFP4_DTYPE_F32, false>, a);
+}
+
+cudaError_t launch_act_summary(const double* moments, const float* row_err2, const float* row_norm2, int64_t M,
+                               const float* col_sq, int64_t K, double* out, cudaStream_t stream) {
+  using namespace st;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(1);
+  cfg.blockDim = dim3(kSumThreads);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, summary_kernel, moments, row_err2, row_norm2, M, col_sq, K, out);
 }
 
 }  // namespace nvfp4

@@ -363,6 +363,25 @@ int nvfp4_activation_stats(const void* x, int x_dtype, int64_t M, int64_t K, int
   return NVFP4_OK;
 }
 
+int nvfp4_activation_summary(const double* moments, const float* row_err2, const float* row_norm2, int64_t M,
+                             const float* col_sq, int64_t K, double* summary, void* stream) {
+  if (moments == nullptr || row_norm2 == nullptr || col_sq == nullptr || summary == nullptr)
+    return NVFP4_ERR_INVALID_ARG;
+  if (M <= 0 || K <= 0) return NVFP4_ERR_INVALID_ARG;
+  if (M > (int64_t(1) << 31) - 1 || K > (int64_t(1) << 30)) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+  if ((reinterpret_cast<uintptr_t>(moments) & 7u) != 0 || (reinterpret_cast<uintptr_t>(summary) & 7u) != 0)
+    return NVFP4_ERR_MISALIGNED;
+  const void* f32s[3] = {row_err2, row_norm2, col_sq};
+  for (const void* q : f32s)
+    if ((reinterpret_cast<uintptr_t>(q) & 3u) != 0) return NVFP4_ERR_MISALIGNED;
+  int st = check_device();
+  if (st != NVFP4_OK) return st;
+  cudaError_t e = nvfp4::launch_act_summary(moments, row_err2, row_norm2, M, col_sq, K, summary,
+                                            static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e);
+  return NVFP4_OK;
+}
+
 int nvfp4_gemm(const nvfp4_operand* A, const float* g_a, const nvfp4_operand* W, const float* g_w,
                void* out, int out_dtype, int64_t ld_out, void* workspace, size_t workspace_bytes,
                void* stream) {

@@ -72,6 +72,10 @@ cudaError_t launch_act_stats(const void* x, int dtype, int64_t M, int64_t K, int
                              double* moments, float* row_err2, float* row_norm2, float* col_sq, float* col_max,
                              cudaStream_t stream);
 
+// Derived figures of the statistics' accumulators (see nvfp4_activation_summary).
+cudaError_t launch_act_summary(const double* moments, const float* row_err2, const float* row_norm2, int64_t M,
+                               const float* col_sq, int64_t K, double* out, cudaStream_t stream);
+
 // Gated delta-rule recurrence (see nvfp4_gdn_recurrence); leading dimensions
 // in elements, d_k = 64 and d_v = 128.
 struct GdnProblem {

@@ -45,6 +45,7 @@ EXPORTED = (
     "nvfp4_gemm_workspace_bytes", "nvfp4_gemm", "nvfp4_fused_proj", "nvfp4_check",
     "nvfp4_quantize_noalloc", "nvfp4_linear", "nvfp4_requantize_segments",
     "nvfp4_kv_fp8_quantize", "nvfp4_kv_fp8_dequantize", "nvfp4_activation_stats",
+    "nvfp4_activation_summary",
     "nvfp4_gdn_workspace_bytes", "nvfp4_gdn_recurrence", "nvfp4_selftest_bounded_wait",
 )
 
@@ -125,6 +126,9 @@ def _lib():
         lib.nvfp4_activation_stats.argtypes = [c.c_void_p, c.c_int, c.c_int64, c.c_int64, c.c_int64, c.c_void_p,
                                                c.c_void_p, c.c_void_p, c.c_void_p, c.c_void_p, c.c_void_p,
                                                c.c_void_p]
+        lib.nvfp4_activation_summary.restype = c.c_int
+        lib.nvfp4_activation_summary.argtypes = [c.c_void_p, c.c_void_p, c.c_void_p, c.c_int64, c.c_void_p,
+                                                 c.c_int64, c.c_void_p, c.c_void_p]
         lib.nvfp4_gdn_workspace_bytes.restype = c.c_size_t
         lib.nvfp4_gdn_workspace_bytes.argtypes = [c.c_int64, c.c_int64]
         lib.nvfp4_gdn_recurrence.restype = c.c_int
@@ -416,25 +420,30 @@ def nvfp4_activation_stats(x: torch.Tensor, g: Optional[torch.Tensor] = None, *,
     return into
 
 
-def activation_summary(stats: dict) -> dict:
-    """Host-side figures from nvfp4_activation_stats' accumulators: max/RMS,
-    kurtosis (fourth central moment / variance^2), dominated-block share,
-    per-token A4 error (mean, min, max) and hot-channel ratio (largest channel
-    RMS over the median channel RMS)."""
-    m = stats["moments"].double().cpu().tolist()
-    n = m[5]
-    mean, m2 = m[0] / n, m[1] / n
-    var = m2 - mean * mean
-    m4c = m[3] / n - 4 * mean * m[2] / n + 6 * mean * mean * m2 - 3 * mean ** 4
-    out = {"max_over_rms": m[4] / m2 ** 0.5 if m2 > 0 else 0.0, "kurtosis": m4c / var ** 2 if var > 0 else 0.0,
-           "dominated_share": m[7] / m[6] if m[6] else 0.0}
-    rows = stats["row_norm2"].double()
-    if stats.get("row_err2") is not None:
-        err = (stats["row_err2"].double() / torch.where(rows > 0, rows, torch.ones_like(rows))).sqrt()
-        out.update(a4_err_mean=err.mean().item(), a4_err_min=err.min().item(), a4_err_max=err.max().item())
-    col_rms = (stats["col_sq"].double() / rows.numel()).sqrt()
-    med = torch.quantile(col_rms, 0.5).item()  # the mean of the two middle values for an even count
-    out["hot_channel_ratio"] = col_rms.max().item() / med if med > 0 else 0.0
+SUMMARY_FIELDS = ("max_over_rms", "kurtosis", "dominated_share", "a4_err_mean", "a4_err_min", "a4_err_max",
+                  "hot_channel_ratio", "channel_rms_median")
+
+
+def nvfp4_activation_summary(stats: dict, *, out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """Device float64[8] of derived figures from nvfp4_activation_stats'
+    accumulators (nvfp4_activation_summary; the order is SUMMARY_FIELDS)."""
+    dev = stats["moments"].device
+    out = torch.empty(8, dtype=torch.float64, device=dev) if out is None else out
+    M = stats["row_norm2"].numel()
+    K = stats["col_sq"].numel()
+    _call("nvfp4_activation_summary", _ptr(stats["moments"]), _ptr(stats.get("row_err2")), _ptr(stats["row_norm2"]),
+          M, _ptr(stats["col_sq"]), K, _ptr(out), _stream(stream))
+    return out
+
+
+def activation_summary(stats: dict, stream=None) -> dict:
+    """The derived figures as a dict (computed by the library on the device;
+    the A4 error fields are absent when the statistics had no global scale)."""
+    vals = nvfp4_activation_summary(stats, stream=stream).cpu().tolist()
+    out = dict(zip(SUMMARY_FIELDS, vals))
+    if stats.get("row_err2") is None:
+        for k in ("a4_err_mean", "a4_err_min", "a4_err_max"):
+            del out[k]
     return out
 
 

@@ -305,13 +305,40 @@ int nvfp4_kv_fp8_dequantize(const uint8_t* codes, int64_t rows, int64_t cols, in
  *            with x_hat the NVFP4 dequantisation under g (the quantiser's
  *            arithmetic), and sum x^2.
  *   col_sq, col_max  device float[K] or NULL: per column, sum x^2 and max |x|.
- * Derived figures: max/RMS = moments[4] / sqrt(moments[1] / moments[5]);
- * kurtosis from the four moments; per-token A4 error sqrt(row_err2/row_norm2);
- * hot-channel ratio from sqrt(col_sq / M) against its median.
+ * The derived figures (max/RMS, kurtosis, dominated share, per-token A4
+ * error, hot-channel ratio) come from nvfp4_activation_summary.
  */
 int nvfp4_activation_stats(const void* x, int x_dtype, int64_t M, int64_t K, int64_t ld_x, const float* g,
                            double* moments, float* row_err2, float* row_norm2, float* col_sq, float* col_max,
                            void* stream);
+
+/*
+ * nvfp4_activation_summary — the figures the pages report for the residual
+ * stream ("Main Findings", activation bullet: max/RMS, kurtosis, the share of
+ * 16-element blocks dominated by one value, the per-token A4 error, hot
+ * channels against the median channel), derived on the device from
+ * nvfp4_activation_stats' accumulators in one small launch.  FP64 throughout,
+ * each product and sum rounded on its own (no fused multiply-add):
+ *   summary[0] max/RMS        moments[4] / sqrt(moments[1] / n), n = moments[5]
+ *   summary[1] kurtosis       (E x^4 - 4 mu E x^3 + 6 mu^2 E x^2 - 3 mu^4) / var^2,
+ *                             mu = E x, var = E x^2 - mu^2 (0 when var <= 0)
+ *   summary[2] dominated share   moments[7] / moments[6]
+ *   summary[3..5] per-token A4 error e_r = sqrt(row_err2[r]) / sqrt(row_norm2[r])
+ *                             (divided by 1 when row_norm2[r] == 0): mean, min,
+ *                             max over the M rows; NaN when row_err2 is NULL
+ *   summary[6] hot-channel ratio  max_c rms_c / median_c rms_c,
+ *                             rms_c = sqrt(col_sq[c] / M); the median of an even
+ *                             count is the mean of the two middle values
+ *   summary[7] median channel RMS (0 gives summary[6] = 0)
+ *   moments    device double[8] as nvfp4_activation_stats writes them.
+ *   row_err2, row_norm2  device float[M] (row_err2 may be NULL).
+ *   col_sq     device float[K], non-negative.
+ *   summary    device double[8], written.
+ * M >= 1 and K >= 1.  Enqueued on `stream` after the statistics; the caller
+ * reads the 64 bytes back when it needs them.
+ */
+int nvfp4_activation_summary(const double* moments, const float* row_err2, const float* row_norm2, int64_t M,
+                             const float* col_sq, int64_t K, double* summary, void* stream);
 
 /*
  * nvfp4_gdn_recurrence — the gated delta-rule recurrence that consumes the

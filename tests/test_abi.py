@@ -213,6 +213,19 @@ def test_activation_stats_rejects_bad_arguments(lib):
     assert call(M=0) == 0
 
 
+def test_activation_summary_rejects_bad_arguments(lib):
+    v = ctypes.c_void_p
+
+    def call(mom=FAKE, re=FAKE, rn=FAKE, M=4, cs=FAKE, K=64, out=FAKE):
+        p = lambda a: v(a) if a else None
+        return lib.nvfp4_activation_summary(p(mom), p(re), p(rn), M, p(cs), K, p(out), None)
+    assert call(mom=0) == 1 and call(rn=0) == 1 and call(cs=0) == 1 and call(out=0) == 1
+    assert call(M=0) == 1 and call(K=0) == 1 and call(M=-3) == 1
+    assert call(M=1 << 31) == 2 and call(K=(1 << 30) + 1) == 2
+    assert call(mom=FAKE + 4) == 3 and call(out=FAKE + 4) == 3
+    assert call(re=FAKE + 2) == 3 and call(rn=FAKE + 1) == 3 and call(cs=FAKE + 2) == 3
+
+
 def test_gdn_recurrence_rejects_bad_arguments(lib):
     v = ctypes.c_void_p
     T, H, Hk = 100, 4, 2

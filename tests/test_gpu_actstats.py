@@ -60,6 +60,52 @@ def test_stats_match_oracle(dtype, M, K):
         assert abs(s_gpu[k] - s_ref[k]) <= 1e-4 * max(1.0, abs(s_ref[k])), k
 
 
+def _host_stats(st):
+    """The device accumulators as the oracle's statistics dict, every value
+    converted exactly to FP64."""
+    m = st["moments"].cpu().numpy()
+    return {"sum": m[0], "sum_sq": m[1], "sum_cube": m[2], "sum_4th": m[3], "amax": m[4], "n": m[5],
+            "blocks": m[6], "dominated": m[7],
+            "row_err2": st["row_err2"].double().cpu().numpy(), "row_norm2": st["row_norm2"].double().cpu().numpy(),
+            "col_sq": st["col_sq"].double().cpu().numpy()}
+
+
+@pytest.mark.parametrize("M,K", [(1, 16), (7, 48), (300, 1040), (257, 5120), (2048, 5120), (64, 17408)])
+def test_device_summary_matches_oracle_summary(M, K):
+    """nvfp4_activation_summary against oracle.activation_summary on the same
+    accumulators: every figure is the same FP64 expression, so they agree to
+    a few ulp (the A4 mean sums M terms in a different order: M ulp)."""
+    x = _x(M, K, 3 * M + K, "bf16")
+    xd = _dev(x, "bf16")
+    A, g = nv.nvfp4_quantize(xd)
+    st = nv.nvfp4_activation_stats(xd, g)
+    dev = nv.nvfp4_activation_summary(st).cpu().numpy()
+    ref = o.activation_summary(_host_stats(st))
+    for i, k in enumerate(nv.SUMMARY_FIELDS[:7]):
+        tol = (4 * M if k == "a4_err_mean" else 8) * np.finfo(np.float64).eps * max(abs(ref[k]), 1e-300)
+        assert abs(dev[i] - ref[k]) <= tol, (k, dev[i], ref[k])
+    col_rms = np.sqrt(_host_stats(st)["col_sq"] * (1.0 / M))
+    assert abs(dev[7] - np.median(col_rms)) <= 8 * np.finfo(np.float64).eps * np.median(col_rms)
+
+
+def test_device_summary_even_and_odd_channel_counts():
+    """The median is the middle channel for an odd count and the mean of the
+    two middle ones for an even count; ties and zero channels included."""
+    for K in (15, 16, 33, 48):
+        rng = np.random.default_rng(K)
+        col = rng.integers(0, 5, size=K).astype(np.float32) * 0.5
+        st = {"moments": torch.tensor([0, 4, 0, 16, 2, 4, 1, 0], dtype=torch.float64, device=DEV),
+              "row_err2": None, "row_norm2": torch.ones(4, device=DEV),
+              "col_sq": torch.from_numpy(col).to(DEV)}
+        out = nv.nvfp4_activation_summary(st).cpu().numpy()
+        rms = np.sqrt(col.astype(np.float64) * 0.25)
+        med = np.median(rms)
+        assert out[7] == med, (K, out[7], med)
+        assert out[6] == (rms.max() / med if med > 0 else 0.0)
+        assert np.isnan(out[3]) and np.isnan(out[4]) and np.isnan(out[5])
+        assert out[2] == 0.0 and out[0] == 2.0 / 1.0  # amax 2 over sqrt(4 / 4)
+
+
 def test_accumulates_over_batches_and_strided_rows():
     x = _x(400, 2048, 3)
     big = torch.zeros((400, 2304), dtype=torch.bfloat16, device=DEV)
