@@ -58,7 +58,16 @@ struct KernelArgs {
   const float* g_a;
   const float* seg_scale;
   int nseg;
+  uint32_t tma_mask;  // bit s: segment s has an output tensor map (staged stores)
   EpiSegment seg[kMaxSeg];
+};
+
+// Output tensor maps of the segments for the staged epilogue (BF16): box 64
+// columns x 16 rows (whole 128-byte lines, 128-byte swizzle) for the fused
+// projections, 32 x 32 (64-byte rows, 64-byte swizzle) for SwiGLU, whose
+// warps hold 32 output columns.
+struct OutMaps {
+  CUtensorMap m[kMaxSeg];
 };
 
 struct SharedTail {
@@ -415,22 +424,30 @@ __global__ void __launch_bounds__(kThreads, 1)
 // issues tcgen05.mma.cta_group::2 with M = 256, and each CTA's TMEM holds its
 // own 128 x 256 accumulator.
 //
-// The operand feed is bound by the number of TMA copies in flight per SM more
-// than by bytes, so copies are kept few and large: the codes of a K-stage are
-// two 16 KB boxes, and the scale atoms of four K-stages arrive together in a
-// separate two-slot ring (one 8 KB box for A, one 16 KB box for the 256 B
-// rows; every CTA keeps the scales of all 256 B rows, as the pair MMA reads
-// them from each CTA's own TMEM).
+// Each of the 5 stages holds one K-stage (256 K) of everything the MMAs read:
+// the codes (two 16 KB boxes) and the scale atoms of this CTA's 128 A rows
+// (2 KB) and of all 256 B rows (4 KB; the pair MMA reads each CTA's scales
+// for the whole B tile from its own TMEM).  The epilogue stages BF16 output
+// chunks in shared memory and writes them with TMA stores.
 constexpr int kStages2 = 5;
-constexpr int kBHalfBytes = kBBytes / 2;                  // 16 KB
-constexpr int kCodeStage2 = kABytes + kBHalfBytes;       // 32 KB
-constexpr int kSFGroup = 4;                              // K-stages per scale group
-constexpr int kSFSlots = 2;
-constexpr int kSFASlotBytes = kSFGroup * kSFABytes;      // 8 KB
-constexpr int kSFBSlotBytes = kSFGroup * kSFBBytes;      // 16 KB
-constexpr int kSFSlotBytes = kSFASlotBytes + kSFBSlotBytes;
-constexpr int kSmemBytes2 = kStages2 * kCodeStage2 + kSFSlots * kSFSlotBytes + 1024 + 256;
-static_assert(kCodeStage2 % 1024 == 0 && kSFSlotBytes % 1024 == 0, "buffers keep 1024-byte alignment");
+constexpr int kBHalfBytes = kBBytes / 2;                                  // 16 KB
+constexpr int kStageBytes2 = kABytes + kBHalfBytes + kSFABytes + kSFBBytes;  // 38 KB
+constexpr int kStageSFA2 = kABytes + kBHalfBytes;                         // offsets in a stage
+constexpr int kStageSFB2 = kStageSFA2 + kSFABytes;
+static_assert(kStageBytes2 % 1024 == 0, "stage buffers keep 1024-byte alignment");
+
+// The pair kernel's epilogue has 16 warps: warp w (2..17) reads TMEM lane
+// quadrant w % 4 and column group (w - 2) / 4, 64 of the tile's 256 columns.
+// Twice the 8 warps of the other kernels, so that one tile's epilogue (TMEM
+// reads, scaling, nonlinearity, stores) keeps pace with the next tile's
+// mainloop and does not hold back its MMAs.
+constexpr int kNumEpiWarps2 = 16;
+constexpr int kThreads2 = 64 + kNumEpiWarps2 * 32;
+// one 32 x 32 BF16 output chunk (2 KB) of staging per epilogue warp
+constexpr int kEpiChunkBytes = 2048;
+constexpr int kEpiBytes2 = kNumEpiWarps2 * kEpiChunkBytes;
+constexpr int kSmemBytes2 = kStages2 * kStageBytes2 + kEpiBytes2 + 1024 + 256;
+static_assert(kSmemBytes2 <= 227 * 1024, "shared memory of one CTA");
 
 // Two accumulators that share 64 TMEM columns: buffer 0 is columns
 // [0, 256), buffer 1 is [192, 448), scales follow at 448.  The epilogue reads
@@ -442,8 +459,6 @@ __device__ __forceinline__ uint32_t col_acc2(int buf) { return buf ? 192u : 0u; 
 struct SharedTail2 {
   uint64_t full[kStages2];
   uint64_t empty[kStages2];
-  uint64_t sf_full[kSFSlots];
-  uint64_t sf_empty[kSFSlots];
   uint64_t tmem_full[2];
   uint64_t tmem_empty[2];
   uint64_t ovl_free[2];
@@ -452,15 +467,120 @@ struct SharedTail2 {
   int abort_flag;
 };
 
-__global__ void __launch_bounds__(kThreads, 1)
+// Staged store of one 32 x 32 BF16 chunk (lane l: row row0 + l, columns
+// j0 .. j0+31 of segment s): the warp writes it to its 2 KB buffer in the
+// map's 64-byte-swizzle layout (16-byte piece c of row r at c ^ ((r / 2) % 4),
+// so the shared stores are free of bank conflicts) and one lane issues the
+// TMA store; rows past M are not written.  The buffer is reused only after
+// the previous store from it has been read.
+__device__ __forceinline__ void stage_and_store_bf16(const CUtensorMap* m, uint8_t* buf, const uint32_t (&w)[16],
+                                                     int32_t j0, int32_t row0) {
+  const int lane = threadIdx.x & 31;
+  if (lane == 0) bulk_wait_group_read<0>();
+  __syncwarp();
+  uint8_t* rowp = buf + lane * 64;
+  const int sw = (lane >> 1) & 3;
+#pragma unroll
+  for (int c = 0; c < 4; ++c)
+    *reinterpret_cast<uint4*>(rowp + ((c ^ sw) << 4)) = make_uint4(w[4 * c], w[4 * c + 1], w[4 * c + 2], w[4 * c + 3]);
+  fence_proxy_async_smem();
+  __syncwarp();
+  if (lane == 0) {
+    tma_store_2d(m, buf, j0, row0);
+    bulk_commit_group();
+  }
+}
+
+// Columns n0 .. n0+63 of rows row0 .. row0+31 (chunks r0 and r1).  When
+// both lie in one BF16 segment with a map, on its 16-byte grid, they leave
+// through the staging buffer as two 16-row x 64-column boxes: rows of 128
+// bytes, so every global write is a whole line.  Lanes 16h .. 16h+15 place
+// their rows for box h (16-byte piece c of box row r at c ^ (r % 8), the
+// map's 128-byte swizzle, free of bank conflicts).  Otherwise (FP32
+// epilogues, a segment boundary inside the 64 columns) each chunk is stored
+// per lane.
+__device__ __forceinline__ void store_pair_staged(const KernelArgs& a, const OutMaps& maps, uint8_t* buf,
+                                                  int64_t row0, int64_t n0, const uint32_t (&r0)[32],
+                                                  const uint32_t (&r1)[32]) {
+  if (n0 >= a.N || row0 >= a.M) return;
+  const int lane = threadIdx.x & 31;
+  const int s = seg_of(a, n0);
+  const EpiSegment& sg = a.seg[s];
+  const int64_t j0 = n0 - sg.n_begin;
+  if (((a.tma_mask >> s) & 1u) == 0 || n0 + 63 >= sg.n_end || (j0 & 7) != 0) {
+    if (row0 + lane < a.M) {
+      store_chunk(a, row0 + lane, n0, r0);
+      store_chunk(a, row0 + lane, n0 + 32, r1);
+    }
+    return;
+  }
+  const float scale = __ldg(a.g_a) * __ldg(a.seg_scale + s);
+  uint32_t w[32];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    w[i] = pack_bf16(__uint_as_float(r0[2 * i]) * scale, __uint_as_float(r0[2 * i + 1]) * scale);
+    w[16 + i] = pack_bf16(__uint_as_float(r1[2 * i]) * scale, __uint_as_float(r1[2 * i + 1]) * scale);
+  }
+  const int rr = lane & 15;
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    if (row0 + 16 * h >= a.M) break;  // uniform
+    if (lane == 0) bulk_wait_group_read<0>();
+    __syncwarp();
+    if ((lane >> 4) == h) {
+      uint8_t* rowp = buf + rr * 128;
+#pragma unroll
+      for (int c = 0; c < 8; ++c)
+        *reinterpret_cast<uint4*>(rowp + ((c ^ (rr & 7)) << 4)) =
+            make_uint4(w[4 * c], w[4 * c + 1], w[4 * c + 2], w[4 * c + 3]);
+    }
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) {
+      tma_store_2d(&maps.m[s], buf, static_cast<int32_t>(j0), static_cast<int32_t>(row0 + 16 * h));
+      bulk_commit_group();
+    }
+  }
+}
+
+// SwiGLU chunk: output columns o0 .. o0+31 of rows row0 .. row0+31.
+__device__ __forceinline__ void store_swiglu_staged(const KernelArgs& a, const OutMaps& maps, uint8_t* buf,
+                                                    int64_t row0, int64_t o0, const uint32_t (&rg)[32],
+                                                    const uint32_t (&ru)[32]) {
+  if (o0 >= a.n_out || row0 >= a.M) return;
+  const int lane = threadIdx.x & 31;
+  if ((a.tma_mask & 1u) == 0 || o0 + 31 >= a.n_out) {
+    if (row0 + lane < a.M) store_swiglu(a, row0 + lane, o0, rg, ru);
+    return;
+  }
+  const float ga = __ldg(a.g_a);
+  const float sgate = ga * __ldg(a.seg_scale + 0);
+  const float sup = ga * __ldg(a.seg_scale + 1);
+  uint32_t w[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    float v[2];
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      const float gv = __uint_as_float(rg[2 * i + k]) * sgate;
+      const float uv = __uint_as_float(ru[2 * i + k]) * sup;
+      v[k] = gv * __frcp_rn(1.0f + __expf(-gv)) * uv;
+    }
+    w[i] = pack_bf16(v[0], v[1]);
+  }
+  stage_and_store_bf16(&maps.m[0], buf, w, static_cast<int32_t>(o0), static_cast<int32_t>(row0));
+}
+
+template <bool SWIGLU>
+__global__ void __launch_bounds__(kThreads2, 1)
     gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
-                     const __grid_constant__ CUtensorMap tm_sfa, const __grid_constant__ CUtensorMap tm_sfb1,
-                     const __grid_constant__ CUtensorMap tm_sfb2, const __grid_constant__ KernelArgs args) {
+                     const __grid_constant__ CUtensorMap tm_sfa, const __grid_constant__ CUtensorMap tm_sfb,
+                     const __grid_constant__ KernelArgs args, const __grid_constant__ OutMaps out_maps) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
-  uint8_t* sf_smem = smem + kStages2 * kCodeStage2;
-  SharedTail2* tail = reinterpret_cast<SharedTail2*>(sf_smem + kSFSlots * kSFSlotBytes);
+  uint8_t* epi_smem = smem + kStages2 * kStageBytes2;
+  SharedTail2* tail = reinterpret_cast<SharedTail2*>(epi_smem + kEpiBytes2);
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const uint32_t rank = cluster_rank() & 1u;  // position in the pair
@@ -476,14 +596,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&tail->full[s], 1);
       mbar_init(&tail->empty[s], 1);
     }
-    for (int s = 0; s < kSFSlots; ++s) {
-      mbar_init(&tail->sf_full[s], 1);
-      mbar_init(&tail->sf_empty[s], 1);
-    }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&tail->tmem_full[b], 1);
-      mbar_init(&tail->tmem_empty[b], 2 * kNumEpiWarps);
-      mbar_init(&tail->ovl_free[b], kNumEpiWarps);  // the 4 warps per CTA holding the shared columns
+      mbar_init(&tail->tmem_empty[b], 2 * kNumEpiWarps2);
+      // the warps of both CTAs that hold the shared columns: 4 per CTA (one
+      // column group), 8 for SwiGLU (gate and up halves of two groups)
+      mbar_init(&tail->ovl_free[b], SWIGLU ? 16 : 8);
     }
     mbar_init(&tail->drain, 1);
     tail->abort_flag = 0;
@@ -491,8 +609,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     prefetch_tmap(&tm_a);
     prefetch_tmap(&tm_b);
     prefetch_tmap(&tm_sfa);
-    prefetch_tmap(&tm_sfb1);
-    prefetch_tmap(&tm_sfb2);
+    prefetch_tmap(&tm_sfb);
+    for (int i = 0; i < args.nseg; ++i)
+      if ((args.tma_mask >> i) & 1u) prefetch_tmap(&out_maps.m[i]);
   }
   if (warp == 1) {
     tmem_alloc_pair(&tail->tmem_base, kTmemCols);
@@ -511,46 +630,34 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0) {
     // ------------------------------------------------------------ producer (both CTAs)
     if (elect_one()) {
-      int stage = 0, sslot = 0;
-      uint32_t phase = 0, sphase = 0;
-      bool issued[kStages2], sissued[kSFSlots];
-      uint32_t issued_phase[kStages2], sissued_phase[kSFSlots];
+      int stage = 0;
+      uint32_t phase = 0;
+      bool issued[kStages2];
+      uint32_t issued_phase[kStages2];
       for (int s = 0; s < kStages2; ++s) issued[s] = false;
-      for (int s = 0; s < kSFSlots; ++s) sissued[s] = false;
       bool ok = true;
       for (int t = pair; t < num_tiles && ok; t += num_pairs) {
         int m_blk, n_blk;
         tile_coords(args, t, m_blk, n_blk);
         const int32_t a_row = m_blk * 256 + static_cast<int32_t>(rank) * 128;
-        const int64_t b_row0 = args.swiglu ? static_cast<int64_t>(n_blk) * 128 : static_cast<int64_t>(n_blk) * BN;
-        const int64_t b_row1 = args.swiglu ? args.up_row0 + static_cast<int64_t>(n_blk) * 128 : b_row0 + 128;
+        const int64_t b_row0 = SWIGLU ? static_cast<int64_t>(n_blk) * 128 : static_cast<int64_t>(n_blk) * BN;
+        const int64_t b_row1 = SWIGLU ? args.up_row0 + static_cast<int64_t>(n_blk) * 128 : b_row0 + 128;
         const int64_t b_mine = rank ? b_row1 : b_row0;
         for (int ks = 0; ks < KS; ++ks) {
-          if (ks % kSFGroup == 0) {
-            // scale atoms of K-stages ks .. ks+3 for this CTA's A rows and all 256 B rows
-            if (!mbar_wait_bounded(&tail->sf_empty[sslot], sphase ^ 1u, abort_flag)) { ok = false; break; }
-            const uint32_t sbar = map_to_rank(smem_u32(&tail->sf_full[sslot]), 0);
-            if (leader) mbar_arrive_expect_tx(&tail->sf_full[sslot], 2 * kSFSlotBytes);
-            uint8_t* slot = sf_smem + sslot * kSFSlotBytes;
-            tma_load_3d_pair(slot, &tm_sfa, sbar, 0, ks * 4, a_row / 128);
-            if (args.swiglu) {
-              tma_load_3d_pair(slot + kSFASlotBytes, &tm_sfb1, sbar, 0, ks * 4, static_cast<int32_t>(b_row0 / 128));
-              tma_load_3d_pair(slot + kSFASlotBytes + kSFBSlotBytes / 2, &tm_sfb1, sbar, 0, ks * 4,
-                               static_cast<int32_t>(b_row1 / 128));
-            } else {
-              tma_load_3d_pair(slot + kSFASlotBytes, &tm_sfb2, sbar, 0, ks * 4, static_cast<int32_t>(b_row0 / 128));
-            }
-            sissued[sslot] = true;
-            sissued_phase[sslot] = sphase;
-            if (++sslot == kSFSlots) { sslot = 0; sphase ^= 1u; }
-          }
           if (!mbar_wait_bounded(&tail->empty[stage], phase ^ 1u, abort_flag)) { ok = false; break; }
-          uint8_t* st = smem + stage * kCodeStage2;
+          uint8_t* st = smem + stage * kStageBytes2;
           const uint32_t bar = map_to_rank(smem_u32(&tail->full[stage]), 0);  // even CTA of the pair
-          if (leader) mbar_arrive_expect_tx(&tail->full[stage], 2 * kCodeStage2);
+          if (leader) mbar_arrive_expect_tx(&tail->full[stage], 2 * kStageBytes2);
           const int32_t kx = ks * (BK / 2);
           tma_load_2d_pair(st, &tm_a, bar, kx, a_row);
           tma_load_2d_pair(st + kABytes, &tm_b, bar, kx, static_cast<int32_t>(b_mine));
+          tma_load_3d_pair(st + kStageSFA2, &tm_sfa, bar, 0, ks * 4, a_row / 128);
+          if (SWIGLU) {
+            tma_load_3d_pair(st + kStageSFB2, &tm_sfb, bar, 0, ks * 4, static_cast<int32_t>(b_row0 / 128));
+            tma_load_3d_pair(st + kStageSFB2 + kSFBBytes / 2, &tm_sfb, bar, 0, ks * 4, static_cast<int32_t>(b_row1 / 128));
+          } else {
+            tma_load_3d_pair(st + kStageSFB2, &tm_sfb, bar, 0, ks * 4, static_cast<int32_t>(b_row0 / 128));
+          }
           issued[stage] = true;
           issued_phase[stage] = phase;
           if (++stage == kStages2) { stage = 0; phase ^= 1u; }
@@ -559,8 +666,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (*abort_flag && leader) {
         for (int s = 0; s < kStages2; ++s)
           if (issued[s]) mbar_wait_bounded(&tail->full[s], issued_phase[s], nullptr, 200000000ull);
-        for (int s = 0; s < kSFSlots; ++s)
-          if (sissued[s]) mbar_wait_bounded(&tail->sf_full[s], sissued_phase[s], nullptr, 200000000ull);
       }
     }
   } else if (warp == 1) {
@@ -570,9 +675,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t idesc = (1u << 7) | (1u << 10) | (static_cast<uint32_t>(BN >> 3) << 17) |
                              (static_cast<uint32_t>(256 >> 4) << 24);
       const uint32_t base = smem_u32(smem);
-      const uint32_t sbase = smem_u32(sf_smem);
-      int stage = 0, sslot = 0;
-      uint32_t phase = 0, sphase = 0;
+      int stage = 0;
+      uint32_t phase = 0;
       int local = 0;
       bool ok = true;
       bool any_issued = false;
@@ -585,22 +689,18 @@ __global__ void __launch_bounds__(kThreads, 1)
             !mbar_wait_bounded(&tail->tmem_empty[buf], ((local - 2) >> 1) & 1, abort_flag)) { ok = false; break; }
         tc_fence_after();
         for (int ks = 0; ks < KS; ++ks) {
-          const int j = ks % kSFGroup;
-          if (j == 0) {
-            if (!mbar_wait_bounded(&tail->sf_full[sslot], sphase, abort_flag)) { ok = false; break; }
-          }
           if (!mbar_wait_bounded(&tail->full[stage], phase, abort_flag)) { ok = false; break; }
           tc_fence_after();
-          const uint32_t sa = base + stage * kCodeStage2;
+          const uint32_t sa = base + stage * kStageBytes2;
           const uint32_t sb = sa + kABytes;
-          const uint32_t ssfa = sbase + sslot * kSFSlotBytes + j * kSFABytes;
-          const uint32_t ssfb0 = sbase + sslot * kSFSlotBytes + kSFASlotBytes + j * kSFABytes;
-          const uint32_t ssfb1 = ssfb0 + kSFBSlotBytes / 2;
+          const uint32_t ssfa = sa + kStageSFA2;
+          const uint32_t ssfb = sa + kStageSFB2;
 #pragma unroll
           for (int kb = 0; kb < 4; ++kb) {
             tmem_cp_32x128b_warpx4_pair(tmem + kColSFA2 + 4 * kb, make_smem_desc(ssfa + 512 * kb, 0, 128, kLayoutSwizzleNone));
-            tmem_cp_32x128b_warpx4_pair(tmem + kColSFB2 + 8 * kb, make_smem_desc(ssfb0 + 512 * kb, 0, 128, kLayoutSwizzleNone));
-            tmem_cp_32x128b_warpx4_pair(tmem + kColSFB2 + 8 * kb + 4, make_smem_desc(ssfb1 + 512 * kb, 0, 128, kLayoutSwizzleNone));
+            tmem_cp_32x128b_warpx4_pair(tmem + kColSFB2 + 8 * kb, make_smem_desc(ssfb + 512 * kb, 0, 128, kLayoutSwizzleNone));
+            tmem_cp_32x128b_warpx4_pair(tmem + kColSFB2 + 8 * kb + 4,
+                                        make_smem_desc(ssfb + kSFBBytes / 2 + 512 * kb, 0, 128, kLayoutSwizzleNone));
           }
           const uint64_t adesc = make_smem_desc(sa, 16, 1024, kLayoutSwizzle128B);
           const uint64_t bdesc = make_smem_desc(sb, 16, 1024, kLayoutSwizzle128B);
@@ -611,10 +711,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           any_issued = true;
           tc_commit_pair_mc(&tail->empty[stage], 0x3);
           if (++stage == kStages2) { stage = 0; phase ^= 1u; }
-          if (j == kSFGroup - 1 || ks == KS - 1) {
-            tc_commit_pair_mc(&tail->sf_empty[sslot], 0x3);
-            if (++sslot == kSFSlots) { sslot = 0; sphase ^= 1u; }
-          }
         }
         if (!ok) break;
         tc_commit_pair_mc(&tail->tmem_full[buf], 0x3);
@@ -626,22 +722,20 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // ------------------------------------------------------------ epilogue (both CTAs)
-    const int q = warp & 3;
-    const int h = (warp - 2) >> 2;
+    const int q = warp & 3;           // TMEM lane quadrant this warp may read
+    const int g = (warp - 2) >> 2;    // column group: 64 of the tile's 256 columns
+    uint8_t* buf_smem = epi_smem + (warp - 2) * kEpiChunkBytes;
     uint32_t empty_leader[2], ovl_leader[2];
     for (int b = 0; b < 2; ++b) {
       empty_leader[b] = map_to_rank(smem_u32(&tail->tmem_empty[b]), 0);
       ovl_leader[b] = map_to_rank(smem_u32(&tail->ovl_free[b]), 0);
     }
-    // chunk c of this warp sits at buffer column cc[c]; the shared columns are
-    // buffer 0's [192, 256) (chunks 2, 3 of the h = 1 warps) and buffer 1's
-    // [0, 64) (chunks 0, 1 of the h = 0 warps), in both layouts
-    uint32_t cc[4];
-    if (!args.swiglu) {
-      cc[0] = h * 128; cc[1] = h * 128 + 32; cc[2] = h * 128 + 64; cc[3] = h * 128 + 96;
-    } else {
-      cc[0] = h * 64; cc[1] = h * 64 + 32; cc[2] = 128 + h * 64; cc[3] = 128 + h * 64 + 32;
-    }
+    // This warp's two 32-column chunks sit at buffer columns c0 and c1: group
+    // g's columns [64g, 64g + 64), or for SwiGLU the gate chunk 32g and its up
+    // chunk 128 + 32g.  The shared columns are buffer 0's [192, 256) and
+    // buffer 1's [0, 64).
+    const uint32_t c0 = SWIGLU ? 32u * g : 64u * g;
+    const uint32_t c1 = SWIGLU ? 128u + 32u * g : 64u * g + 32u;
     int local = 0;
     for (int t = pair; t < num_tiles; t += num_pairs, ++local) {
       int m_blk, n_blk;
@@ -650,53 +744,27 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!mbar_wait_bounded(&tail->tmem_full[buf], (local >> 1) & 1, abort_flag)) break;
       tc_fence_after();
       const uint32_t base = tmem + (static_cast<uint32_t>(q * 32) << 16) + col_acc2(buf);
-      uint32_t r0[32], r1[32], r2[32], r3[32];
-      const bool shared = h == (buf ? 0 : 1);
-      if (shared) {
-        if (buf == 0) {
-          tmem_ld_32x32b_x32(base + cc[2], r2);
-          tmem_ld_32x32b_x32(base + cc[3], r3);
-        } else {
-          tmem_ld_32x32b_x32(base + cc[0], r0);
-          tmem_ld_32x32b_x32(base + cc[1], r1);
-        }
-        tmem_ld_wait();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive_remote(ovl_leader[buf]);
-        if (buf == 0) {
-          tmem_ld_32x32b_x32(base + cc[0], r0);
-          tmem_ld_32x32b_x32(base + cc[1], r1);
-        } else {
-          tmem_ld_32x32b_x32(base + cc[2], r2);
-          tmem_ld_32x32b_x32(base + cc[3], r3);
-        }
-      } else {
-        tmem_ld_32x32b_x32(base + cc[0], r0);
-        tmem_ld_32x32b_x32(base + cc[1], r1);
-        tmem_ld_32x32b_x32(base + cc[2], r2);
-        tmem_ld_32x32b_x32(base + cc[3], r3);
-      }
+      uint32_t r0[32], r1[32];
+      tmem_ld_32x32b_x32(base + c0, r0);
+      tmem_ld_32x32b_x32(base + c1, r1);
       tmem_ld_wait();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive_remote(empty_leader[buf]);
-
-      const int64_t row = static_cast<int64_t>(m_blk) * 256 + rank * 128 + q * 32 + lane;
-      if (row < args.M) {
-        if (!args.swiglu) {
-          const int64_t n0 = static_cast<int64_t>(n_blk) * BN + h * 128;
-          store_chunk(args, row, n0 + 0, r0);
-          store_chunk(args, row, n0 + 32, r1);
-          store_chunk(args, row, n0 + 64, r2);
-          store_chunk(args, row, n0 + 96, r3);
-        } else {
-          const int64_t o0 = static_cast<int64_t>(n_blk) * 128 + h * 64;
-          store_swiglu(args, row, o0, r0, r2);
-          store_swiglu(args, row, o0 + 32, r1, r3);
-        }
+      const bool shared = buf == 0 ? (c1 >= 192u) : (c0 < 64u);
+      if (lane == 0) {
+        if (shared) mbar_arrive_remote(ovl_leader[buf]);
+        mbar_arrive_remote(empty_leader[buf]);
+      }
+      const int64_t row0 = static_cast<int64_t>(m_blk) * 256 + rank * 128 + q * 32;
+      if constexpr (!SWIGLU) {
+        store_pair_staged(args, out_maps, buf_smem, row0, static_cast<int64_t>(n_blk) * BN + 64 * g, r0, r1);
+      } else {
+        store_swiglu_staged(args, out_maps, buf_smem, row0, static_cast<int64_t>(n_blk) * 128 + 32 * g, r0, r1);
       }
     }
+    // every TMA store has read its buffer and written global memory
+    if (lane == 0) bulk_wait_group_all();
+    __syncwarp();
   }
 
   tc_fence_before();
@@ -966,6 +1034,30 @@ bool make_sf_map(CUtensorMap* m, const uint8_t* sf, int64_t rows, int64_t K, uin
                      CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Output maps for the staged epilogue of the pair kernel: one per BF16
+// segment (identity or SwiGLU output) at least 64 columns wide, dims
+// {segment width, M}, with the box of the kernel's mode (see OutMaps).
+// Other segments keep the per-lane stores (mask bit clear).
+uint32_t make_out_maps(const GemmProblem& p, OutMaps* maps) {
+  uint32_t mask = 0;
+  for (int s = 0; s < p.nseg; ++s) {
+    const EpiSegment& sg = p.seg[s];
+    const bool bf16 = sg.kind == NVFP4_EPI_IDENTITY_BF16 || sg.kind == NVFP4_EPI_SWIGLU_GATE;
+    if (!bf16 || sg.out == nullptr) continue;
+    const int64_t width = p.swiglu ? p.N / 2 : sg.n_end - sg.n_begin;
+    if (width < 64 || p.M < 1 || (sg.ld_out * 2) % 16 != 0) continue;
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(width), static_cast<cuuint64_t>(p.M)};
+    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(sg.ld_out * 2)};
+    const cuuint32_t box[2] = {p.swiglu ? 32u : 64u, p.swiglu ? 32u : 16u};
+    const cuuint32_t estr[2] = {1, 1};
+    if (encode_fn()(&maps->m[s], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, sg.out, dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, p.swiglu ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS)
+      mask |= 1u << s;
+  }
+  return mask;
+}
+
 }  // namespace gk
 
 size_t gemm_workspace_bytes(int64_t, int64_t, int64_t) { return 0; }
@@ -999,15 +1091,16 @@ cudaError_t launch_gemm(const GemmProblem& p, void*, size_t, cudaStream_t stream
   a.num_m_blocks = static_cast<int>(ceil_div(p.M, pair_kernel ? 2 * BM : BM));
   a.num_n_blocks = static_cast<int>(p.swiglu ? ceil_div(p.N / 2, 128) : ceil_div(p.N, BN));
   a.num_k_stages = static_cast<int>(ceil_div(p.K, BK));
-  a.group_m = pair_kernel ? 8 : 16;
+  a.group_m = pair_kernel ? 32 : 16;
   if (pair_kernel) {
     // Tiles are walked m-fastest inside groups of group_m row blocks: the
     // group's A panels stay in L2 while W streams through once per group.
     // When all of A fits in L2 with room for the output stream, one group
-    // covers every row block, so W is read from DRAM once.  (Keeping W
-    // resident instead, one row block per group, cut DRAM reads for the GDN
-    // shape but ran slower: every pair then starts the same new A panel at
-    // once.)
+    // covers every row block, so W is read from DRAM once; otherwise groups
+    // of 32 row blocks (8192 rows, about 24 MB of A at K = 5120) read W once
+    // per group.  (Measured on the GDN shape: groups of 32 ran 2.5% faster
+    // than groups of 8 or 16; one row block per group, keeping W resident,
+    // ran slower: every pair then starts the same new A panel at once.)
     const double a_bytes = static_cast<double>(p.M) * static_cast<double>(p.K) * (0.5 + 1.0 / 16);
     constexpr double kResident = 48.0 * 1024 * 1024;
     if (a_bytes <= kResident) a.group_m = a.num_m_blocks;
@@ -1081,19 +1174,26 @@ cudaError_t launch_gemm(const GemmProblem& p, void*, size_t, cudaStream_t stream
     cfg.numAttrs = 2;
     return cudaLaunchKernelEx(&cfg, gemm_pair_db_kernel, tm_a, tm_b3, tm_sfa, tm_sfb3, b);
   }
-  CUtensorMap tm_sfa4, tm_sfb4, tm_sfb8;
-  if (!make_sf_map(&tm_sfa4, p.a_sf, p.M, p.K, 4 * kSFGroup, 1) || !make_sf_map(&tm_sfb4, p.w_sf, p.N, p.K, 4 * kSFGroup, 1) ||
-      !make_sf_map(&tm_sfb8, p.w_sf, p.N, p.K, 4 * kSFGroup, 2))
+  // scale atoms of one K-stage: this CTA's 128 A rows; the tile's 256 B rows
+  // (two consecutive 128-row blocks, or for SwiGLU the gate and up blocks,
+  // one box each)
+  CUtensorMap tm_sfa1, tm_sfb2;
+  if (!make_sf_map(&tm_sfa1, p.a_sf, p.M, p.K, 4, 1) || !make_sf_map(&tm_sfb2, p.w_sf, p.N, p.K, 4, p.swiglu ? 1 : 2))
     return cudaErrorInvalidValue;
+  OutMaps maps{};
+  a.tma_mask = make_out_maps(p, &maps);
   static std::atomic<uint64_t> attr2_done{0};
   cudaError_t ea = once_per_device(attr2_done, [] {
-    return cudaFuncSetAttribute(gemm_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes2);
+    cudaError_t e = cudaFuncSetAttribute(gemm_pair_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes2);
+    return e != cudaSuccess ? e
+                            : cudaFuncSetAttribute(gemm_pair_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                   kSmemBytes2);
   });
   if (ea != cudaSuccess) return ea;
   const int pairs = tiles < sms / 2 ? tiles : sms / 2;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(2 * pairs);
-  cfg.blockDim = dim3(kThreads);
+  cfg.blockDim = dim3(kThreads2);
   cfg.dynamicSmemBytes = kSmemBytes2;
   cfg.stream = stream;
   cudaLaunchAttribute attr[2];
@@ -1105,7 +1205,8 @@ cudaError_t launch_gemm(const GemmProblem& p, void*, size_t, cudaStream_t stream
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 2;
-  return cudaLaunchKernelEx(&cfg, gemm_pair_kernel, tm_a, tm_b, tm_sfa4, tm_sfb4, tm_sfb8, a);
+  if (p.swiglu) return cudaLaunchKernelEx(&cfg, gemm_pair_kernel<true>, tm_a, tm_b, tm_sfa1, tm_sfb2, a, maps);
+  return cudaLaunchKernelEx(&cfg, gemm_pair_kernel<false>, tm_a, tm_b, tm_sfa1, tm_sfb2, a, maps);
 }
 
 }  // namespace nvfp4
