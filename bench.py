@@ -352,6 +352,17 @@ def run_product(args):
             step.gg[r].replay()
         evs[2].record(stream)
 
+    def chain(fn):
+        # K calls of one stage over the rotating input sets, captured in one
+        # CUDA graph: consecutive launches overlap prologue and tail through
+        # programmatic dependent launch, as a model's layer sequence does
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for i in range(K):
+                fn(step.sets[i % R])
+        return g
+
+    main = chain(step.linear if step.w is not None else step.quantize)
     for i in range(Wm):
         step.step_graph(i % R).replay()
     torch.cuda.synchronize()
@@ -360,12 +371,12 @@ def run_product(args):
     clocks = ClockSampler(local)
     clocks.start()
     time.sleep(0.3)
-    # timed region: K steps, each one pass of the path (the layer call)
+    # timed region: K steps, each one pass of the path (the layer call), as
+    # one graph replay
     dist_barrier(dist)
     torch.cuda.synchronize()
     t0.record(stream)
-    for i in range(K):
-        step.step_graph(i % R).replay()
+    main.replay()
     t1.record(stream)
     torch.cuda.synchronize()
     dist_barrier(dist)
@@ -377,27 +388,27 @@ def run_product(args):
         staged(i, evs[i])
     torch.cuda.synchronize()
 
-    def replay_ms(graphs):
-        # K replays of one graph form, after a short warm-up
-        for i in range(min(Wm, 3)):
-            graphs[i % R].replay()
+    def chain_ms(fn):
+        # K chained launches of one stage in one graph, after one warm-up replay
+        g = chain(fn)
+        g.replay()
         torch.cuda.synchronize()
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record(stream)
-        for i in range(K):
-            graphs[i % R].replay()
+        g.replay()
         b.record(stream)
         torch.cuda.synchronize()
+        del g
         return a.elapsed_time(b) / K
 
     # one-pass (calibrated static scale) forms beside the two-pass ones
-    q1_ms = replay_ms(step.gqs)
-    l1_ms = replay_ms(step.gls) if step.w is not None else None
+    q1_ms = chain_ms(step.quantize_static)
+    l1_ms = chain_ms(step.linear_static) if step.w is not None else None
     # each stage launched back to back K times (rotating inputs): the average
     # launch duration the roofline divides by; the isolated, event-bracketed
     # stage times are reported beside it
-    qb2b_ms = replay_ms(step.gq)
-    gb2b_ms = replay_ms(step.gg) if step.w is not None else None
+    qb2b_ms = chain_ms(step.quantize)
+    gb2b_ms = chain_ms(step.gemm) if step.w is not None else None
     clk = clocks.stop()
     total_ms = t0.elapsed_time(t1)
     total_ms = dist_max(dist, total_ms, device)
@@ -470,7 +481,9 @@ def run_product(args):
         "config": {"workload": step.name if step.w is None else step.w.name, "M": step.M, "N": step.N, "K": step.K,
                    "parallelism": "replicas" if world > 1 else "single",
                    "l2": f"{R} rotating input sets, {'weights rotated too, ' if args.workload.startswith('decode') else ''}"
-                         "working set above the 126 MB L2" if R > 1 else "input larger than L2"},
+                         "working set above the 126 MB L2" if R > 1 else "input larger than L2",
+                   "launch": "the K timed steps are one CUDA graph of K chained layer calls (programmatic dependent "
+                             "launch between kernels); dominant-kernel back-to-back times likewise"},
         "roofline": roof, "kernels": kernels, "clocks": clk, "e2e": e2e,
         "gpu_launches": step.launches_per_step() * K,
     }
@@ -550,20 +563,24 @@ def measure_quantizer(device, K, Wm, hbm):
     step.capture()
     stream = torch.cuda.current_stream()
 
-    def b2b(graphs):
-        for i in range(max(Wm, 3)):
-            graphs[0].replay()
+    def b2b(fn):
+        # K chained launches in one CUDA graph, after one warm-up replay
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for _ in range(K):
+                fn(step.sets[0])
+        g.replay()
         torch.cuda.synchronize()
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record(stream)
-        for _ in range(K):
-            graphs[0].replay()
+        g.replay()
         b.record(stream)
         torch.cuda.synchronize()
+        del g
         return a.elapsed_time(b) / K
 
-    dyn_ms = b2b(step.gq)
-    cal_ms = b2b(step.gqs)
+    dyn_ms = b2b(step.quantize)
+    cal_ms = b2b(step.quantize_static)
     qb = step.alg_bytes_quant()
     dyn_gbs = (qb["amax"] + qb["quantize"]) / (dyn_ms * 1e-3) / 1e9
     cal_gbs = qb["quantize"] / (cal_ms * 1e-3) / 1e9
