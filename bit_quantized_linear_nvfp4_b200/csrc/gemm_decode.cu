@@ -247,7 +247,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     grid_dependency_wait();  // g_a, the segment scales and the outputs
     const int q = warp & 3;
     const int row_local = q * 32 + lane;
-    const int64_t n = static_cast<int64_t>(rb) * BM + row_local;
     float acc[BN];
     bool have = (ks1 > ks0) && mbar_wait_bounded(&tail->tmem_full, 0, abort_flag);
     if (have) {

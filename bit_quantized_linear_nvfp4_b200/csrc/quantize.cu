@@ -28,10 +28,11 @@
 // backwards, so that when x is larger than L2 it starts on the chunks the
 // amax kernel read last.
 //
-// Small inputs with a device-computed scale (up to 8 blocks' worth): one
-// launch of a thread-block cluster; each block copies its share of x into
-// shared memory once, the blocks exchange their maxima through distributed
-// shared memory, and quantise from shared memory.
+// Small inputs with a device-computed scale (up to 512 chunks, 256 K
+// elements: a decode step's activations): one launch of a cluster of up to 8
+// small blocks; each block takes the amax of its share with register loads,
+// the blocks exchange their maxima through distributed shared memory, and
+// each quantises its share reading x again from L2.
 #include <cfloat>
 #include <cstdint>
 
@@ -295,12 +296,12 @@ __device__ __forceinline__ void quantize_block(const QuantArgs& a, const float* 
 // (w / 4) + 32 * (w % 4) of the block, so a warp walks an atom's 128 words in
 // order (coalesced 128-byte stores) and writes those of padding rows.  Warps
 // of the whole grid take atoms.
-__device__ __forceinline__ void zero_padding_rows(const QuantArgs& a) {
+__device__ __forceinline__ void zero_padding_rows_n(const QuantArgs& a, int warps_per_block) {
   if (a.rows_pad == a.M) return;
   const int32_t KA = (a.K + 63) / 64;
   const int32_t rb = a.M >> 7;
   const int lane = threadIdx.x & 31;
-  const int32_t gw = blockIdx.x * kWarps + (threadIdx.x >> 5), nw = gridDim.x * kWarps;
+  const int32_t gw = blockIdx.x * warps_per_block + (threadIdx.x >> 5), nw = gridDim.x * warps_per_block;
   for (int32_t kb = gw; kb < KA; kb += nw) {
     uint32_t* atom = reinterpret_cast<uint32_t*>(a.sf + (static_cast<int64_t>(rb) * KA + kb) * 512);
 #pragma unroll
@@ -310,6 +311,8 @@ __device__ __forceinline__ void zero_padding_rows(const QuantArgs& a) {
     }
   }
 }
+
+__device__ __forceinline__ void zero_padding_rows(const QuantArgs& a) { zero_padding_rows_n(a, kWarps); }
 
 // Pass 1 (device-computed scale): per-segment amax of the block's chunks,
 // stored to partial[block][segment].
@@ -404,111 +407,57 @@ __global__ void __launch_bounds__(kThreads, 1) quant_kernel(const __grid_constan
   zero_padding_rows(a);
 }
 
-// Copies of up to 32 consecutive chunks [i0, i1) (lane j: chunk i0 + j) into
-// dst + j * kChunkBytes.  Chunks that follow one another both in x and in dst
-// (full chunks of one row, or of consecutive rows when rows are packed) are
-// merged into one copy, because a bulk copy costs about the same whatever its
-// size up to several KB.  plan() is warp-collective; issue() then starts the
-// copies on `bar`, after the caller has raised the barrier's expected bytes by
-// `total`.
-template <int DTYPE>
-struct ChunkCopies {
-  using C = Cfg<DTYPE>;
-  const uint8_t* src = nullptr;
-  uint32_t run = 0;    // bytes of the copy this lane starts (0: none)
-  uint32_t total = 0;  // bytes of all the chunks
-
-  __device__ __forceinline__ void plan(const QuantArgs& a, int64_t i0, int64_t i1) {
-    const int lane = threadIdx.x & 31;
-    const int64_t item = i0 + lane;
-    uint32_t bytes = 0;
-    if (item < i1) {
-      int32_t row, col;
-      chunk_pos(a, item, row, col);
-      const int32_t n = a.K - col < kChunk ? a.K - col : kChunk;
-      bytes = static_cast<uint32_t>(n) * C::kEsz;
-      src = a.x + row * a.ld_bytes + static_cast<int64_t>(col) * C::kEsz;
-    }
-    // a copy starts at every chunk that does not continue the previous one
-    const uint32_t prev_bytes = __shfl_up_sync(0xffffffffu, bytes, 1);
-    const uint64_t prev_src = __shfl_up_sync(0xffffffffu, reinterpret_cast<uint64_t>(src), 1);
-    const bool continues = lane > 0 && prev_bytes == static_cast<uint32_t>(C::kChunkBytes) &&
-                           reinterpret_cast<uint64_t>(src) == prev_src + C::kChunkBytes;
-    const uint32_t starts = __ballot_sync(0xffffffffu, bytes != 0 && !continues);
-    // exclusive prefix sum of the chunk sizes
-    uint32_t incl = bytes;
-#pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-      const uint32_t v = __shfl_up_sync(0xffffffffu, incl, off);
-      if (lane >= off) incl += v;
-    }
-    total = __shfl_sync(0xffffffffu, incl, 31);
-    const uint32_t excl = incl - bytes;
-    const uint32_t later = lane < 31 ? starts & (0xfffffffeu << lane) : 0u;
-    const int next = later ? __ffs(later) - 1 : 32;
-    const uint32_t end = __shfl_sync(0xffffffffu, excl, next & 31);
-    run = ((starts >> lane) & 1u) ? (next < 32 ? end : total) - excl : 0u;
-  }
-
-  __device__ __forceinline__ void issue(uint8_t* dst, uint64_t* bar) const {
-    if (run != 0) bulk_load(dst + (threadIdx.x & 31) * C::kChunkBytes, src, run, bar);
-  }
-};
-
 // Small inputs with a device-computed scale, in one launch: a cluster of C
-// blocks (C <= 8) each copies its whole share of x into shared memory, takes
-// the block amax, reads the other blocks' maxima through distributed shared
-// memory, and quantises from shared memory; x is read once.
-constexpr int kSmallSmem = 200 * 1024;
+// blocks (C <= 8) of 8 warps.  Each block takes the amax of its share of x
+// with register loads, reads the other blocks' maxima through distributed
+// shared memory after a cluster barrier, and quantises its share, reading x
+// again (it is a few hundred KB at most, and still in L2).  No shared-memory
+// staging: the blocks need a few KB of shared memory and 256 threads, so
+// they can run beside the weight-streaming GEMM's CTAs of the layer before.
+constexpr int kSmallWarps = 8;
+constexpr int kSmallThreads = kSmallWarps * 32;
+constexpr int kSmallChunksPerBlock = 64;  // 8 chunks per warp
 constexpr int kMaxSmallBlocks = 8;
 
-template <int DTYPE>
-__global__ void __launch_bounds__(kThreads, 1) small_kernel(const __grid_constant__ QuantArgs a) {
+template <int DTYPE, bool WIDE>
+__global__ void __launch_bounds__(kSmallThreads, 1) small_kernel(const __grid_constant__ QuantArgs a) {
   using C = Cfg<DTYPE>;
-  extern __shared__ __align__(1024) uint8_t buf[];
-  __shared__ uint64_t full;
-  __shared__ float red[kWarps][kMaxSeg];
+  __shared__ float red[kSmallWarps][kMaxSeg];
   __shared__ float blk_amax[kMaxSeg];
   __shared__ float g_sh[kMaxSeg];
-  __shared__ int abort_flag;
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  if (threadIdx.x == 0) {
-    mbar_init(&full, 1);
-    abort_flag = 0;
-    fence_mbarrier_init();
-  }
-  __syncthreads();
   if (threadIdx.x == 0) grid_launch_dependents();
-  grid_dependency_wait();
+  grid_dependency_wait();  // x may come from the kernel before this one
   int64_t lo, hi;
   block_range(a.items, lo, hi);
-  if (warp == 0) {
-    for (int64_t i0 = lo; i0 < hi; i0 += 32) {
-      ChunkCopies<DTYPE> cc;
-      cc.plan(a, i0, hi < i0 + 32 ? hi : i0 + 32);
-      if (lane == 0) mbar_expect_tx(&full, cc.total);
-      __syncwarp();
-      cc.issue(buf + (i0 - lo) * C::kChunkBytes, &full);
-    }
-    __syncwarp();
-    if (lane == 0) mbar_arrive(&full);
-  }
-  const bool ok = mbar_wait_bounded(&full, 0, &abort_flag);
-
   SegMax sm;
-  if (ok)
-    for (int64_t i = lo + warp; i < hi; i += kWarps) {
-      int32_t row, col;
-      chunk_pos(a, i, row, col);
-      if (col + lane * 16 < a.K) {
-        Blk<DTYPE> b;
-        load_shared<DTYPE>(buf + (i - lo) * C::kChunkBytes + lane * 16 * C::kEsz, b);
-        sm.add(find_segment(a, row), block_amax<DTYPE>(b));
-      }
+  for (int64_t i = lo + warp; i < hi; i += kSmallWarps) {
+    int32_t row, col;
+    chunk_pos(a, i, row, col);
+    col += lane * 16;
+    if (col < a.K) {
+      Blk<DTYPE> b;
+      load_global<DTYPE, WIDE>(a.x + row * a.ld_bytes + static_cast<int64_t>(col) * C::kEsz, b);
+      sm.add(find_segment(a, row), block_amax<DTYPE>(b));
     }
-  const float m = sm.reduce(a.nseg, red);
-  if (warp < a.nseg && lane == 0) blk_amax[warp] = m;
+  }
+  // block maxima per segment: warp-reduce, then warp s combines segment s
+#pragma unroll
+  for (int s = 0; s < kMaxSeg; ++s) {
+    if (s >= a.nseg) break;  // uniform
+    float v = sm.m[s];
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, off));
+    if (lane == 0) red[warp][s] = v;
+  }
+  __syncthreads();
+  if (threadIdx.x < a.nseg) {
+    float v = 0.0f;
+#pragma unroll
+    for (int w = 0; w < kSmallWarps; ++w) v = fmaxf(v, red[w][threadIdx.x]);
+    blk_amax[threadIdx.x] = v;
+  }
   cluster_sync_all();  // every block's maxima are visible to the cluster
   if (threadIdx.x < a.nseg) {
     float v = 0.0f;
@@ -518,19 +467,16 @@ __global__ void __launch_bounds__(kThreads, 1) small_kernel(const __grid_constan
   }
   __syncthreads();
   if (blockIdx.x == 0 && threadIdx.x < a.nseg) a.g_out[threadIdx.x] = g_sh[threadIdx.x];
-  if (ok)
-    for (int64_t i = lo + warp; i < hi; i += kWarps) {
-      int32_t row, col;
-      chunk_pos(a, i, row, col);
-      col += lane * 16;
-      Blk<DTYPE> b;
-      const bool have = col < a.K;
-      if (have) load_shared<DTYPE>(buf + (i - lo) * C::kChunkBytes + lane * 16 * C::kEsz, b);
-      quantize_block<DTYPE>(a, g_sh, b, have, row, col);
-    }
-  zero_padding_rows(a);
-  if (!ok && threadIdx.x == 0)  // let copies still in flight land (bounded)
-    mbar_wait_bounded(&full, 0, nullptr, 200000000ull);
+  for (int64_t i = lo + warp; i < hi; i += kSmallWarps) {
+    int32_t row, col;
+    chunk_pos(a, i, row, col);
+    col += lane * 16;
+    Blk<DTYPE> b;
+    const bool have = col < a.K;
+    if (have) load_global<DTYPE, WIDE>(a.x + row * a.ld_bytes + static_cast<int64_t>(col) * C::kEsz, b);
+    quantize_block<DTYPE>(a, g_sh, b, have, row, col);
+  }
+  zero_padding_rows_n(a, kSmallWarps);
   cluster_sync_all();  // no block leaves while another may read its maxima
 }
 
@@ -650,10 +596,11 @@ int grid_for(int64_t items) {
 }
 
 template <class Kern>
-cudaError_t launch_pdl(Kern kern, int grid, int cluster, int smem, const QuantArgs& a, cudaStream_t stream) {
+cudaError_t launch_pdl(Kern kern, int grid, int cluster, int smem, const QuantArgs& a, cudaStream_t stream,
+                       int threads = kThreads) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
-  cfg.blockDim = dim3(kThreads);
+  cfg.blockDim = dim3(threads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
   cudaLaunchAttribute attr[2];
@@ -670,17 +617,10 @@ cudaError_t launch_pdl(Kern kern, int grid, int cluster, int smem, const QuantAr
 
 template <int DTYPE, bool WIDE>
 cudaError_t launch_t(QuantArgs a, bool dynamic, cudaStream_t stream) {
-  using C = Cfg<DTYPE>;
-  static std::atomic<uint64_t> attr_done{0};
-  cudaError_t ea = once_per_device(attr_done, [] {
-    return cudaFuncSetAttribute(small_kernel<DTYPE>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmallSmem);
-  });
-  if (ea != cudaSuccess) return ea;
-  constexpr int64_t kSmallChunks = kSmallSmem / C::kChunkBytes;  // per block
-  const int64_t nsmall = (a.items + kSmallChunks - 1) / kSmallChunks;
+  const int64_t nsmall = (a.items + kSmallChunksPerBlock - 1) / kSmallChunksPerBlock;
   if (dynamic && nsmall <= kMaxSmallBlocks) {
     const int blocks = nsmall < 1 ? 1 : static_cast<int>(nsmall);
-    return launch_pdl(small_kernel<DTYPE>, blocks, blocks, kSmallSmem, a, stream);
+    return launch_pdl(small_kernel<DTYPE, WIDE>, blocks, blocks, 0, a, stream, kSmallThreads);
   }
   const int grid = grid_for(a.items);
   if (dynamic) {
