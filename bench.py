@@ -186,6 +186,11 @@ class ProductStep:
             self.rotate = 1
             return
         w = self.w
+        if rows is not None and not name.startswith("decode"):
+            # the first `rows` rows of the same workload (a smaller case of the
+            # same kernels, for profiler captures)
+            import dataclasses
+            w = self.w = dataclasses.replace(w, M=rows)
         self.M, self.K, self.N = w.M, w.K, w.N
         self.flops = w.flops()
         x_np = wl.make_x(w)
@@ -1297,7 +1302,8 @@ def main():
                     help="projection workloads: skip the standalone quantiser measurement on X[32768,17408]")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--rows", type=int, default=None,
-                    help="quant: quantise [rows, 17408]; gdnrec: the first rows tokens (smaller cases for profiler captures)")
+                    help="quant: quantise [rows, 17408]; oproj/mlp/gdn: the first rows tokens; gdnrec: the first rows "
+                         "tokens (smaller cases for profiler captures)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
