@@ -46,9 +46,9 @@ TRAFFIC_BYTES = {
     "decode1": 50362112,
     "decode64": 50922752,
     "decode8": 50422528,
-    "gdn": 1401560576,
+    "gdn": 1135872000,
     "kvfp8": 73506560,
-    "mlp": 381300224,
+    "mlp": 378899712,
     "oproj": 28804864,
     "quant": 2563600000,
     "requant": 36475136,
