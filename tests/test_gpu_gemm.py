@@ -367,3 +367,37 @@ def test_wide_tiles_two_segments():
     y1, m1, _, _ = o.linear(x, w1)
     check_bf16(to_np(o0), y0, TOL_ACC * m0, "wide bf16")
     check_fp32(to_np(o1), y1, m1, "wide f32")
+
+
+def test_wide_tiles_ragged_segments():
+    """The 256-wide kernel (one M block, N above 74 x 192) with BF16 segments
+    whose boundaries are off the 8-column grid, one narrower than 64 columns
+    and an FP32 one: 64-column groups that cross a boundary or start off the
+    grid take the per-lane stores, the rest the staged TMA stores; padded
+    output strides; 200 rows, so the last 16-row store box is clipped."""
+    M, K = 200, 256
+    widths = [100, 8000, 36, 6200]
+    kinds = ["identity_bf16", "identity_bf16", "identity_bf16", "identity_f32"]
+    N = sum(widths)
+    x = _rand(M, K, 71, outliers=2)
+    ws = [_rand(w, K, 72 + i, 0.02 * (i + 1)) for i, w in enumerate(widths)]
+    bounds = np.concatenate([[0], np.cumsum(widths)])
+    A, ga = nv.nvfp4_quantize(_dev(x))
+    W, gw = nv.nvfp4_quantize_segments(_dev(np.concatenate(ws)), bounds)
+    outs, segs = [], []
+    for i, (w, kind) in enumerate(zip(widths, kinds)):
+        dt = torch.bfloat16 if kind == "identity_bf16" else torch.float32
+        unit = 8 if dt == torch.bfloat16 else 4  # row strides of 16 bytes
+        full = torch.full((M, (w // unit + 1) * unit), -7.0, dtype=dt, device=DEV)
+        outs.append(full)
+        segs.append(nv.Segment(int(bounds[i]), int(bounds[i + 1]), kind, full[:, :w]))
+    nv.nvfp4_fused_proj(A, ga, W, gw, segs)
+    torch.cuda.synchronize()
+    for i, w in enumerate(widths):
+        y, mag, _, _ = o.linear(x, ws[i])
+        got = to_np(outs[i])
+        assert np.all(got[:, w:] == -7.0), f"segment {i} wrote past its width"
+        if kinds[i] == "identity_bf16":
+            check_bf16(got[:, :w], y, TOL_ACC * mag, f"segment {i}")
+        else:
+            check_fp32(got[:, :w], y, mag, f"segment {i}")
