@@ -15,11 +15,13 @@
 //   col_sq[K], col_max[K] (FP32): sum x^2 and max |x| per column.
 //
 // HBM-bound.  A warp owns a unit = (512-column strip, range of rows); lane l
-// reads block l of the strip in each row with one 256-bit load, several rows in
-// flight.  Per-column sums stay in the lane's registers for the whole unit,
-// so the column outputs take one atomic per column and unit; row sums are
-// warp-reduced, one atomic per row and strip; FP64 moments are block-reduced,
-// one atomic per block.
+// reads block l of the strip in each row with one 256-bit load; rows stream
+// in pairs through two register buffers, the next pair loading while the
+// current one is processed.  Per-column sums stay in the lane's registers for
+// the whole unit, so the column outputs take one atomic per column and unit;
+// the row sums of four rows are reduced together (one reduce-scatter), one
+// atomic per row and strip; FP64 moments are block-reduced, one atomic per
+// block.
 #include <cfloat>
 #include <cstdint>
 
@@ -137,16 +139,109 @@ __device__ __forceinline__ double warp_sum(double v) {
   for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
   return v;
 }
-__device__ __forceinline__ float warp_sumf(float v) {
+
+// Sums over the warp of eight per-lane values in 9 shuffles (a reduce-scatter
+// of halves, then a butterfly over groups of four lanes).  Afterwards every
+// lane holds the total of value ((l >> 4) & 1) * 4 + ((l >> 3) & 1) * 2 +
+// ((l >> 2) & 1), l its lane.
+__device__ __forceinline__ float warp_sum8(const float (&v)[8], int lane) {
+  const bool b4 = (lane & 16) != 0, b3 = (lane & 8) != 0, b2 = (lane & 4) != 0;
+  float h4[4], h2[2];
 #pragma unroll
-  for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
-  return v;
+  for (int i = 0; i < 4; ++i) {
+    const float send = b4 ? v[i] : v[i + 4];
+    h4[i] = (b4 ? v[i + 4] : v[i]) + __shfl_xor_sync(0xffffffffu, send, 16);
+  }
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    const float send = b3 ? h4[i] : h4[i + 2];
+    h2[i] = (b3 ? h4[i + 2] : h4[i]) + __shfl_xor_sync(0xffffffffu, send, 8);
+  }
+  float h1 = (b2 ? h2[1] : h2[0]) + __shfl_xor_sync(0xffffffffu, b2 ? h2[0] : h2[1], 4);
+  h1 += __shfl_xor_sync(0xffffffffu, h1, 2);
+  h1 += __shfl_xor_sync(0xffffffffu, h1, 1);
+  return h1;
+}
+
+// Statistics of one lane's 16-element block of one row: moments, column
+// accumulators, dominance, and the row's sum x^2 (rn2) and sum (x - x_hat)^2
+// (re2).
+template <int DTYPE>
+__device__ __forceinline__ void block_stats(const Raw<DTYPE>& raw, bool quant, float g, float (&csq)[16],
+                                            float (&cmx)[16], double& s1, double& s2, double& s3, double& s4,
+                                            float& amax, double& blocks, double& dom, float& rn2, float& re2) {
+  float v[16];
+  to_f32<DTYPE>(raw, v);
+  float am = 0.0f, asum = 0.0f;
+  uint64_t p1 = 0, p2 = 0, p3 = 0, p4 = 0;  // packed even/odd partial sums
+#pragma unroll
+  for (int e = 0; e < 16; e += 2) {
+    const uint64_t xv = pk(v[e], v[e + 1]);
+    const uint64_t x2 = mul2(xv, xv);
+    p1 = add2(p1, xv);
+    p2 = add2(p2, x2);
+    p3 = fma2(x2, xv, p3);
+    p4 = fma2(x2, x2, p4);
+    const float2 sq = upk(x2);
+    csq[e] += sq.x;
+    csq[e + 1] += sq.y;
+    const float a0 = fabsf(v[e]), a1 = fabsf(v[e + 1]);
+    cmx[e] = fmaxf(cmx[e], a0);
+    cmx[e + 1] = fmaxf(cmx[e + 1], a1);
+    am = fmaxf(am, fmaxf(a0, a1));
+    asum += a0 + a1;
+  }
+  const float2 f1 = upk(p1), f2 = upk(p2), f3 = upk(p3), f4 = upk(p4);
+  amax = fmaxf(amax, am);
+  s1 += f1.x + f1.y; s2 += f2.x + f2.y; s3 += f3.x + f3.y; s4 += f4.x + f4.y;
+  blocks += 1.0;
+  // Dominated: am > (sum |x|) - am, decided in FP64 like the definition.  The
+  // FP32 sum of 16 non-negative terms is within 2^-20 of the exact sum, so
+  // outside a 2^-18 margin the FP32 comparison gives the same answer; inside
+  // it the exact FP64 test runs.
+  const float two_am = 2.0f * am;
+  bool d;
+  if (two_am > asum * (1.0f + 0x1p-18f)) {
+    d = true;
+  } else if (two_am < asum * (1.0f - 0x1p-18f)) {
+    d = false;
+  } else {
+    double asum64 = 0.0;
+#pragma unroll
+    for (int e = 0; e < 16; ++e) asum64 += static_cast<double>(fabsf(v[e]));
+    d = static_cast<double>(am) > asum64 - static_cast<double>(am);
+  }
+  if (d) dom += 1.0;
+  rn2 = f2.x + f2.y;
+  re2 = 0.0f;
+  if (quant) {
+    // the quantiser's arithmetic (block scale, reciprocal, codes)
+    const float s = (am / 6.0f) / g;
+    uint16_t sr;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(sr) : "f"(0.0f), "f"(s));
+    const float S = e4m3_val(sr & 0xFFu);
+    const float denom = S * g;
+    float inv = denom > 0.0f ? 1.0f / denom : 0.0f;
+    inv = fminf(inv, FLT_MAX);
+    const uint64_t inv2 = pk(inv, inv), S2 = pk(S, S), g2 = pk(g, g);
+    uint64_t e2 = 0;
+#pragma unroll
+    for (int e = 0; e < 16; e += 2) {
+      const uint64_t xv = pk(v[e], v[e + 1]);
+      const float2 c = e2m1_round2(upk(mul2(xv, inv2)));
+      // x_hat = (e2m1 * S) * g, each product rounded on its own
+      const uint64_t xh = mul2(mul2(pk(c.x, c.y), S2), g2);
+      const uint64_t dd = add2(xv, xh ^ 0x8000000080000000ull);  // x - x_hat
+      e2 = fma2(dd, dd, e2);
+    }
+    const float2 fe = upk(e2);
+    re2 = fe.x + fe.y;
+  }
 }
 
 template <int DTYPE, bool WIDE>
 __global__ void __launch_bounds__(kThreads, 2) stats_kernel(const __grid_constant__ StatsArgs a) {
   constexpr int kEsz = DTYPE == NVFP4_DTYPE_BF16 ? 2 : 4;
-  constexpr int kRows = DTYPE == NVFP4_DTYPE_BF16 ? 4 : 2;  // rows in flight per warp
   __shared__ double red[kWarps][8];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   grid_dependency_wait();
@@ -164,77 +259,48 @@ __global__ void __launch_bounds__(kThreads, 2) stats_kernel(const __grid_constan
     const int32_t r1 = static_cast<int32_t>(static_cast<int64_t>(a.M) * (rr + 1) / a.ranges);
     const int32_t col = strip * 512 + lane * 16;
     const bool have = col < a.K;
+    const uint8_t* xp = a.x + static_cast<int64_t>(col) * kEsz;
     float csq[16], cmx[16];
 #pragma unroll
     for (int e = 0; e < 16; ++e) csq[e] = cmx[e] = 0.0f;
-    for (int32_t row0 = r0; row0 < r1; row0 += kRows) {
-      Raw<DTYPE> raw[kRows];
+    // Rows stream in pairs through two register buffers: the loads of the
+    // next pair are issued before the current pair is processed.  Every four
+    // rows, their row sums are reduced together and added with one atomic
+    // per lane group.
+    Raw<DTYPE> ra[2], rb[2];
 #pragma unroll
-      for (int k = 0; k < kRows; ++k)
+    for (int k = 0; k < 2; ++k)
+      if (have && r0 + k < r1) load<DTYPE, WIDE>(xp + static_cast<int64_t>(r0 + k) * a.ld_bytes, ra[k]);
+    for (int32_t row0 = r0; row0 < r1; row0 += 4) {
+      float sums[8];
+#pragma unroll
+      for (int k = 0; k < 2; ++k)
+        if (have && row0 + 2 + k < r1) load<DTYPE, WIDE>(xp + static_cast<int64_t>(row0 + 2 + k) * a.ld_bytes, rb[k]);
+#pragma unroll
+      for (int k = 0; k < 2; ++k) {
+        sums[k] = sums[4 + k] = 0.0f;
         if (have && row0 + k < r1)
-          load<DTYPE, WIDE>(a.x + static_cast<int64_t>(row0 + k) * a.ld_bytes + static_cast<int64_t>(col) * kEsz, raw[k]);
+          block_stats<DTYPE>(ra[k], quant, g, csq, cmx, s1, s2, s3, s4, amax, blocks, dom, sums[k], sums[4 + k]);
+      }
 #pragma unroll
-      for (int k = 0; k < kRows; ++k) {
-        if (row0 + k >= r1) break;  // uniform across the warp
-        float rn2 = 0.0f, re2 = 0.0f;
-        if (have) {
-          float v[16];
-          to_f32<DTYPE>(raw[k], v);
-          float am = 0.0f;
-          double asum = 0.0;
-          uint64_t p1 = 0, p2 = 0, p3 = 0, p4 = 0;  // packed even/odd partial sums
+      for (int k = 0; k < 2; ++k)
+        if (have && row0 + 4 + k < r1) load<DTYPE, WIDE>(xp + static_cast<int64_t>(row0 + 4 + k) * a.ld_bytes, ra[k]);
 #pragma unroll
-          for (int e = 0; e < 16; e += 2) {
-            const uint64_t xv = pk(v[e], v[e + 1]);
-            const uint64_t x2 = mul2(xv, xv);
-            p1 = add2(p1, xv);
-            p2 = add2(p2, x2);
-            p3 = fma2(x2, xv, p3);
-            p4 = fma2(x2, x2, p4);
-            const float2 sq = upk(x2);
-            csq[e] += sq.x;
-            csq[e + 1] += sq.y;
-            const float a0 = fabsf(v[e]), a1 = fabsf(v[e + 1]);
-            cmx[e] = fmaxf(cmx[e], a0);
-            cmx[e + 1] = fmaxf(cmx[e + 1], a1);
-            am = fmaxf(am, fmaxf(a0, a1));
-            asum += static_cast<double>(a0) + static_cast<double>(a1);
+      for (int k = 0; k < 2; ++k) {
+        sums[2 + k] = sums[6 + k] = 0.0f;
+        if (have && row0 + 2 + k < r1)
+          block_stats<DTYPE>(rb[k], quant, g, csq, cmx, s1, s2, s3, s4, amax, blocks, dom, sums[2 + k], sums[6 + k]);
+      }
+      const float total = warp_sum8(sums, lane);
+      if ((lane & 3) == 0) {
+        const int idx = (lane >> 2) & 7;
+        const int32_t row = row0 + (idx & 3);
+        if (row < r1) {
+          if (idx < 4) {
+            if (a.row_norm2 != nullptr) atomicAdd(a.row_norm2 + row, total);
+          } else if (a.row_err2 != nullptr && quant) {
+            atomicAdd(a.row_err2 + row, total);
           }
-          const float2 f1 = upk(p1), f2 = upk(p2), f3 = upk(p3), f4 = upk(p4);
-          amax = fmaxf(amax, am);
-          s1 += f1.x + f1.y; s2 += f2.x + f2.y; s3 += f3.x + f3.y; s4 += f4.x + f4.y;
-          blocks += 1.0;
-          if (static_cast<double>(am) > asum - static_cast<double>(am)) dom += 1.0;
-          rn2 = f2.x + f2.y;
-          if (quant) {
-            // the quantiser's arithmetic (block scale, reciprocal, codes)
-            const float s = (am / 6.0f) / g;
-            uint16_t sr;
-            asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(sr) : "f"(0.0f), "f"(s));
-            const float S = e4m3_val(sr & 0xFFu);
-            const float denom = S * g;
-            float inv = denom > 0.0f ? 1.0f / denom : 0.0f;
-            inv = fminf(inv, FLT_MAX);
-            const uint64_t inv2 = pk(inv, inv), S2 = pk(S, S), g2 = pk(g, g);
-            uint64_t e2 = 0;
-#pragma unroll
-            for (int e = 0; e < 16; e += 2) {
-              const uint64_t xv = pk(v[e], v[e + 1]);
-              const float2 c = e2m1_round2(upk(mul2(xv, inv2)));
-              // x_hat = (e2m1 * S) * g, each product rounded on its own
-              const uint64_t xh = mul2(mul2(pk(c.x, c.y), S2), g2);
-              const uint64_t d = add2(xv, xh ^ 0x8000000080000000ull);  // x - x_hat
-              e2 = fma2(d, d, e2);
-            }
-            const float2 fe = upk(e2);
-            re2 = fe.x + fe.y;
-          }
-        }
-        rn2 = warp_sumf(rn2);
-        re2 = warp_sumf(re2);
-        if (lane == 0) {
-          if (a.row_norm2 != nullptr) atomicAdd(a.row_norm2 + row0 + k, rn2);
-          if (a.row_err2 != nullptr && quant) atomicAdd(a.row_err2 + row0 + k, re2);
         }
       }
     }
