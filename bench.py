@@ -41,11 +41,11 @@ ROTATE = 4          # rotating input sets so consecutive steps miss in L2
 # and scaled by 4 rows-wise (the traffic grows with the rows).  "gdnrec": both
 # recurrence launches, captured at 8192 tokens and scaled by 4 (all of it is per chunk).
 TRAFFIC_BYTES = {
-    "actstats": 339406592,
+    "actstats": 339345408,
     "gdnrec": 3817484288,
     "decode1": 50362112,
-    "decode64": 50922752,
-    "decode8": 50422528,
+    "decode64": 50916352,
+    "decode8": 50420224,
     "gdn": 1135872000,
     "kvfp8": 73506560,
     "mlp": 378899712,
