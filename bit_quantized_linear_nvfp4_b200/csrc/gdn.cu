@@ -47,10 +47,16 @@ constexpr int C = 64;        // tokens per chunk
 constexpr int DK = 64;       // key / query head dimension
 constexpr int DV = 128;      // value head dimension
 constexpr int LD64 = 68;     // padded row stride (floats) of 64-wide tiles in shared memory
-constexpr int LD128 = 132;   // of 128-wide tiles
 constexpr int kThreads = 256;
 constexpr int kRows = 32;    // state rows per CTA of the state pass
 constexpr int kRec = 3 * 128 * 64;  // floats per (chunk, head) record: [M^T; R], N, Y^T
+
+// Element (r, c) of a row-major tile of 64-float rows whose 16-byte pieces are
+// XOR-swizzled by the row: piece c / 4 of row r sits at piece (c / 4) ^ (r % 8).
+// Eight consecutive rows then place any one piece in eight different bank
+// groups, so 8-row fragment loads are conflict-free without padding and a tile
+// moves as one contiguous copy.  The records use this layout in global memory.
+__device__ __forceinline__ int sw64(int r, int c) { return r * 64 + (((c >> 2) ^ (r & 7)) << 2) + (c & 3); }
 
 struct GdnArgs {
   const uint8_t* q;
@@ -104,55 +110,44 @@ __device__ __forceinline__ void mma_3xtf32(float (&d)[4], const float (&a)[4], f
   mma(d, ah, bh0, bh1);
 }
 
-// Fragment loaders.  gid = lane / 4, tig = lane % 4.  An A fragment holds
+// Fragment layouts (gid = lane / 4, tig = lane % 4).  An A fragment holds
 // (m0+gid, k0+tig), (m0+gid+8, k0+tig), (m0+gid, k0+tig+4), (m0+gid+8, k0+tig+4);
 // a B fragment (k0+tig, n0+gid), (k0+tig+4, n0+gid); the accumulator
 // (m0+gid, n0+2tig), (m0+gid, n0+2tig+1), (m0+gid+8, n0+2tig), (m0+gid+8, n0+2tig+1).
-
-// A[m][k] = X[m][k] (X row-major, stride ld).
-__device__ __forceinline__ void frag_a(uint32_t (&a)[4], const float* X, int ld, int m0, int k0, int gid, int tig) {
-  a[0] = tf32(X[(m0 + gid) * ld + k0 + tig]);
-  a[1] = tf32(X[(m0 + gid + 8) * ld + k0 + tig]);
-  a[2] = tf32(X[(m0 + gid) * ld + k0 + tig + 4]);
-  a[3] = tf32(X[(m0 + gid + 8) * ld + k0 + tig + 4]);
+//
+// Both operand fragments are blocks of 8 rows x 4 consecutive FP32 words of a
+// row-major tile (for B, a tile stored with n as the row), which is what
+// ldmatrix distributes: four 8 x 8 matrices of 16-bit elements, lane l
+// supplying the address of row l % 8 of matrix l / 8 and receiving word
+// (row l / 4, column l % 4) of every matrix.  Tiles in shared memory have row
+// strides of 68 floats (17 pieces of 16 bytes), so eight consecutive rows hit
+// eight different bank groups.
+__device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], uint32_t addr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr)
+               : "memory");
 }
-// B[k][n] = X[n][k] (X stored with n as the row).
-__device__ __forceinline__ void frag_bt(uint32_t& b0, uint32_t& b1, const float* X, int ld, int n0, int k0, int gid,
-                                        int tig) {
-  b0 = tf32(X[(n0 + gid) * ld + k0 + tig]);
-  b1 = tf32(X[(n0 + gid) * ld + k0 + tig + 4]);
+// A[m][k] = X[m][k], rows m0 .. m0+15, columns k0 .. k0+7 (X row-major, stride ld).
+__device__ __forceinline__ void lda(uint32_t (&a)[4], const float* X, int ld, int m0, int k0, int lane) {
+  const int rr = lane & 7, j = lane >> 3;
+  ldsm_x4(a, smem_u32(X + (m0 + rr + 8 * (j & 1)) * ld + k0 + 4 * (j >> 1)));
 }
-// Loaders for values already rounded to TF32 (no conversion); frag_at_raw
-// reads A[m][k] = X[k][m] (X stored with k as the row).
-__device__ __forceinline__ void frag_a_raw(uint32_t (&a)[4], const float* X, int ld, int m0, int k0, int gid, int tig) {
-  a[0] = __float_as_uint(X[(m0 + gid) * ld + k0 + tig]);
-  a[1] = __float_as_uint(X[(m0 + gid + 8) * ld + k0 + tig]);
-  a[2] = __float_as_uint(X[(m0 + gid) * ld + k0 + tig + 4]);
-  a[3] = __float_as_uint(X[(m0 + gid + 8) * ld + k0 + tig + 4]);
+// B[k][n] = X[n][k] for columns n0 .. n0+7 and two k-steps: b[0], b[1] at k0,
+// b[2], b[3] at k0 + 8.
+__device__ __forceinline__ void ldb2(uint32_t (&b)[4], const float* X, int ld, int n0, int k0, int lane) {
+  ldsm_x4(b, smem_u32(X + (n0 + (lane & 7)) * ld + k0 + 4 * (lane >> 3)));
 }
-__device__ __forceinline__ void frag_bt_raw(uint32_t& b0, uint32_t& b1, const float* X, int ld, int n0, int k0,
-                                            int gid, int tig) {
-  b0 = __float_as_uint(X[(n0 + gid) * ld + k0 + tig]);
-  b1 = __float_as_uint(X[(n0 + gid) * ld + k0 + tig + 4]);
+template <int N>
+__device__ __forceinline__ void round_tf32(uint32_t (&r)[N]) {
+#pragma unroll
+  for (int i = 0; i < N; ++i) r[i] = tf32(__uint_as_float(r[i]));
 }
-__device__ __forceinline__ void frag_at_raw(uint32_t (&a)[4], const float* X, int ld, int m0, int k0, int gid,
-                                            int tig) {
-  a[0] = __float_as_uint(X[(k0 + tig) * ld + m0 + gid]);
-  a[1] = __float_as_uint(X[(k0 + tig) * ld + m0 + gid + 8]);
-  a[2] = __float_as_uint(X[(k0 + tig + 4) * ld + m0 + gid]);
-  a[3] = __float_as_uint(X[(k0 + tig + 4) * ld + m0 + gid + 8]);
-}
-__device__ __forceinline__ void frag_b_raw(uint32_t& b0, uint32_t& b1, const float* X, int ld, int n0, int k0,
-                                           int gid, int tig) {
-  b0 = __float_as_uint(X[(k0 + tig) * ld + n0 + gid]);
-  b1 = __float_as_uint(X[(k0 + tig + 4) * ld + n0 + gid]);
-}
-// B[k][n] = s[k] X[k][n] (X stored with k as the row).
+// B[k][n] = s[k] X[k][n] (X stored with k as the row), rounded to TF32.
 __device__ __forceinline__ void frag_b(uint32_t& b0, uint32_t& b1, const float* X, int ld, const float* s, int n0,
                                        int k0, int gid, int tig) {
-  const float s0 = s ? s[k0 + tig] : 1.0f, s1 = s ? s[k0 + tig + 4] : 1.0f;
-  b0 = tf32(s0 * X[(k0 + tig) * ld + n0 + gid]);
-  b1 = tf32(s1 * X[(k0 + tig + 4) * ld + n0 + gid]);
+  b0 = tf32(s[k0 + tig] * X[(k0 + tig) * ld + n0 + gid]);
+  b1 = tf32(s[k0 + tig + 4] * X[(k0 + tig + 4) * ld + n0 + gid]);
 }
 
 // 16 consecutive elements (BF16 or F32) -> FP32.
@@ -182,11 +177,11 @@ __device__ __forceinline__ void load16(const uint8_t* p, float (&f)[16]) {
 }
 
 struct PrepSmem {
-  float q[C * LD64];   // q^ (normalised and scaled)
-  float k[C * LD64];   // k^
-  float al[C * LD64];  // A, then L, then W
-  float p[C * LD64];   // P
-  float v[C * LD128];  // V, then U~
+  float q[C * LD64];   // q^ rows (normalised and scaled), FP32
+  float k[C * LD64];   // k^ rows, FP32; from step 3 on K_d^T [d_k][token] (TF32)
+  float al[C * LD64];  // A, then L (TF32), then W^T [d_k][token] (TF32)
+  float p[C * LD64];   // P (TF32)
+  float vt[DV * LD64]; // (diag(beta) V)^T [value][token] (TF32), then U~^T
   float gam[C];        // inclusive running sum of g
   float beta[C];
   float bg[C];         // beta e^gam
@@ -196,6 +191,9 @@ struct PrepSmem {
 };
 
 // One CTA per (chunk, value head): the S-independent matrices of the chunk.
+// Every operand fragment is read with ldmatrix from a row-major tile, so the
+// matrices that are contracted over tokens (W, U~, K_d, diag(beta) V) are kept
+// transposed, token index along the row.
 template <int DTYPE>
 __global__ void __launch_bounds__(kThreads, 2) gdn_prep_kernel(const __grid_constant__ GdnArgs a) {
   extern __shared__ __align__(16) uint8_t smem_raw[];
@@ -209,11 +207,15 @@ __global__ void __launch_bounds__(kThreads, 2) gdn_prep_kernel(const __grid_cons
   grid_dependency_wait();
   if (tid == 0) grid_launch_dependents();
 
-  // ---- q, k rows: four threads per row, 16 elements each; L2 norms in FP32
   {
+    // q, k rows: four threads per row, 16 elements each.  v: one token per
+    // lane, 32 consecutive values per thread (so the transposed writes below
+    // are conflict-free).  Every load is issued before any is used.
     const int row = tid >> 2, part = tid & 3;
     const int64_t t = t0 + row;
-    float fq[16], fk[16];
+    const int vrow = lane + 32 * (warp & 1), vcol = 32 * (warp >> 1);
+    const int64_t tv = t0 + vrow;
+    float fq[16], fk[16], fv[2][16], bv = 0.0f;
     if (t < a.T) {
       load16<DTYPE>(a.q + t * a.ld_q + (static_cast<int64_t>(hq) * DK + part * 16) * kEsz, fq);
       load16<DTYPE>(a.k + t * a.ld_k + (static_cast<int64_t>(hq) * DK + part * 16) * kEsz, fk);
@@ -221,6 +223,16 @@ __global__ void __launch_bounds__(kThreads, 2) gdn_prep_kernel(const __grid_cons
 #pragma unroll
       for (int i = 0; i < 16; ++i) fq[i] = fk[i] = 0.0f;
     }
+    if (tv < a.T) {
+      const uint8_t* src = a.v + tv * a.ld_v + (static_cast<int64_t>(h) * DV + vcol) * kEsz;
+      load16<DTYPE>(src, fv[0]);
+      load16<DTYPE>(src + 16 * kEsz, fv[1]);
+      bv = a.beta[tv * a.ld_beta + h];
+    } else {
+#pragma unroll
+      for (int i = 0; i < 16; ++i) fv[0][i] = fv[1][i] = 0.0f;
+    }
+    // L2 norms in FP32
     float sq = 0.0f, sk = 0.0f;
 #pragma unroll
     for (int i = 0; i < 16; ++i) {
@@ -239,21 +251,12 @@ __global__ void __launch_bounds__(kThreads, 2) gdn_prep_kernel(const __grid_cons
       *reinterpret_cast<float4*>(&s.k[row * LD64 + part * 16 + i]) =
           make_float4(fk[i] * ik, fk[i + 1] * ik, fk[i + 2] * ik, fk[i + 3] * ik);
     }
-    // ---- v rows: 32 elements per thread
-    float fv[16];
+    // V is read only as diag(beta) V, a TF32 operand: scaled, rounded and
+    // transposed here once
 #pragma unroll
-    for (int hh = 0; hh < 2; ++hh) {
-      const int col = part * 32 + hh * 16;
-      if (t < a.T) {
-        load16<DTYPE>(a.v + t * a.ld_v + (static_cast<int64_t>(h) * DV + col) * kEsz, fv);
-      } else {
+    for (int hh = 0; hh < 2; ++hh)
 #pragma unroll
-        for (int i = 0; i < 16; ++i) fv[i] = 0.0f;
-      }
-#pragma unroll
-      for (int i = 0; i < 16; i += 4)
-        *reinterpret_cast<float4*>(&s.v[row * LD128 + col + i]) = make_float4(fv[i], fv[i + 1], fv[i + 2], fv[i + 3]);
-    }
+      for (int i = 0; i < 16; ++i) s.vt[(vcol + 16 * hh + i) * LD64 + vrow] = __uint_as_float(tf32(bv * fv[hh][i]));
   }
   // ---- gates: running sum of the log decay inside the chunk (warp 0)
   if (warp == 0) {
@@ -286,41 +289,51 @@ __global__ void __launch_bounds__(kThreads, 2) gdn_prep_kernel(const __grid_cons
   }
   __syncthreads();
 
-  // ---- step 1: Gram matrices K K^T (-> A) and Q K^T (-> P), lower triangle
+  // ---- step 1: Gram matrices K K^T (-> A) and Q K^T (-> P), lower triangle.
+  // The 20 tiles (mt, nt) with nt <= 2 mt + 1 of each matrix go five to a
+  // warp: w = warp % 4 takes row block 3 (w < 2) or 2 with half of its tiles,
+  // then row block 0 or 1 with half of its tiles.
   {
-    const int mat = warp >> 2, mt = warp & 3;
+    const int mat = warp >> 2, w4 = warp & 3;
     const float* X = mat == 0 ? s.k : s.q;
     float* out = mat == 0 ? s.al : s.p;
-    uint32_t af[8][4];
+    const int mt_big = w4 < 2 ? 3 : 2, mt_small = 3 - mt_big;
+    const int n_big = mt_big + 1, n_small = mt_small + 1;  // tiles per warp in each row block
+#pragma unroll 1
+    for (int seg = 0; seg < 2; ++seg) {
+      const int mt = seg ? mt_small : mt_big;
+      const int cnt = seg ? n_small : n_big;
+      const int nt0 = (w4 & 1) * cnt;
+      uint32_t af[8][4];
 #pragma unroll
-    for (int ks = 0; ks < 8; ++ks) frag_a(af[ks], X, LD64, 16 * mt, 8 * ks, gid, tig);
-    for (int nt = 0; nt < 8; ++nt) {
-      float d[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-      if (nt < 2 * mt + 2) {
+      for (int ks = 0; ks < 8; ++ks) {
+        lda(af[ks], X, LD64, 16 * mt, 8 * ks, lane);
+        round_tf32(af[ks]);
+      }
+#pragma unroll 1
+      for (int nt = nt0; nt < nt0 + cnt; ++nt) {
+        float d[4] = {0.0f, 0.0f, 0.0f, 0.0f};
 #pragma unroll
-        for (int ks = 0; ks < 8; ++ks) {
-          uint32_t b0, b1;
-          frag_bt(b0, b1, s.k, LD64, 8 * nt, 8 * ks, gid, tig);
-          mma(d, af[ks], b0, b1);
+        for (int kp = 0; kp < 4; ++kp) {
+          uint32_t b[4];
+          ldb2(b, s.k, LD64, 8 * nt, 16 * kp, lane);
+          round_tf32(b);
+          mma(d, af[2 * kp], b[0], b[1]);
+          mma(d, af[2 * kp + 1], b[2], b[3]);
+        }
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int t = 16 * mt + gid + (e >= 2 ? 8 : 0), j = 8 * nt + 2 * tig + (e & 1);
+          float val = 0.0f;
+          if (mat == 0) {
+            if (j < t) val = s.beta[t] * __expf(s.gam[t] - s.gam[j]) * d[e];
+          } else {
+            // P is read only as a TF32 MMA operand: rounded here once
+            if (j <= t) val = __uint_as_float(tf32(__expf(s.gam[t] - s.gam[j]) * d[e]));
+          }
+          out[t * LD64 + j] = val;
         }
       }
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int t = 16 * mt + gid + (e >= 2 ? 8 : 0), j = 8 * nt + 2 * tig + (e & 1);
-        float val = 0.0f;
-        if (mat == 0) {
-          if (j < t) val = s.beta[t] * __expf(s.gam[t] - s.gam[j]) * d[e];
-        } else {
-          // P is read only as a TF32 MMA operand: rounded here once
-          if (j <= t) val = __uint_as_float(tf32(__expf(s.gam[t] - s.gam[j]) * d[e]));
-        }
-        out[t * LD64 + j] = val;
-      }
-    }
-    // V is read only as diag(beta) V, a TF32 operand: scale and round it in place
-    for (int idx = tid; idx < C * DV; idx += kThreads) {
-      const int j = idx >> 7, n = idx & 127;
-      s.v[j * LD128 + n] = __uint_as_float(tf32(s.beta[j] * s.v[j * LD128 + n]));
     }
   }
   __syncthreads();
@@ -423,75 +436,107 @@ __global__ void __launch_bounds__(kThreads, 2) gdn_prep_kernel(const __grid_cons
   }
   __syncthreads();
 
-  // ---- step 3: W = L diag(beta e^gam) K  and  U~ = L diag(beta) V
+  // ---- step 3: W = L diag(beta e^gam) K  and  U~ = L diag(beta) V.
+  // 24 column tiles (0-7: W, 8-23: U~) x 4 row blocks, 2 mt + 2 k-steps each
+  // (L is lower triangular).  Warp w takes column tiles 6 (w % 4) .. +5 of row
+  // blocks 3 and 0 (w < 4) or 2 and 1: 60 k-steps for every warp, and the two
+  // row blocks share each B fragment.
   {
-    const int mt = warp & 3, half = warp >> 2;
-    const int nks = 2 * mt + 2;  // L is lower triangular: k-steps past the diagonal block are zero
-    uint32_t af[8][4];
+    const int mt_big = warp < 4 ? 3 : 2, mt_small = 3 - mt_big;
+    const int nkb = 2 * mt_big + 2, nks = 2 * mt_small + 2;
+    const int ntb = 6 * (warp & 3);
+    float db[6][4], ds[6][4];
 #pragma unroll
-    for (int ks = 0; ks < 8; ++ks)
-      if (ks < nks) frag_a_raw(af[ks], s.al, LD64, 16 * mt, 8 * ks, gid, tig);
-    float d[12][4];
+    for (int i = 0; i < 6; ++i)
 #pragma unroll
-    for (int i = 0; i < 12; ++i) d[i][0] = d[i][1] = d[i][2] = d[i][3] = 0.0f;
+      for (int e = 0; e < 4; ++e) db[i][e] = ds[i][e] = 0.0f;
+    // k-step pairs outermost: only two A fragments of each row block are live
 #pragma unroll
-    for (int i = 0; i < 12; ++i) {
-      const int nt = half * 12 + i;  // 0..7: W columns, 8..23: U~ columns
+    for (int kp = 0; kp < 4; ++kp) {
+      if (2 * kp >= nkb) continue;
+      const bool small = 2 * kp < nks;
+      uint32_t ab0[4], ab1[4], as0[4], as1[4];
+      lda(ab0, s.al, LD64, 16 * mt_big, 16 * kp, lane);
+      lda(ab1, s.al, LD64, 16 * mt_big, 16 * kp + 8, lane);
+      if (small) {
+        lda(as0, s.al, LD64, 16 * mt_small, 16 * kp, lane);
+        lda(as1, s.al, LD64, 16 * mt_small, 16 * kp + 8, lane);
+      }
 #pragma unroll
-      for (int ks = 0; ks < 8; ++ks) {
-        if (ks >= nks) continue;
-        uint32_t b0, b1;
-        if (nt < 8) frag_b(b0, b1, s.k, LD64, s.bg, 8 * nt, 8 * ks, gid, tig);
-        else frag_b_raw(b0, b1, s.v, LD128, 8 * (nt - 8), 8 * ks, gid, tig);
-        mma(d[i], af[ks], b0, b1);
+      for (int i = 0; i < 6; ++i) {
+        const int nt = ntb + i;
+        uint32_t b[4];
+        if (nt < 8) {
+          frag_b(b[0], b[1], s.k, LD64, s.bg, 8 * nt, 16 * kp, gid, tig);
+          frag_b(b[2], b[3], s.k, LD64, s.bg, 8 * nt, 16 * kp + 8, gid, tig);
+        } else {
+          ldb2(b, s.vt, LD64, 8 * (nt - 8), 16 * kp, lane);
+        }
+        mma(db[i], ab0, b[0], b[1]);
+        mma(db[i], ab1, b[2], b[3]);
+        if (small) {
+          mma(ds[i], as0, b[0], b[1]);
+          mma(ds[i], as1, b[2], b[3]);
+        }
       }
     }
-    __syncthreads();  // L, V and K are read; W goes over L, U~ over V, K_d over K
-    // W and U~ are read only as TF32 operands: rounded here once
+    // K for K_d, read before the barrier (token j = idx % 64, column n = idx / 64)
+    float kr[16];
 #pragma unroll
-    for (int i = 0; i < 12; ++i) {
-      const int nt = half * 12 + i;
-      const int r = 16 * mt + gid;
-      float* dst = nt < 8 ? &s.al[r * LD64 + 8 * nt + 2 * tig] : &s.v[r * LD128 + 8 * (nt - 8) + 2 * tig];
-      const int ld = nt < 8 ? LD64 : LD128;
-      *reinterpret_cast<float2*>(dst) = make_float2(__uint_as_float(tf32(d[i][0])), __uint_as_float(tf32(d[i][1])));
-      *reinterpret_cast<float2*>(dst + 8 * ld) =
-          make_float2(__uint_as_float(tf32(d[i][2])), __uint_as_float(tf32(d[i][3])));
+    for (int e = 0; e < 16; ++e) {
+      const int idx = tid + e * kThreads;
+      kr[e] = s.k[(idx & 63) * LD64 + (idx >> 6)];
     }
-    // from here on K is read only as K_d = diag(e^(gam_C - gam)) K, a TF32 operand
-    for (int idx = tid; idx < C * DK; idx += kThreads) {
-      const int j = idx >> 6, n = idx & 63;
-      s.k[j * LD64 + n] = __uint_as_float(tf32(s.kdec[j] * s.k[j * LD64 + n]));
+    __syncthreads();  // L, V and K are read; W^T goes over L, U~^T over V^T, K_d^T over K
+    // W and U~ are read only as TF32 operands: rounded here once, stored transposed
+#pragma unroll
+    for (int i = 0; i < 6; ++i) {
+      const int nt = ntb + i;
+      float* dst = nt < 8 ? &s.al[(8 * nt + 2 * tig) * LD64] : &s.vt[(8 * (nt - 8) + 2 * tig) * LD64];
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        const float(&d)[4] = half ? ds[i] : db[i];
+        const int r = 16 * (half ? mt_small : mt_big) + gid;
+        dst[r] = __uint_as_float(tf32(d[0]));
+        dst[LD64 + r] = __uint_as_float(tf32(d[1]));
+        dst[r + 8] = __uint_as_float(tf32(d[2]));
+        dst[LD64 + r + 8] = __uint_as_float(tf32(d[3]));
+      }
+    }
+    // from here on K is read only as K_d^T = (diag(e^(gam_C - gam)) K)^T, a TF32 operand
+#pragma unroll
+    for (int e = 0; e < 16; ++e) {
+      const int idx = tid + e * kThreads, j = idx & 63;
+      s.k[(idx >> 6) * LD64 + j] = __uint_as_float(tf32(s.kdec[j] * kr[e]));
     }
   }
   __syncthreads();
 
-  // ---- step 4: the record: [M^T; R] (128 x 64), N (128 x 64), Y^T (128 x 64)
+  // ---- step 4: the record: [M^T; R] (128 x 64), N (128 x 64), Y^T (128 x 64),
+  // rows swizzled (sw64)
   float* rec = a.ws + (static_cast<int64_t>(c) * a.H + h) * kRec;
   {
     const float eC = s.eg[C - 1];
-    // M^T (warps 0-3) or R (warps 4-7): 16 rows each
+    // M^T = e^gam_C I - K_d^T W (warps 0-3) or R = diag(e^gam) Q - P W (warps 4-7): 16 rows each
     {
       const bool is_r = warp >= 4;
       const int mt = warp & 3;
       const int nks = is_r ? 2 * mt + 2 : 8;  // P is lower triangular
       uint32_t af[8][4];
 #pragma unroll
-      for (int ks = 0; ks < 8; ++ks) {
-        if (ks >= nks) continue;
-        if (is_r) frag_a_raw(af[ks], s.p, LD64, 16 * mt, 8 * ks, gid, tig);
-        else frag_at_raw(af[ks], s.k, LD64, 16 * mt, 8 * ks, gid, tig);
-      }
+      for (int ks = 0; ks < 8; ++ks)
+        if (ks < nks) lda(af[ks], is_r ? s.p : s.k, LD64, 16 * mt, 8 * ks, lane);
       float* dst = rec + (is_r ? 64 : 0) * 64;
 #pragma unroll
       for (int nt = 0; nt < 8; ++nt) {
         float d[4] = {0.0f, 0.0f, 0.0f, 0.0f};
 #pragma unroll
-        for (int ks = 0; ks < 8; ++ks) {
-          if (ks >= nks) continue;
-          uint32_t b0, b1;
-          frag_b_raw(b0, b1, s.al, LD64, 8 * nt, 8 * ks, gid, tig);
-          mma(d, af[ks], b0, b1);
+        for (int kp = 0; kp < 4; ++kp) {
+          if (2 * kp >= nks) continue;
+          uint32_t b[4];
+          ldb2(b, s.al, LD64, 8 * nt, 16 * kp, lane);
+          mma(d, af[2 * kp], b[0], b[1]);
+          mma(d, af[2 * kp + 1], b[2], b[3]);
         }
 #pragma unroll
         for (int hh = 0; hh < 2; ++hh) {
@@ -505,71 +550,51 @@ __global__ void __launch_bounds__(kThreads, 2) gdn_prep_kernel(const __grid_cons
             v1 = (r == col + 1 ? eC : 0.0f) - d[2 * hh + 1];
           }
           // rounded here once: the state pass reads these rows only as TF32 MMA operands
-          *reinterpret_cast<float2*>(dst + r * 64 + col) =
+          *reinterpret_cast<float2*>(dst + sw64(r, col)) =
               make_float2(__uint_as_float(tf32(v0)), __uint_as_float(tf32(v1)));
         }
       }
     }
-    // N = U~^T Kd and Y^T = U~^T P^T: rows 16*warp .. +16 of both
+    // N = U~^T K_d and Y^T = U~^T P^T: rows 16*warp .. +16 of both
     {
       const int mt = warp;
       uint32_t af[8][4];
 #pragma unroll
-      for (int ks = 0; ks < 8; ++ks) frag_at_raw(af[ks], s.v, LD128, 16 * mt, 8 * ks, gid, tig);
+      for (int ks = 0; ks < 8; ++ks) lda(af[ks], s.vt, LD64, 16 * mt, 8 * ks, lane);
 #pragma unroll
       for (int nt = 0; nt < 16; ++nt) {
         const bool is_y = nt >= 8;
         const int n0 = 8 * (nt & 7);
         float d[4] = {0.0f, 0.0f, 0.0f, 0.0f};
 #pragma unroll
-        for (int ks = 0; ks < 8; ++ks) {
-          if (is_y && ks > (nt & 7)) continue;  // P[t][j] = 0 for j > t
-          uint32_t b0, b1;
-          if (is_y) frag_bt_raw(b0, b1, s.p, LD64, n0, 8 * ks, gid, tig);
-          else frag_b_raw(b0, b1, s.k, LD64, n0, 8 * ks, gid, tig);
-          mma(d, af[ks], b0, b1);
+        for (int kp = 0; kp < 4; ++kp) {
+          if (is_y && 2 * kp > (nt & 7)) continue;  // P[t][j] = 0 for j > t
+          uint32_t b[4];
+          ldb2(b, is_y ? s.p : s.k, LD64, n0, 16 * kp, lane);
+          mma(d, af[2 * kp], b[0], b[1]);
+          if (!is_y || 2 * kp + 1 <= (nt & 7)) mma(d, af[2 * kp + 1], b[2], b[3]);
         }
         float* dst = rec + (is_y ? 2 : 1) * 128 * 64;
         const int r = 16 * mt + gid, col = n0 + 2 * tig;
-        *reinterpret_cast<float2*>(dst + r * 64 + col) = make_float2(d[0], d[1]);
-        *reinterpret_cast<float2*>(dst + (r + 8) * 64 + col) = make_float2(d[2], d[3]);
+        *reinterpret_cast<float2*>(dst + sw64(r, col)) = make_float2(d[0], d[1]);
+        *reinterpret_cast<float2*>(dst + sw64(r + 8, col)) = make_float2(d[2], d[3]);
       }
     }
   }
 }
 
 constexpr int kBufs = 3;  // record buffers of the state pass
+// floats of one record buffer of the state pass: [M^T; R] (128 rows), then
+// this CTA's 32 rows of N and of Y^T
+constexpr int kRecCta = (128 + 2 * kRows) * 64;
 
 struct StateSmem {
-  float bc[kBufs][128 * LD64];    // [M^T; R] (TF32 values)
-  float nn[kBufs][kRows * LD64];  // N rows of this CTA
-  float yt[kBufs][kRows * LD64];  // Y^T rows of this CTA
-  float st[2][kRows * LD64];      // the state rows, current and next (TF32 values but the last)
-  float os[2][C * 36];            // output staging [t][i], two chunks
+  float rec[kBufs][kRecCta];  // swizzled rows, as stored by the per-chunk pass
+  float st[2][kRows * 64];    // the state rows, current and next (TF32 values but the last), swizzled
+  float os[2][C * 36];        // output staging [t][i], two chunks
+  uint64_t full[kBufs];
+  int abort_flag;
 };
-
-__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-__device__ __forceinline__ void cp_async_wait_1() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
-__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
-
-__device__ __forceinline__ void load_record(StateSmem& s, int buf, const float* rec, int i0, int tid) {
-  for (int idx = tid; idx < 3072; idx += kThreads) {
-    const int c16 = idx & 15;
-    if (idx < 2048) {
-      const int r = idx >> 4;
-      cp_async16(&s.bc[buf][r * LD64 + 4 * c16], rec + r * 64 + 4 * c16);
-    } else if (idx < 2560) {
-      const int r = (idx - 2048) >> 4;
-      cp_async16(&s.nn[buf][r * LD64 + 4 * c16], rec + 128 * 64 + (i0 + r) * 64 + 4 * c16);
-    } else {
-      const int r = (idx - 2560) >> 4;
-      cp_async16(&s.yt[buf][r * LD64 + 4 * c16], rec + 2 * 128 * 64 + (i0 + r) * 64 + 4 * c16);
-    }
-  }
-}
 
 // O rows of chunk c from the staging buffer: 64 tokens x 32 values, 8 per thread.
 __device__ __forceinline__ void store_out(const GdnArgs& a, const float* os, int c, int h, int i0, int tid) {
@@ -595,45 +620,72 @@ __device__ __forceinline__ void store_out(const GdnArgs& a, const float* os, int
 }
 
 // One CTA per (value head, 32 state rows): the chunks in order, one block
-// barrier per chunk.  Chunk c's record lands in buffer c % 3 (requested two
-// chunks ahead); its output goes out from the staging buffer during chunk c + 1.
+// barrier per chunk.  Chunk c's record (the shared [M^T; R] and this CTA's rows
+// of N and Y^T, three bulk copies) lands in buffer c % 3, requested two chunks
+// ahead; its output goes out from the staging buffer during chunk c + 1.
+// Fragments come from shared memory with ldmatrix: the records and the state
+// rows are swizzled (sw64), so the loads are free of bank conflicts.
 __global__ void __launch_bounds__(kThreads, 1) gdn_state_kernel(const __grid_constant__ GdnArgs a) {
   extern __shared__ __align__(16) uint8_t smem_raw[];
   StateSmem& s = *reinterpret_cast<StateSmem*>(smem_raw);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int gid = lane >> 2, tig = lane & 3;
   const int h = blockIdx.x, i0 = blockIdx.y * kRows;
+  volatile int* abort_flag = &s.abort_flag;
 
+  if (tid == 0) {
+    for (int b = 0; b < kBufs; ++b) mbar_init(&s.full[b], 1);
+    s.abort_flag = 0;
+    fence_mbarrier_init();
+  }
+  __syncthreads();
   grid_dependency_wait();
   if (tid == 0) grid_launch_dependents();
 
-  auto rec_of = [&](int c) { return a.ws + (static_cast<int64_t>(c) * a.H + h) * kRec; };
-  load_record(s, 0, rec_of(0), i0, tid);
-  cp_async_commit();
-  if (a.nchunks > 1) load_record(s, 1, rec_of(1), i0, tid);
-  cp_async_commit();
+  auto issue = [&](int c) {  // thread 0 only
+    const int b = c % kBufs;
+    const float* rec = a.ws + (static_cast<int64_t>(c) * a.H + h) * kRec;
+    mbar_arrive_expect_tx(&s.full[b], kRecCta * 4);
+    bulk_load(s.rec[b], rec, 128 * 64 * 4, &s.full[b]);
+    bulk_load(s.rec[b] + 128 * 64, rec + 128 * 64 + i0 * 64, kRows * 64 * 4, &s.full[b]);
+    bulk_load(s.rec[b] + (128 + kRows) * 64, rec + 256 * 64 + i0 * 64, kRows * 64 * 4, &s.full[b]);
+  };
+  if (tid == 0) {
+    if (a.nchunks > 0) issue(0);
+    if (a.nchunks > 1) issue(1);
+  }
   // entering state, as the TF32 operand it is used as
   for (int idx = tid; idx < kRows * DK; idx += kThreads) {
     const int r = idx / DK, col = idx % DK;
     const float v = a.h0 ? a.h0[(static_cast<int64_t>(h) * DV + i0 + r) * DK + col] : 0.0f;
-    s.st[0][r * LD64 + col] = __uint_as_float(tf32(v));
+    s.st[0][sw64(r, col)] = __uint_as_float(tf32(v));
   }
-  int cur = 0;
-  for (int c = 0; c < a.nchunks; ++c) {
+  // this lane's rows and pieces for ldmatrix: A (state) rows rr + 8 (j & 1),
+  // piece 2 ks + (j >> 1); B ([M^T; R]) rows rr + 8 (j >> 1), piece 2 ks + (j & 1)
+  const int rr = lane & 7, jm = lane >> 3;
+  const int a_row = rr + 8 * (jm & 1), a_pc = jm >> 1;
+  const int nbase = 16 * warp;  // warps 0-3: state columns, 4-7: tokens
+  const int b_row = nbase + rr + 8 * (jm >> 1), b_pc = jm & 1;
+  int cur = 0, c = 0;
+  for (; c < a.nchunks; ++c) {
     const int buf = c % kBufs;
-    cp_async_wait_1();
-    __syncthreads();
+    const bool ok = mbar_wait_bounded(&s.full[buf], static_cast<uint32_t>(c / kBufs) & 1u, abort_flag);
+    if (__syncthreads_or(!ok)) break;  // a copy did not arrive in time: every thread stops
     // buffer (c + 2) % 3 was last read during chunk c - 1
-    if (c + 2 < a.nchunks) load_record(s, (c + 2) % kBufs, rec_of(c + 2), i0, tid);
-    cp_async_commit();
+    if (tid == 0 && c + 2 < a.nchunks) issue(c + 2);
     if (c > 0) store_out(a, s.os[(c - 1) & 1], c - 1, h, i0, tid);
+    const float* bc = s.rec[buf];
+    const float* nn = bc + 128 * 64;
+    const float* yt = bc + (128 + kRows) * 64;
     // D[i][n] = sum_k S[i][k] Bc[n][k]: n < 64 -> (S M)[i][n], n >= 64 -> (S R^T)[i][t = n - 64]
     {
+      const uint32_t st_u = smem_u32(s.st[cur]), bc_u = smem_u32(bc);
       uint32_t af[2][8][4];
 #pragma unroll
       for (int mt = 0; mt < 2; ++mt)
 #pragma unroll
-        for (int ks = 0; ks < 8; ++ks) frag_a_raw(af[mt][ks], s.st[cur], LD64, 16 * mt, 8 * ks, gid, tig);
+        for (int ks = 0; ks < 8; ++ks)
+          ldsm_x4(af[mt][ks], st_u + (16 * mt + a_row) * 256 + (((2 * ks + a_pc) ^ rr) << 4));
       // two accumulators per tile (even and odd k-steps) halve the dependent MMA chain
       float d[2][2][4], d2[2][2][4];
 #pragma unroll
@@ -642,16 +694,16 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_state_kernel(const __grid_con
         for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
           for (int e = 0; e < 4; ++e) d[mt][nt][e] = d2[mt][nt][e] = 0.0f;
-      const int nbase = 16 * warp;  // warps 0-3: state columns, 4-7: tokens
 #pragma unroll
-      for (int ks = 0; ks < 8; ++ks)
+      for (int ks = 0; ks < 8; ++ks) {
+        uint32_t bq[4];  // b0, b1 of columns nbase .. +7, then of nbase + 8 .. +15
+        ldsm_x4(bq, bc_u + b_row * 256 + (((2 * ks + b_pc) ^ rr) << 4));
 #pragma unroll
         for (int nt = 0; nt < 2; ++nt) {
-          uint32_t b0, b1;
-          frag_bt_raw(b0, b1, s.bc[buf], LD64, nbase + 8 * nt, 8 * ks, gid, tig);
-          mma((ks & 1) ? d2[0][nt] : d[0][nt], af[0][ks], b0, b1);
-          mma((ks & 1) ? d2[1][nt] : d[1][nt], af[1][ks], b0, b1);
+          mma((ks & 1) ? d2[0][nt] : d[0][nt], af[0][ks], bq[2 * nt], bq[2 * nt + 1]);
+          mma((ks & 1) ? d2[1][nt] : d[1][nt], af[1][ks], bq[2 * nt], bq[2 * nt + 1]);
         }
+      }
 #pragma unroll
       for (int mt = 0; mt < 2; ++mt)
 #pragma unroll
@@ -668,13 +720,13 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_state_kernel(const __grid_con
 #pragma unroll
             for (int hh = 0; hh < 2; ++hh) {
               const int r = 16 * mt + gid + 8 * hh, col = nbase + 8 * nt + 2 * tig;
-              const float2 n2 = *reinterpret_cast<const float2*>(&s.nn[buf][r * LD64 + col]);
+              const float2 n2 = *reinterpret_cast<const float2*>(&nn[sw64(r, col)]);
               float v0 = d[mt][nt][2 * hh] + n2.x, v1 = d[mt][nt][2 * hh + 1] + n2.y;
               if (!last) {
                 v0 = __uint_as_float(tf32(v0));
                 v1 = __uint_as_float(tf32(v1));
               }
-              *reinterpret_cast<float2*>(&s.st[cur ^ 1][r * LD64 + col]) = make_float2(v0, v1);
+              *reinterpret_cast<float2*>(&s.st[cur ^ 1][sw64(r, col)]) = make_float2(v0, v1);
             }
       } else {
         float* os = s.os[c & 1];
@@ -683,22 +735,31 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_state_kernel(const __grid_con
 #pragma unroll
           for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const int r = 16 * mt + gid + (e >= 2 ? 8 : 0);
-              const int t = nbase - 64 + 8 * nt + 2 * tig + (e & 1);
-              os[t * 36 + r] = d[mt][nt][e] + s.yt[buf][r * LD64 + t];
+            for (int hh = 0; hh < 2; ++hh) {
+              const int r = 16 * mt + gid + 8 * hh;
+              const int t = nbase - 64 + 8 * nt + 2 * tig;
+              const float2 y2 = *reinterpret_cast<const float2*>(&yt[sw64(r, t)]);
+              os[t * 36 + r] = d[mt][nt][2 * hh] + y2.x;
+              os[(t + 1) * 36 + r] = d[mt][nt][2 * hh + 1] + y2.y;
             }
       }
     }
     cur ^= 1;
   }
-  cp_async_wait_all();
+  if (c < a.nchunks) {
+    // a record copy did not arrive in time (the error word is set): wait, with
+    // a limit, for the copies still in flight into this CTA's buffers, then stop
+    if (tid == 0)
+      for (int cc = c; cc < a.nchunks && cc < c + 2; ++cc)
+        mbar_wait_bounded(&s.full[cc % kBufs], static_cast<uint32_t>(cc / kBufs) & 1u, nullptr);
+    return;
+  }
   __syncthreads();
   if (a.nchunks > 0) store_out(a, s.os[(a.nchunks - 1) & 1], a.nchunks - 1, h, i0, tid);
   if (a.h_out) {
     for (int idx = tid; idx < kRows * DK; idx += kThreads) {
       const int r = idx / DK, col = idx % DK;
-      a.h_out[(static_cast<int64_t>(h) * DV + i0 + r) * DK + col] = s.st[cur][r * LD64 + col];
+      a.h_out[(static_cast<int64_t>(h) * DV + i0 + r) * DK + col] = s.st[cur][sw64(r, col)];
     }
   }
 }
