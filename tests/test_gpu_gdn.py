@@ -6,12 +6,13 @@ state in FP32; the triangular inverse is FP32 substitution plus 3xTF32 block
 products (about FP32).  A rounded product sum_k a_k b_k is off by at most
 2^-10 sum_k |a_k b_k|; between the inputs and an output sit four such
 products in sequence (W and U~ through L, then M, N, R and Y, then S M and
-S R^T), each amplified by at most |L| = |(I + A)^-1|, which stays below 4 for
-unit keys and beta in [0, 1] on these inputs.  So every output is held to
-    |o_gpu - o| <= 2^-6 |S_t[i, :]|_2 |q_t|_2,
+S R^T), each amplified by at most |L| = |(I + A)^-1|, which stays below 2 for
+unit keys and beta in [0, 1] on these inputs (checked on CPU for every chunk
+of every case here; the largest value is 1.64).  So every output is held to
+    |o_gpu - o| <= 4 * 2 * 2^-10 |S_t[i, :]|_2 |q_t|_2 = 2^-7 |S_t[i, :]|_2 |q_t|_2,
 the right-hand side being the natural size of o_t[i] (|o_t[i]| <= |S_t[i,:]| |q_t|),
 plus half a BF16 ulp for BF16 outputs; the final state to
-|S_gpu - S| <= 2^-6 |S[i, :]|_2 per row.  The largest error / bound ratio is
+|S_gpu - S| <= 2^-7 |S[i, :]|_2 per row.  The largest error / bound ratio is
 printed for every case.
 """
 import numpy as np
@@ -24,7 +25,7 @@ from oracle import nvfp4_oracle as o
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda:0"
-TAU = 2.0 ** -6
+TAU = 2.0 ** -7
 DK, DV = 64, 128
 
 
