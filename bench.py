@@ -39,10 +39,10 @@ ROTATE = 4          # rotating input sets so consecutive steps miss in L2
 # commands are in profiles/); an entry is removed when its kernel changes,
 # until it is captured again.  "quant": both passes, captured on X[8192, 17408]
 # and scaled by 4 rows-wise (the traffic grows with the rows).  "gdnrec": both
-# recurrence launches, captured at 8192 tokens and scaled by 4 (all of it is per chunk).
+# recurrence launches, captured at full length (one pass each).
 TRAFFIC_BYTES = {
     "actstats": 339345408,
-    "gdnrec": 3817484288,
+    "gdnrec": 4052776533,
     "decode1": 50362112,
     "decode64": 50916352,
     "decode8": 50420224,

@@ -187,7 +187,7 @@ struct PrepSmem {
   float bg[C];         // beta e^gam
   float eg[C];         // e^gam
   float kdec[C];       // e^(gam_C - gam)
-  float tmp[3 * 272];  // per-warp T blocks of the triangular inverse (16 x 17 each)
+  float tmp[6 * 144];  // per-warp 16 x 8 parts of T in the triangular inverse (row stride 9)
 };
 
 // One CTA per (chunk, value head): the S-independent matrices of the chunk.
@@ -207,6 +207,20 @@ __global__ void __launch_bounds__(kThreads, 2) gdn_prep_kernel(const __grid_cons
   grid_dependency_wait();
   if (tid == 0) grid_launch_dependents();
 
+  // decay and write strength of tokens 2 lane and 2 lane + 1 (warp 0), loaded
+  // together with q, k and v
+  float ga = 0.0f, gb = 0.0f, ba = 0.0f, bb = 0.0f;
+  if (warp == 0) {
+    const int64_t ta = t0 + 2 * lane, tb = ta + 1;
+    if (ta < a.T) {
+      ga = a.g[ta * a.ld_g + h];
+      ba = a.beta[ta * a.ld_beta + h];
+    }
+    if (tb < a.T) {
+      gb = a.g[tb * a.ld_g + h];
+      bb = a.beta[tb * a.ld_beta + h];
+    }
+  }
   {
     // q, k rows: four threads per row, 16 elements each.  v: one token per
     // lane, 32 consecutive values per thread (so the transposed writes below
@@ -260,11 +274,6 @@ __global__ void __launch_bounds__(kThreads, 2) gdn_prep_kernel(const __grid_cons
   }
   // ---- gates: running sum of the log decay inside the chunk (warp 0)
   if (warp == 0) {
-    const int64_t ta = t0 + 2 * lane, tb = ta + 1;
-    const float ga = ta < a.T ? a.g[ta * a.ld_g + h] : 0.0f;
-    const float gb = tb < a.T ? a.g[tb * a.ld_g + h] : 0.0f;
-    const float ba = ta < a.T ? a.beta[ta * a.ld_beta + h] : 0.0f;
-    const float bb = tb < a.T ? a.beta[tb * a.ld_beta + h] : 0.0f;
     const float pair = ga + gb;
     float run = pair;
 #pragma unroll
@@ -291,48 +300,61 @@ __global__ void __launch_bounds__(kThreads, 2) gdn_prep_kernel(const __grid_cons
 
   // ---- step 1: Gram matrices K K^T (-> A) and Q K^T (-> P), lower triangle.
   // The 20 tiles (mt, nt) with nt <= 2 mt + 1 of each matrix go five to a
-  // warp: w = warp % 4 takes row block 3 (w < 2) or 2 with half of its tiles,
-  // then row block 0 or 1 with half of its tiles.
+  // warp: w = warp % 4 takes half of the tiles of row block 3 (w < 2) or 2,
+  // and half of those of row block 0 or 1.  The five tiles are independent
+  // accumulations, interleaved.
   {
     const int mat = warp >> 2, w4 = warp & 3;
     const float* X = mat == 0 ? s.k : s.q;
     float* out = mat == 0 ? s.al : s.p;
     const int mt_big = w4 < 2 ? 3 : 2, mt_small = 3 - mt_big;
-    const int n_big = mt_big + 1, n_small = mt_small + 1;  // tiles per warp in each row block
-#pragma unroll 1
-    for (int seg = 0; seg < 2; ++seg) {
-      const int mt = seg ? mt_small : mt_big;
-      const int cnt = seg ? n_small : n_big;
-      const int nt0 = (w4 & 1) * cnt;
-      uint32_t af[8][4];
+    const int nb = mt_big + 1;  // tiles of the big row block; 5 - nb of the small one
+    const int nb0 = (w4 & 1) * nb, ns0 = (w4 & 1) * (5 - nb);
+    float d[5][4];
 #pragma unroll
-      for (int ks = 0; ks < 8; ++ks) {
-        lda(af[ks], X, LD64, 16 * mt, 8 * ks, lane);
-        round_tf32(af[ks]);
-      }
-#pragma unroll 1
-      for (int nt = nt0; nt < nt0 + cnt; ++nt) {
-        float d[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+    for (int i = 0; i < 5; ++i) d[i][0] = d[i][1] = d[i][2] = d[i][3] = 0.0f;
 #pragma unroll
-        for (int kp = 0; kp < 4; ++kp) {
-          uint32_t b[4];
-          ldb2(b, s.k, LD64, 8 * nt, 16 * kp, lane);
-          round_tf32(b);
-          mma(d, af[2 * kp], b[0], b[1]);
-          mma(d, af[2 * kp + 1], b[2], b[3]);
-        }
+    for (int kp = 0; kp < 4; ++kp) {
+      uint32_t ab0[4], ab1[4], as0[4], as1[4];
+      lda(ab0, X, LD64, 16 * mt_big, 16 * kp, lane);
+      lda(ab1, X, LD64, 16 * mt_big, 16 * kp + 8, lane);
+      lda(as0, X, LD64, 16 * mt_small, 16 * kp, lane);
+      lda(as1, X, LD64, 16 * mt_small, 16 * kp + 8, lane);
+      round_tf32(ab0);
+      round_tf32(ab1);
+      round_tf32(as0);
+      round_tf32(as1);
+#pragma unroll
+      for (int i = 0; i < 5; ++i) {
+        const bool big = i < nb;
+        const int nt = big ? nb0 + i : ns0 + i - nb;
+        uint32_t b[4], a0[4], a1[4];
+        ldb2(b, s.k, LD64, 8 * nt, 16 * kp, lane);
+        round_tf32(b);
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          const int t = 16 * mt + gid + (e >= 2 ? 8 : 0), j = 8 * nt + 2 * tig + (e & 1);
-          float val = 0.0f;
-          if (mat == 0) {
-            if (j < t) val = s.beta[t] * __expf(s.gam[t] - s.gam[j]) * d[e];
-          } else {
-            // P is read only as a TF32 MMA operand: rounded here once
-            if (j <= t) val = __uint_as_float(tf32(__expf(s.gam[t] - s.gam[j]) * d[e]));
-          }
-          out[t * LD64 + j] = val;
+          a0[e] = big ? ab0[e] : as0[e];
+          a1[e] = big ? ab1[e] : as1[e];
         }
+        mma(d[i], a0, b[0], b[1]);
+        mma(d[i], a1, b[2], b[3]);
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < 5; ++i) {
+      const bool big = i < nb;
+      const int mt = big ? mt_big : mt_small, nt = big ? nb0 + i : ns0 + i - nb;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int t = 16 * mt + gid + (e >= 2 ? 8 : 0), j = 8 * nt + 2 * tig + (e & 1);
+        float val = 0.0f;
+        if (mat == 0) {
+          if (j < t) val = s.beta[t] * __expf(s.gam[t] - s.gam[j]) * d[i][e];
+        } else {
+          // P is read only as a TF32 MMA operand: rounded here once
+          if (j <= t) val = __uint_as_float(tf32(__expf(s.gam[t] - s.gam[j]) * d[i][e]));
+        }
+        out[t * LD64 + j] = val;
       }
     }
   }
@@ -364,59 +386,47 @@ __global__ void __launch_bounds__(kThreads, 2) gdn_prep_kernel(const __grid_cons
         if (i > jj) s.al[(base + jj) * LD64 + base + i] = col[i];
     }
     __syncthreads();
-    // Off-diagonal blocks, one block diagonal dd at a time, one warp per block
-    // (i, j) = (j + dd, j): T = sum_{m=j}^{i-1} A_im L_mj, then L_ij = -L_ii T,
-    // both 16 x 16 x 16k products on the tensor cores in 3xTF32.
+    // Off-diagonal blocks, one block diagonal dd at a time; warp w takes
+    // block (i, j) = (w / 2 + dd, w / 2) and its 8 columns 8 (w % 2) .. +7:
+    // T = sum_{m=j}^{i-1} A_im L_mj, then L_ij = -L_ii T, both on the tensor
+    // cores in 3xTF32, even and odd k-steps in separate accumulators.
     // lval(mb, j, r, c) = L[16mb + r][16j + c] (mb >= j), read from the transposed copy.
     auto lval = [&](int mb, int j, int r, int c) -> float {
       if (mb > j) return s.al[(16 * j + c) * LD64 + 16 * mb + r];
       return r > c ? s.al[(16 * j + c) * LD64 + 16 * j + r] : (r == c ? 1.0f : 0.0f);
     };
     for (int dd = 1; dd < 4; ++dd) {
-      if (warp < 4 - dd) {
-        const int j = warp, i = warp + dd;
-        float* tw = &s.tmp[warp * 272];  // this warp's T, 16 x 17
-        float t[2][4];
-#pragma unroll
-        for (int nt = 0; nt < 2; ++nt) t[nt][0] = t[nt][1] = t[nt][2] = t[nt][3] = 0.0f;
+      if (warp < 2 * (4 - dd)) {
+        const int j = warp >> 1, i = j + dd, nt = warp & 1;
+        float* tw = &s.tmp[warp * 144];  // this warp's 16 x 8 columns of T, row stride 9
+        float t[2][4] = {{0.0f, 0.0f, 0.0f, 0.0f}, {0.0f, 0.0f, 0.0f, 0.0f}};
         for (int mb = j; mb < i; ++mb) {
 #pragma unroll
           for (int kk = 0; kk < 2; ++kk) {
             const float* arow = &s.al[(16 * i) * LD64 + 16 * mb + 8 * kk];
             const float a[4] = {arow[gid * LD64 + tig], arow[(gid + 8) * LD64 + tig], arow[gid * LD64 + tig + 4],
                                 arow[(gid + 8) * LD64 + tig + 4]};
-#pragma unroll
-            for (int nt = 0; nt < 2; ++nt)
-              mma_3xtf32(t[nt], a, lval(mb, j, 8 * kk + tig, 8 * nt + gid), lval(mb, j, 8 * kk + tig + 4, 8 * nt + gid));
+            mma_3xtf32(t[kk], a, lval(mb, j, 8 * kk + tig, 8 * nt + gid), lval(mb, j, 8 * kk + tig + 4, 8 * nt + gid));
           }
         }
-#pragma unroll
-        for (int nt = 0; nt < 2; ++nt) {
-          tw[gid * 17 + 8 * nt + 2 * tig] = t[nt][0];
-          tw[gid * 17 + 8 * nt + 2 * tig + 1] = t[nt][1];
-          tw[(gid + 8) * 17 + 8 * nt + 2 * tig] = t[nt][2];
-          tw[(gid + 8) * 17 + 8 * nt + 2 * tig + 1] = t[nt][3];
-        }
+        tw[gid * 9 + 2 * tig] = t[0][0] + t[1][0];
+        tw[gid * 9 + 2 * tig + 1] = t[0][1] + t[1][1];
+        tw[(gid + 8) * 9 + 2 * tig] = t[0][2] + t[1][2];
+        tw[(gid + 8) * 9 + 2 * tig + 1] = t[0][3] + t[1][3];
         __syncwarp();
-        float l[2][4];
-#pragma unroll
-        for (int nt = 0; nt < 2; ++nt) l[nt][0] = l[nt][1] = l[nt][2] = l[nt][3] = 0.0f;
+        float l[2][4] = {{0.0f, 0.0f, 0.0f, 0.0f}, {0.0f, 0.0f, 0.0f, 0.0f}};
 #pragma unroll
         for (int kk = 0; kk < 2; ++kk) {
           const float a[4] = {lval(i, i, gid, 8 * kk + tig), lval(i, i, gid + 8, 8 * kk + tig),
                               lval(i, i, gid, 8 * kk + tig + 4), lval(i, i, gid + 8, 8 * kk + tig + 4)};
-#pragma unroll
-          for (int nt = 0; nt < 2; ++nt)
-            mma_3xtf32(l[nt], a, tw[(8 * kk + tig) * 17 + 8 * nt + gid], tw[(8 * kk + tig + 4) * 17 + 8 * nt + gid]);
+          mma_3xtf32(l[kk], a, tw[(8 * kk + tig) * 9 + gid], tw[(8 * kk + tig + 4) * 9 + gid]);
         }
         // L_ij, negated, into the transposed copy: L[16i + r][16j + c] at al[16j + c][16i + r]
 #pragma unroll
-        for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int r = gid + (e >= 2 ? 8 : 0), c = 8 * nt + 2 * tig + (e & 1);
-            s.al[(16 * j + c) * LD64 + 16 * i + r] = -l[nt][e];
-          }
+        for (int e = 0; e < 4; ++e) {
+          const int r = gid + (e >= 2 ? 8 : 0), c = 8 * nt + 2 * tig + (e & 1);
+          s.al[(16 * j + c) * LD64 + 16 * i + r] = -(l[0][e] + l[1][e]);
+        }
       }
       __syncthreads();
     }
@@ -584,6 +594,7 @@ __global__ void __launch_bounds__(kThreads, 2) gdn_prep_kernel(const __grid_cons
 }
 
 constexpr int kBufs = 3;  // record buffers of the state pass
+constexpr int kAhead = kBufs - 1;  // chunks whose records are requested ahead
 // floats of one record buffer of the state pass: [M^T; R] (128 rows), then
 // this CTA's 32 rows of N and of Y^T
 constexpr int kRecCta = (128 + 2 * kRows) * 64;
@@ -621,8 +632,8 @@ __device__ __forceinline__ void store_out(const GdnArgs& a, const float* os, int
 
 // One CTA per (value head, 32 state rows): the chunks in order, one block
 // barrier per chunk.  Chunk c's record (the shared [M^T; R] and this CTA's rows
-// of N and Y^T, three bulk copies) lands in buffer c % 3, requested two chunks
-// ahead; its output goes out from the staging buffer during chunk c + 1.
+// of N and Y^T, three bulk copies) lands in buffer c % kBufs, requested kAhead
+// chunks ahead; its output goes out from the staging buffer during chunk c + 1.
 // Fragments come from shared memory with ldmatrix: the records and the state
 // rows are swizzled (sw64), so the loads are free of bank conflicts.
 __global__ void __launch_bounds__(kThreads, 1) gdn_state_kernel(const __grid_constant__ GdnArgs a) {
@@ -651,8 +662,7 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_state_kernel(const __grid_con
     bulk_load(s.rec[b] + (128 + kRows) * 64, rec + 256 * 64 + i0 * 64, kRows * 64 * 4, &s.full[b]);
   };
   if (tid == 0) {
-    if (a.nchunks > 0) issue(0);
-    if (a.nchunks > 1) issue(1);
+    for (int cc = 0; cc < kAhead && cc < a.nchunks; ++cc) issue(cc);
   }
   // entering state, as the TF32 operand it is used as
   for (int idx = tid; idx < kRows * DK; idx += kThreads) {
@@ -671,8 +681,8 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_state_kernel(const __grid_con
     const int buf = c % kBufs;
     const bool ok = mbar_wait_bounded(&s.full[buf], static_cast<uint32_t>(c / kBufs) & 1u, abort_flag);
     if (__syncthreads_or(!ok)) break;  // a copy did not arrive in time: every thread stops
-    // buffer (c + 2) % 3 was last read during chunk c - 1
-    if (tid == 0 && c + 2 < a.nchunks) issue(c + 2);
+    // buffer (c + kAhead) % kBufs was last read during chunk c - 1
+    if (tid == 0 && c + kAhead < a.nchunks) issue(c + kAhead);
     if (c > 0) store_out(a, s.os[(c - 1) & 1], c - 1, h, i0, tid);
     const float* bc = s.rec[buf];
     const float* nn = bc + 128 * 64;
@@ -750,7 +760,7 @@ __global__ void __launch_bounds__(kThreads, 1) gdn_state_kernel(const __grid_con
     // a record copy did not arrive in time (the error word is set): wait, with
     // a limit, for the copies still in flight into this CTA's buffers, then stop
     if (tid == 0)
-      for (int cc = c; cc < a.nchunks && cc < c + 2; ++cc)
+      for (int cc = c; cc < a.nchunks && cc < c + kAhead; ++cc)
         mbar_wait_bounded(&s.full[cc % kBufs], static_cast<uint32_t>(cc / kBufs) & 1u, nullptr);
     return;
   }
