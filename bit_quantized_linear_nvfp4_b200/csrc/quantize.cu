@@ -408,16 +408,20 @@ __global__ void __launch_bounds__(kThreads, 1) quant_kernel(const __grid_constan
 }
 
 // Small inputs with a device-computed scale, in one launch: a cluster of C
-// blocks (C <= 8) of 8 warps.  Each block takes the amax of its share of x
-// with register loads, reads the other blocks' maxima through distributed
-// shared memory after a cluster barrier, and quantises its share, reading x
-// again (it is a few hundred KB at most, and still in L2).  No shared-memory
-// staging: the blocks need a few KB of shared memory and 256 threads, so
-// they can run beside the weight-streaming GEMM's CTAs of the layer before.
+// blocks (C <= 8) of 8 warps, as many as give each warp about one chunk (a
+// decode token's row of 17408 elements is 34 chunks: 5 blocks).  Each block
+// takes the amax of its share of x with register loads (up to kSmallUnroll
+// chunks in flight per warp), reads the other blocks' maxima through
+// distributed shared memory after a cluster barrier, and quantises its share,
+// reading x again (it is a few hundred KB at most, and still in L2).  No
+// shared-memory staging: the blocks need a few KB of shared memory and 256
+// threads, so they can run beside the weight-streaming GEMM's CTAs of the
+// layer before.
 constexpr int kSmallWarps = 8;
 constexpr int kSmallThreads = kSmallWarps * 32;
-constexpr int kSmallChunksPerBlock = 64;  // 8 chunks per warp
+constexpr int kSmallChunksPerBlock = 64;  // the path takes up to 8 blocks of 64 chunks
 constexpr int kMaxSmallBlocks = 8;
+constexpr int kSmallUnroll = 4;
 
 template <int DTYPE, bool WIDE>
 __global__ void __launch_bounds__(kSmallThreads, 1) small_kernel(const __grid_constant__ QuantArgs a) {
@@ -432,15 +436,26 @@ __global__ void __launch_bounds__(kSmallThreads, 1) small_kernel(const __grid_co
   int64_t lo, hi;
   block_range(a.items, lo, hi);
   SegMax sm;
-  for (int64_t i = lo + warp; i < hi; i += kSmallWarps) {
-    int32_t row, col;
-    chunk_pos(a, i, row, col);
-    col += lane * 16;
-    if (col < a.K) {
-      Blk<DTYPE> b;
-      load_global<DTYPE, WIDE>(a.x + row * a.ld_bytes + static_cast<int64_t>(col) * C::kEsz, b);
-      sm.add(find_segment(a, row), block_amax<DTYPE>(b));
+  for (int64_t base = lo + warp; base < hi; base += kSmallWarps * kSmallUnroll) {
+    Blk<DTYPE> b[kSmallUnroll];
+    int32_t rows[kSmallUnroll];
+    bool act[kSmallUnroll];
+#pragma unroll
+    for (int u = 0; u < kSmallUnroll; ++u) {  // every load before the first use
+      const int64_t i = base + u * kSmallWarps;
+      int32_t col = 0;
+      rows[u] = 0;
+      act[u] = false;
+      if (i < hi) {
+        chunk_pos(a, i, rows[u], col);
+        col += lane * 16;
+        act[u] = col < a.K;
+        if (act[u]) load_global<DTYPE, WIDE>(a.x + rows[u] * a.ld_bytes + static_cast<int64_t>(col) * C::kEsz, b[u]);
+      }
     }
+#pragma unroll
+    for (int u = 0; u < kSmallUnroll; ++u)
+      if (act[u]) sm.add(find_segment(a, rows[u]), block_amax<DTYPE>(b[u]));
   }
   // block maxima per segment: warp-reduce, then warp s combines segment s
 #pragma unroll
@@ -467,14 +482,27 @@ __global__ void __launch_bounds__(kSmallThreads, 1) small_kernel(const __grid_co
   }
   __syncthreads();
   if (blockIdx.x == 0 && threadIdx.x < a.nseg) a.g_out[threadIdx.x] = g_sh[threadIdx.x];
-  for (int64_t i = lo + warp; i < hi; i += kSmallWarps) {
-    int32_t row, col;
-    chunk_pos(a, i, row, col);
-    col += lane * 16;
-    Blk<DTYPE> b;
-    const bool have = col < a.K;
-    if (have) load_global<DTYPE, WIDE>(a.x + row * a.ld_bytes + static_cast<int64_t>(col) * C::kEsz, b);
-    quantize_block<DTYPE>(a, g_sh, b, have, row, col);
+  for (int64_t base = lo + warp; base < hi; base += kSmallWarps * kSmallUnroll) {
+    Blk<DTYPE> b[kSmallUnroll];
+    int32_t rows[kSmallUnroll], cols[kSmallUnroll];
+    bool inr[kSmallUnroll], have[kSmallUnroll];
+#pragma unroll
+    for (int u = 0; u < kSmallUnroll; ++u) {  // every load before the first use
+      const int64_t i = base + u * kSmallWarps;
+      inr[u] = i < hi;
+      have[u] = false;
+      rows[u] = cols[u] = 0;
+      if (inr[u]) {
+        chunk_pos(a, i, rows[u], cols[u]);
+        cols[u] += lane * 16;
+        have[u] = cols[u] < a.K;
+        if (have[u])
+          load_global<DTYPE, WIDE>(a.x + rows[u] * a.ld_bytes + static_cast<int64_t>(cols[u]) * C::kEsz, b[u]);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kSmallUnroll; ++u)
+      if (inr[u]) quantize_block<DTYPE>(a, g_sh, b[u], have[u], rows[u], cols[u]);  // uniform across the warp
   }
   zero_padding_rows_n(a, kSmallWarps);
   cluster_sync_all();  // no block leaves while another may read its maxima
@@ -619,7 +647,10 @@ template <int DTYPE, bool WIDE>
 cudaError_t launch_t(QuantArgs a, bool dynamic, cudaStream_t stream) {
   const int64_t nsmall = (a.items + kSmallChunksPerBlock - 1) / kSmallChunksPerBlock;
   if (dynamic && nsmall <= kMaxSmallBlocks) {
-    const int blocks = nsmall < 1 ? 1 : static_cast<int>(nsmall);
+    // about one chunk per warp, up to kMaxSmallBlocks blocks
+    int64_t nb = (a.items + kSmallWarps - 1) / kSmallWarps;
+    if (nb > kMaxSmallBlocks) nb = kMaxSmallBlocks;
+    const int blocks = nb < 1 ? 1 : static_cast<int>(nb);
     return launch_pdl(small_kernel<DTYPE, WIDE>, blocks, blocks, 0, a, stream, kSmallThreads);
   }
   const int grid = grid_for(a.items);
