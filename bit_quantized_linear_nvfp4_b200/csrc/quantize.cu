@@ -409,7 +409,10 @@ __global__ void __launch_bounds__(kThreads, 1) quant_kernel(const __grid_constan
 
 // Small inputs with a device-computed scale, in one launch: a cluster of C
 // blocks (C <= 8) of 8 warps, as many as give each warp about one chunk (a
-// decode token's row of 17408 elements is 34 chunks: 5 blocks).  Each block
+// decode token's row of 17408 elements is 34 chunks: 5 blocks).  (Eight
+// blocks of 32 warps for up to 2560 chunks were slower than the two-launch
+// path at 64 decode tokens, 17.8 against 6.3 us: eight SMs stream the input
+// twice.)  Each block
 // takes the amax of its share of x with register loads (up to kSmallUnroll
 // chunks in flight per warp), reads the other blocks' maxima through
 // distributed shared memory after a cluster barrier, and quantises its share,

@@ -40,7 +40,10 @@ def test_tiny_workload_activation_and_weight():
 
 
 @pytest.mark.parametrize("dtype", ["bf16", "f32"])
-@pytest.mark.parametrize("M,K", [(1, 16), (3, 48), (127, 256), (129, 272), (300, 512), (64, 5120), (5, 17408)])
+@pytest.mark.parametrize("M,K", [(1, 16), (3, 48), (127, 256), (129, 272), (300, 512), (64, 5120), (5, 17408),
+                                 # chunks of 512 elements: the one-launch path's limit (512), one row
+                                 # past it, and 64 decode tokens (two launches)
+                                 (16, 16384), (17, 16384), (64, 17408)])
 def test_ragged_shapes(dtype, M, K):
     x = _rand(M, K, M * 7 + K, dtype, outliers=min(3, K // 16))
     op, g = nv.nvfp4_quantize(_dev(x, dtype))

@@ -8,9 +8,10 @@ through the C ABI (ctypes, no Python wrapper) and checks that its codes, scale
 bytes and global scale equal those of nvfp4_quantize bit for bit (the
 tolerance the quantiser tests use), on calls in a row.
 
-The first two inputs are larger than what the one-launch cluster path takes
-(about 1.6 MB of BF16), so both go through the two launches that pass the
-per-block maxima through the static scratch.  The first has a large amax
+The first two inputs (8192 and 4096 chunks of 512 elements) are larger than
+what the one-launch cluster path takes (512 chunks, 512 KB of BF16), so both
+go through the two launches that pass the per-block maxima through the static
+scratch.  The first has a large amax
 (x40) and fills the scratch with large maxima; the second, FP32 with a much
 smaller amax (x0.01) and fewer rows (so fewer amax blocks), would show any
 scratch word left over from the first call as a wrong global scale.  Two
