@@ -137,6 +137,22 @@ def dist_init(world, backend=None):
     return dist
 
 
+def tensor_peak(peaks: dict, chain_ms: float, clock_reasons) -> tuple:
+    """The dense-FP4 roofline denominator (TFLOP/s) and its regime: a measured
+    BF16 figure times the nominal FP4/BF16 ratio, the burst figure for a
+    short chain of launches, the sustained one when the chain lasts a second
+    or more or the sampled clocks show the power cap (a kernel timed inside a
+    long run)."""
+    sustained = chain_ms >= 1000.0 or "sw_power_cap" in (clock_reasons or [])
+    key = "bf16_tflops_sustained" if sustained else "bf16_tflops"
+    return float(peaks[key]) * FP4_PER_BF16, ("sustained" if sustained else "burst")
+
+
+def e2e_choice(ms_pipelined: float, ms_serial: float) -> tuple:
+    """The faster of the two end-to-end forms: (ms per step, mode)."""
+    return (ms_pipelined, "pipelined") if ms_pipelined <= ms_serial else (ms_serial, "serial")
+
+
 def dist_max(dist, value: float, device) -> float:
     """Max over ranks (device-timed milliseconds)."""
     if dist is None:
@@ -463,13 +479,11 @@ def run_product(args):
         # reported beside it.
         fp4_burst = float(peaks["bf16_tflops"]) * FP4_PER_BF16
         fp4_sustained = float(peaks["bf16_tflops_sustained"]) * FP4_PER_BF16
-        sustained = gb2b_ms * K >= 1000.0 or "sw_power_cap" in (clk.get("reasons") or [])
-        fp4_peak = fp4_sustained if sustained else fp4_burst
+        fp4_peak, regime = tensor_peak(peaks, gb2b_ms * K, clk.get("reasons"))
         ach = step.flops / (gb2b_ms * 1e-3) / 1e12
         roof = {"bound": "tensor", "achieved": ach, "peak": fp4_peak, "unit": "TFLOP/s",
                 "frac": ach / fp4_peak, "traffic": TRAFFIC_BYTES.get(args.workload),
-                "peak_source": f"{peak_src} {'sustained' if sustained else 'burst'} bf16 x {FP4_PER_BF16:g} "
-                               "(nominal dense FP4/BF16)",
+                "peak_source": f"{peak_src} {regime} bf16 x {FP4_PER_BF16:g} (nominal dense FP4/BF16)",
                 "kernel": "nvfp4 gemm (tcgen05 mxf4nvf4)", "ms_per_launch": gb2b_ms,
                 "ms_per_isolated_launch": g_ms, "frac_of_nominal_9pf": ach / NOMINAL_FP4_TFLOPS,
                 "frac_of_burst_bf16_x4": ach / fp4_burst, "frac_of_sustained_bf16_x4": ach / fp4_sustained,
@@ -623,8 +637,7 @@ def measure_e2e(step, K, Wm, stream):
     unit = "TFLOP/s" if step.w is not None else "GB/s"
     # the faster of the two forms is the value (for a few tokens the three
     # streams' host-side bookkeeping costs more than the overlap saves)
-    mode = "pipelined" if ms <= ms_serial else "serial"
-    best = min(ms, ms_serial)
+    best, mode = e2e_choice(ms, ms_serial)
     return {"value": rate(best), "unit": unit, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
             "ms_per_step": best, "call": "nvfp4_linear" if step.w is not None else "nvfp4_quantize",
             "mode": mode,
